@@ -1,0 +1,25 @@
+import os
+import sys
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+
+def pytest_configure(config):
+    config.addinivalue_line("markers", "gpu: needs a CUDA device (B200, sm_100a)")
+
+
+@pytest.fixture(scope="session")
+def codebooks():
+    """Oracle Lloyd-Max codebooks, built once per session and cached by (d, bits)."""
+    from oracle.codebook import lloyd_max
+    cache = {}
+
+    def get(d, bits):
+        if (d, bits) not in cache:
+            cache[(d, bits)] = lloyd_max(d, bits)
+        return cache[(d, bits)]
+    return get
