@@ -1,0 +1,518 @@
+// Host side of the C ABI: handles, RPBH planning, the Lloyd-Max codebook,
+// argument checks, per-device tables and the device status word.
+//
+// Sources: "OrbitQuant: Data-Agnostic Quantization for Image and Video
+// Diffusion Transformers" ([OQ]) -- Methodology (RPBH, offline weight and
+// online activation quantization), Theoretical Basis (f_d, codebook, q_hat);
+// "TurboQuant: Online Vector Quantization with Near-optimal Distortion Rate"
+// ([TQ]) slides 14-16 (sphere marginal, continuous k-means).
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <new>
+#include <string>
+
+#include "oq_internal.h"
+
+namespace oq {
+
+static thread_local std::string g_last_error;
+
+int fail(int code, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  g_last_error = buf;
+  return code;
+}
+
+void clear_error() { g_last_error.clear(); }
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// SplitMix64 (Steele, Lea & Flood 2014): state += golden gamma, then a
+// bijective 64-bit mix of the new state.
+uint64_t splitmix64_next(uint64_t& state) {
+  state += 0x9E3779B97F4A7C15ull;
+  uint64_t z = state;
+  z = (z ^ (z >> 30)) * 0xBF58476D1CE4E5B9ull;
+  z = (z ^ (z >> 27)) * 0x94D049BB133111EBull;
+  return z ^ (z >> 31);
+}
+
+// ---------------------------------------------------------------------------
+// Lloyd-Max for f_d.  Integrals of t^p f_d(t) dt are taken in theta = asin t,
+// where f_d(t) dt = C cos(theta)^(d-2) dtheta (smooth for d >= 3), on equal
+// panels of width <= 0.25/sqrt(d-2) over |theta| <= min(pi/2, 40/sqrt(d-2)),
+// each panel (or part of one) by 16-point Gauss-Legendre.
+// ---------------------------------------------------------------------------
+namespace {
+
+constexpr int kGL = 16;
+
+void gauss_legendre(int n, double* x, double* w) {
+  // Newton iteration on P_n from the usual cosine initial guesses.
+  for (int i = 0; i < n; ++i) {
+    double z = std::cos(M_PI * (i + 0.75) / (n + 0.5));
+    double dp = 1.0;
+    for (int it = 0; it < 100; ++it) {
+      double p0 = 1.0, p1 = z;
+      for (int k = 2; k <= n; ++k) {
+        double p2 = ((2.0 * k - 1.0) * z * p1 - (k - 1.0) * p0) / k;
+        p0 = p1;
+        p1 = p2;
+      }
+      dp = n * (z * p1 - p0) / (z * z - 1.0);
+      double dz = p1 / dp;
+      z -= dz;
+      if (std::fabs(dz) < 1e-16) break;
+    }
+    double p0 = 1.0, p1 = z;
+    for (int k = 2; k <= n; ++k) {
+      double p2 = ((2.0 * k - 1.0) * z * p1 - (k - 1.0) * p0) / k;
+      p0 = p1;
+      p1 = p2;
+    }
+    dp = n * (z * p1 - p0) / (z * z - 1.0);
+    x[i] = z;
+    w[i] = 2.0 / ((1.0 - z * z) * dp * dp);
+  }
+}
+
+struct ThetaIntegrator {
+  int d;
+  double logC, tmax, width;
+  int npan;
+  double gx[kGL], gw[kGL];
+  std::vector<double> panel[3];
+
+  explicit ThetaIntegrator(int d_) : d(d_) {
+    logC = std::lgamma(d / 2.0) - 0.5 * std::log(M_PI) - std::lgamma((d - 1) / 2.0);
+    tmax = std::fmin(M_PI / 2.0, 40.0 / std::sqrt(d - 2.0));
+    double wmax = 0.25 / std::sqrt(d - 2.0);
+    int per_side = (int)std::ceil(tmax / wmax);
+    if (per_side < 1) per_side = 1;
+    npan = 2 * per_side;
+    width = 2.0 * tmax / npan;
+    gauss_legendre(kGL, gx, gw);
+    for (int p = 0; p < 3; ++p) {
+      panel[p].resize(npan);
+      for (int q = 0; q < npan; ++q) panel[p][q] = gl(edge(q), edge(q + 1), p);
+    }
+  }
+  double edge(int q) const { return q == npan ? tmax : -tmax + q * width; }
+  double gl(double a, double b, int p) const {
+    double half = 0.5 * (b - a), mid = 0.5 * (b + a), s = 0.0;
+    for (int i = 0; i < kGL; ++i) {
+      double th = mid + half * gx[i];
+      double c = std::cos(th);
+      double f = c > 0.0 ? std::exp(logC + (d - 2) * std::log(c)) : 0.0;
+      double sn = std::sin(th);
+      double g = p == 0 ? 1.0 : (p == 1 ? sn : sn * sn);
+      s += gw[i] * f * g;
+    }
+    return half * s;
+  }
+  double to_theta(double t) const {
+    double th = std::asin(std::fmax(-1.0, std::fmin(1.0, t)));
+    return std::fmax(-tmax, std::fmin(tmax, th));
+  }
+  int panel_of(double th) const {
+    int q = (int)std::floor((th + tmax) / width);
+    return q < 0 ? 0 : (q >= npan ? npan - 1 : q);
+  }
+  // int_{ta}^{tb} t^p f_d(t) dt
+  double cell(double ta, double tb, int p) const {
+    double a = to_theta(ta), b = to_theta(tb);
+    int pa = panel_of(a), pb = panel_of(b);
+    if (pa == pb) return gl(a, b, p);
+    long double s = gl(a, edge(pa + 1), p);
+    for (int q = pa + 1; q < pb; ++q) s += panel[p][q];
+    s += gl(edge(pb), b, p);
+    return (double)s;
+  }
+};
+
+}  // namespace
+
+void lloyd_max(int d, int bits, std::vector<double>& c, std::vector<double>& beta, int& iterations,
+               double& distortion) {
+  const int L = 1 << bits;
+  ThetaIntegrator integ(d);
+  const double sd = std::sqrt((double)d);
+  const double a = std::fmin(3.0 / sd, 0.9);
+  c.resize(L);
+  for (int k = 0; k < L; ++k) c[k] = L == 1 ? 0.0 : -a + 2.0 * a * k / (L - 1);
+  std::vector<double> e(L + 1), cn(L);
+  const double tol = 1e-13;
+  const int max_iters = 200000;
+  int it = 0;
+  for (it = 1; it <= max_iters; ++it) {
+    e[0] = -1.0;
+    e[L] = 1.0;
+    for (int k = 1; k < L; ++k) e[k] = 0.5 * (c[k - 1] + c[k]);  // nearest-neighbour condition
+    double delta = 0.0;
+    for (int k = 0; k < L; ++k) {                                  // centroid condition
+      double m0 = integ.cell(e[k], e[k + 1], 0);
+      double m1 = integ.cell(e[k], e[k + 1], 1);
+      cn[k] = m1 / m0;
+      delta = std::fmax(delta, std::fabs(cn[k] - c[k]));
+    }
+    c.swap(cn);
+    if (delta * sd < tol) break;
+  }
+  if (it > max_iters) it = max_iters;
+  iterations = it;
+  // exact antisymmetry: the optimum for the symmetric f_d is symmetric
+  for (int k = 0; k < L / 2; ++k) {
+    double v = 0.5 * (c[L - 1 - k] - c[k]);
+    c[L - 1 - k] = v;
+    c[k] = -v;
+  }
+  beta.resize(L - 1);
+  for (int k = 0; k + 1 < L; ++k) beta[k] = 0.5 * (c[k] + c[k + 1]);
+  double dist = 0.0;
+  for (int k = 0; k < L; ++k) {
+    double lo = k == 0 ? -1.0 : beta[k - 1], hi = k == L - 1 ? 1.0 : beta[k];
+    double m0 = integ.cell(lo, hi, 0), m1 = integ.cell(lo, hi, 1), m2 = integ.cell(lo, hi, 2);
+    dist += m2 - 2.0 * c[k] * m1 + c[k] * c[k] * m0;
+  }
+  distortion = dist;
+}
+
+// IEEE binary16 bits of v rounded to nearest, ties to even (finite |v| < 65520).
+uint16_t double_to_fp16_rne(double v) {
+  uint16_t sign = std::signbit(v) ? 0x8000 : 0;
+  double a = std::fabs(v);
+  if (a == 0.0) return sign;
+  int e;
+  double m = std::frexp(a, &e);  // a = m 2^e, 0.5 <= m < 1
+  if (e - 1 < -14) {             // subnormal: multiples of 2^-24
+    double q = std::nearbyint(a * 16777216.0);
+    return (uint16_t)(sign | (uint16_t)q);  // q == 1024 becomes the smallest normal
+  }
+  double q = std::nearbyint(m * 2048.0);  // 11 significant bits
+  if (q >= 2048.0) {
+    q *= 0.5;
+    e += 1;
+  }
+  int exp_field = e - 1 + 15;
+  if (exp_field >= 31) return (uint16_t)(sign | 0x7C00);
+  return (uint16_t)(sign | (exp_field << 10) | ((uint16_t)q & 0x3FF));
+}
+
+// ---------------------------------------------------------------------------
+// Device state
+// ---------------------------------------------------------------------------
+static std::mutex g_dev_mu;
+static int* g_status[OQ_MAX_DEVICES] = {};
+static int g_sms[OQ_MAX_DEVICES] = {};
+
+int current_device(int* dev) {
+  cudaError_t e = cudaGetDevice(dev);
+  if (e != cudaSuccess) return fail(OQ_ERR_CUDA, "cudaGetDevice: %s", cudaGetErrorString(e));
+  if (*dev < 0 || *dev >= OQ_MAX_DEVICES) return fail(OQ_ERR_UNSUPPORTED, "device index %d too large", *dev);
+  return OQ_OK;
+}
+
+int device_status_word(int** status) {
+  int dev;
+  if (int rc = current_device(&dev)) return rc;
+  std::lock_guard<std::mutex> lk(g_dev_mu);
+  if (!g_status[dev]) {
+    int* p = nullptr;
+    cudaError_t e = cudaMalloc(&p, sizeof(int));
+    if (e != cudaSuccess) return fail(OQ_ERR_CUDA, "cudaMalloc(status): %s", cudaGetErrorString(e));
+    e = cudaMemset(p, 0, sizeof(int));
+    if (e != cudaSuccess) return fail(OQ_ERR_CUDA, "cudaMemset(status): %s", cudaGetErrorString(e));
+    g_status[dev] = p;
+  }
+  *status = g_status[dev];
+  return OQ_OK;
+}
+
+int sm_count(int* n) {
+  int dev;
+  if (int rc = current_device(&dev)) return rc;
+  std::lock_guard<std::mutex> lk(g_dev_mu);
+  if (!g_sms[dev]) {
+    int v = 0;
+    cudaError_t e = cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess) return fail(OQ_ERR_CUDA, "cudaDeviceGetAttribute: %s", cudaGetErrorString(e));
+    g_sms[dev] = v;
+  }
+  *n = g_sms[dev];
+  return OQ_OK;
+}
+
+static int upload_rpbh(oq_rpbh_t r, int dev) {
+  std::vector<uint16_t> p16(r->d);
+  for (int j = 0; j < r->d; ++j) p16[j] = (uint16_t)r->perm[j];
+  uint16_t* dp = nullptr;
+  uint32_t* ds = nullptr;
+  cudaError_t e = cudaMalloc(&dp, sizeof(uint16_t) * r->d);
+  if (e == cudaSuccess) e = cudaMalloc(&ds, sizeof(uint32_t) * r->sign_bits.size());
+  if (e == cudaSuccess) e = cudaMemcpy(dp, p16.data(), sizeof(uint16_t) * r->d, cudaMemcpyHostToDevice);
+  if (e == cudaSuccess)
+    e = cudaMemcpy(ds, r->sign_bits.data(), sizeof(uint32_t) * r->sign_bits.size(), cudaMemcpyHostToDevice);
+  if (e != cudaSuccess) {
+    cudaFree(dp);
+    cudaFree(ds);
+    return fail(OQ_ERR_CUDA, "uploading RPBH tables: %s", cudaGetErrorString(e));
+  }
+  r->dev_perm[dev] = dp;
+  r->dev_signs[dev] = ds;
+  return OQ_OK;
+}
+
+int rpbh_device_tables(oq_rpbh_t r, const uint16_t** perm, const uint32_t** signs) {
+  int dev;
+  if (int rc = current_device(&dev)) return rc;
+  std::lock_guard<std::mutex> lk(r->mu);
+  if (!r->dev_perm[dev]) {
+    if (int rc = upload_rpbh(r, dev)) return rc;
+  }
+  *perm = r->dev_perm[dev];
+  *signs = r->dev_signs[dev];
+  return OQ_OK;
+}
+
+}  // namespace oq
+
+// ===========================================================================
+// C ABI
+// ===========================================================================
+using namespace oq;
+
+extern "C" {
+
+int oq_version(void) { return OQ_VERSION; }
+
+const char* oq_last_error(void) { return g_last_error.c_str(); }
+
+int oq_get_device_status(void* stream) {
+  clear_error();
+  cudaError_t e = cudaStreamSynchronize((cudaStream_t)stream);
+  if (e != cudaSuccess) return fail(OQ_ERR_CUDA, "cudaStreamSynchronize: %s", cudaGetErrorString(e));
+  int* st;
+  if (int rc = device_status_word(&st)) return rc;
+  int v = 0;
+  e = cudaMemcpy(&v, st, sizeof(int), cudaMemcpyDeviceToHost);
+  if (e == cudaSuccess) e = cudaMemset(st, 0, sizeof(int));
+  if (e != cudaSuccess) return fail(OQ_ERR_CUDA, "reading device status: %s", cudaGetErrorString(e));
+  if (v != OQ_OK) return fail(v, "a kernel reported device status %d (bounded wait gave up)", v);
+  return OQ_OK;
+}
+
+int oq_make_rpbh(uint64_t seed, int d, int block, oq_rpbh_t* out) {
+  clear_error();
+  if (!out) return fail(OQ_ERR_ARG, "out is NULL");
+  *out = nullptr;
+  if (d < 1) return fail(OQ_ERR_ARG, "d must be >= 1 (got %d)", d);
+  int h = block == 0 ? (d & -d) : block;
+  if (h < 1 || (h & (h - 1)) != 0 || d % h != 0)
+    return fail(OQ_ERR_ARG, "block %d must be a power of two dividing d=%d", block, d);
+  oq_rpbh_t r = new (std::nothrow) oq_rpbh_s;
+  if (!r) return fail(OQ_ERR_NOMEM, "allocating the RPBH handle");
+  r->seed = seed;
+  r->d = d;
+  r->h = h;
+  r->perm.resize(d);
+  for (int j = 0; j < d; ++j) r->perm[j] = j;
+  uint64_t st = seed;
+  for (int i = d - 1; i >= 1; --i) {  // Fisher-Yates
+    uint64_t j = splitmix64_next(st) % (uint64_t)(i + 1);
+    int32_t tmp = r->perm[i];
+    r->perm[i] = r->perm[j];
+    r->perm[j] = tmp;
+  }
+  r->sign_bits.assign((d + 31) / 32, 0u);
+  for (int j = 0; j < d; ++j)
+    if (splitmix64_next(st) >> 63) r->sign_bits[j >> 5] |= 1u << (j & 31);
+  // Upload to the current device now when one is present; otherwise lazily.
+  int ndev = 0;
+  if (cudaGetDeviceCount(&ndev) == cudaSuccess && ndev > 0 && d <= 65536) {
+    int dev;
+    if (cudaGetDevice(&dev) == cudaSuccess && dev < OQ_MAX_DEVICES) {
+      if (int rc = upload_rpbh(r, dev)) {
+        delete r;
+        return rc;
+      }
+    }
+  } else {
+    cudaGetLastError();  // no device here: clear the sticky "no device" error
+  }
+  *out = r;
+  return OQ_OK;
+}
+
+int oq_rpbh_info(oq_rpbh_t r, int* d, int* block) {
+  clear_error();
+  if (!r) return fail(OQ_ERR_ARG, "NULL rpbh handle");
+  if (d) *d = r->d;
+  if (block) *block = r->h;
+  return OQ_OK;
+}
+
+int oq_rpbh_export(oq_rpbh_t r, int32_t* perm, uint32_t* sign_bits) {
+  clear_error();
+  if (!r) return fail(OQ_ERR_ARG, "NULL rpbh handle");
+  if (perm) std::memcpy(perm, r->perm.data(), sizeof(int32_t) * r->d);
+  if (sign_bits) std::memcpy(sign_bits, r->sign_bits.data(), sizeof(uint32_t) * r->sign_bits.size());
+  return OQ_OK;
+}
+
+void oq_free_rpbh(oq_rpbh_t r) {
+  if (!r) return;
+  int prev = -1;
+  bool have_prev = cudaGetDevice(&prev) == cudaSuccess;
+  for (int dev = 0; dev < OQ_MAX_DEVICES; ++dev) {
+    if (!r->dev_perm[dev] && !r->dev_signs[dev]) continue;
+    if (cudaSetDevice(dev) == cudaSuccess) {
+      cudaFree(r->dev_perm[dev]);
+      cudaFree(r->dev_signs[dev]);
+    }
+  }
+  if (have_prev) cudaSetDevice(prev);
+  delete r;
+}
+
+int oq_build_codebook(int d, int bits, oq_codebook_t* out) {
+  clear_error();
+  if (!out) return fail(OQ_ERR_ARG, "out is NULL");
+  *out = nullptr;
+  if (d < 3) return fail(OQ_ERR_ARG, "d must be >= 3 (got %d)", d);
+  if (bits < 1 || bits > 8) return fail(OQ_ERR_ARG, "bits must be in 1..8 (got %d)", bits);
+  oq_codebook_t cb = new (std::nothrow) oq_codebook_s;
+  if (!cb) return fail(OQ_ERR_NOMEM, "allocating the codebook handle");
+  cb->d = d;
+  cb->bits = bits;
+  lloyd_max(d, bits, cb->centroids, cb->bounds, cb->iterations, cb->distortion);
+  cb->lut.resize(cb->centroids.size());
+  const double sd = std::sqrt((double)d);
+  for (size_t k = 0; k < cb->centroids.size(); ++k) cb->lut[k] = double_to_fp16_rne(sd * cb->centroids[k]);
+  *out = cb;
+  return OQ_OK;
+}
+
+int oq_codebook_info(oq_codebook_t cb, int* d, int* bits) {
+  clear_error();
+  if (!cb) return fail(OQ_ERR_ARG, "NULL codebook handle");
+  if (d) *d = cb->d;
+  if (bits) *bits = cb->bits;
+  return OQ_OK;
+}
+
+int oq_codebook_export(oq_codebook_t cb, double* centroids, double* bounds, uint16_t* lut_fp16, int* iterations,
+                       double* distortion) {
+  clear_error();
+  if (!cb) return fail(OQ_ERR_ARG, "NULL codebook handle");
+  if (centroids) std::memcpy(centroids, cb->centroids.data(), sizeof(double) * cb->centroids.size());
+  if (bounds) std::memcpy(bounds, cb->bounds.data(), sizeof(double) * cb->bounds.size());
+  if (lut_fp16) std::memcpy(lut_fp16, cb->lut.data(), sizeof(uint16_t) * cb->lut.size());
+  if (iterations) *iterations = cb->iterations;
+  if (distortion) *distortion = cb->distortion;
+  return OQ_OK;
+}
+
+void oq_free_codebook(oq_codebook_t cb) { delete cb; }
+
+static int check_quant_args(oq_rpbh_t r, oq_codebook_t cb, const void* X, int M, const void* codes,
+                            const void* norms) {
+  if (!r || !cb) return fail(OQ_ERR_ARG, "NULL handle");
+  if (M < 0) return fail(OQ_ERR_ARG, "M must be >= 0 (got %d)", M);
+  if (r->d != cb->d) return fail(OQ_ERR_ARG, "rpbh d=%d and codebook d=%d differ", r->d, cb->d);
+  if (r->d % 32 != 0 || r->d > 16384)
+    return fail(OQ_ERR_UNSUPPORTED, "kernels need d %% 32 == 0 and d <= 16384 (d=%d)", r->d);
+  if (r->h < 32 || r->h > 1024) return fail(OQ_ERR_UNSUPPORTED, "kernels need 32 <= block <= 1024 (h=%d)", r->h);
+  if (cb->bits > 6) return fail(OQ_ERR_UNSUPPORTED, "kernels need bits <= 6 (bits=%d)", cb->bits);
+  if (M == 0) return OQ_OK;
+  if (!X || !codes || !norms) return fail(OQ_ERR_ARG, "NULL buffer");
+  if (!aligned16(X) || !aligned16(codes) || !aligned16(norms))
+    return fail(OQ_ERR_ALIGN, "X, codes and norms must be 16-byte aligned");
+  return OQ_OK;
+}
+
+int oq_quantize_act(oq_rpbh_t r, oq_codebook_t cb, const void* X, int M, uint8_t* codes, float* norms,
+                    void* stream) {
+  clear_error();
+  if (int rc = check_quant_args(r, cb, X, M, codes, norms)) return rc;
+  if (M == 0) return OQ_OK;
+  return launch_rotq(r, cb, X, M, codes, norms, nullptr, stream);
+}
+
+int oq_quantize_weight(oq_rpbh_t r, oq_codebook_t cb, const void* W, int N, uint8_t* codes, void* norms_bf16,
+                       void* stream) {
+  clear_error();
+  if (int rc = check_quant_args(r, cb, W, N, codes, norms_bf16)) return rc;
+  if (N == 0) return OQ_OK;
+  return launch_rotq(r, cb, W, N, codes, nullptr, (uint16_t*)norms_bf16, stream);
+}
+
+size_t oq_linear_workspace_bytes(int M, int d, int bits_a) {
+  if (M <= 0 || d <= 0 || bits_a <= 0) return 0;
+  size_t code_bytes = ((size_t)M * (size_t)d * (size_t)bits_a + 7) / 8;
+  code_bytes = (code_bytes + 255) & ~(size_t)255;
+  return code_bytes + 4 * (size_t)M;
+}
+
+static int check_linear_args(int d, oq_codebook_t cb_a, oq_codebook_t cb_w, int M, const void* w_codes,
+                             const void* w_norm, int N, const void* bias, int epilogue, const void* Y_f32,
+                             const void* Y_bf16) {
+  if (!cb_a || !cb_w) return fail(OQ_ERR_ARG, "NULL codebook handle");
+  if (cb_a->d != d || cb_w->d != d)
+    return fail(OQ_ERR_ARG, "codebook dims (%d, %d) must equal d=%d", cb_a->d, cb_w->d, d);
+  if (M < 0 || N < 0) return fail(OQ_ERR_ARG, "M and N must be >= 0");
+  if (epilogue != OQ_EPI_NONE && epilogue != OQ_EPI_GELU) return fail(OQ_ERR_ARG, "unknown epilogue %d", epilogue);
+  if (d % 64 != 0) return fail(OQ_ERR_UNSUPPORTED, "the GEMM needs d %% 64 == 0 (d=%d)", d);
+  if (N % 16 != 0) return fail(OQ_ERR_UNSUPPORTED, "the GEMM needs N %% 16 == 0 (N=%d)", N);
+  auto ok_bits = [](int b) { return b == 2 || b == 4 || b == 6; };
+  if (!ok_bits(cb_a->bits) || !ok_bits(cb_w->bits))
+    return fail(OQ_ERR_UNSUPPORTED, "the GEMM needs bits in {2,4,6} (a=%d, w=%d)", cb_a->bits, cb_w->bits);
+  if (!Y_f32 && !Y_bf16) return fail(OQ_ERR_ARG, "at least one of Y_f32 / Y_bf16 is needed");
+  if (M == 0 || N == 0) return OQ_OK;
+  if (!w_codes || !w_norm) return fail(OQ_ERR_ARG, "NULL weight buffer");
+  if (!aligned16(w_codes) || !aligned16(w_norm) || (bias && !aligned16(bias)) || (Y_f32 && !aligned16(Y_f32)) ||
+      (Y_bf16 && !aligned16(Y_bf16)))
+    return fail(OQ_ERR_ALIGN, "GEMM buffers must be 16-byte aligned");
+  return OQ_OK;
+}
+
+int oq_linear_codes(int d, oq_codebook_t cb_a, oq_codebook_t cb_w, const uint8_t* a_codes, const float* a_norm,
+                    int M, const uint8_t* w_codes, const void* w_norm, int N, const void* bias, int epilogue,
+                    float* Y_f32, void* Y_bf16, void* stream) {
+  clear_error();
+  if (int rc = check_linear_args(d, cb_a, cb_w, M, w_codes, w_norm, N, bias, epilogue, Y_f32, Y_bf16)) return rc;
+  if (M == 0 || N == 0) return OQ_OK;
+  if (!a_codes || !a_norm) return fail(OQ_ERR_ARG, "NULL activation buffer");
+  if (!aligned16(a_codes) || !aligned16(a_norm)) return fail(OQ_ERR_ALIGN, "activation buffers must be 16-byte aligned");
+  return launch_cbgemm(d, cb_a, cb_w, a_codes, a_norm, M, w_codes, (const uint16_t*)w_norm, N,
+                       (const uint16_t*)bias, epilogue, Y_f32, (uint16_t*)Y_bf16, stream);
+}
+
+int oq_linear(oq_rpbh_t r, oq_codebook_t cb_a, oq_codebook_t cb_w, const void* X, int M, const uint8_t* w_codes,
+              const void* w_norm, int N, const void* bias, int epilogue, float* Y_f32, void* Y_bf16,
+              void* workspace, size_t workspace_bytes, void* stream) {
+  clear_error();
+  if (!r) return fail(OQ_ERR_ARG, "NULL rpbh handle");
+  if (int rc = check_linear_args(r->d, cb_a, cb_w, M, w_codes, w_norm, N, bias, epilogue, Y_f32, Y_bf16)) return rc;
+  if (M == 0 || N == 0) return OQ_OK;
+  size_t need = oq_linear_workspace_bytes(M, r->d, cb_a->bits);
+  if (!workspace || workspace_bytes < need)
+    return fail(OQ_ERR_ARG, "workspace of %zu bytes is smaller than the %zu needed", workspace_bytes, need);
+  if (!aligned16(workspace)) return fail(OQ_ERR_ALIGN, "workspace must be 16-byte aligned");
+  uint8_t* a_codes = (uint8_t*)workspace;
+  size_t code_bytes = need - 4 * (size_t)M;
+  float* a_norm = (float*)((uint8_t*)workspace + code_bytes);
+  if (int rc = check_quant_args(r, cb_a, X, M, a_codes, a_norm)) return rc;
+  if (int rc = launch_rotq(r, cb_a, X, M, a_codes, a_norm, nullptr, stream)) return rc;
+  return launch_cbgemm(r->d, cb_a, cb_w, a_codes, a_norm, M, w_codes, (const uint16_t*)w_norm, N,
+                       (const uint16_t*)bias, epilogue, Y_f32, (uint16_t*)Y_bf16, stream);
+}
+
+}  // extern "C"

@@ -1,0 +1,59 @@
+// Internal declarations shared by the library's translation units only.
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+#include <mutex>
+#include <vector>
+
+#include "../../include/orbitquant.h"
+
+#define OQ_MAX_DEVICES 64
+#define OQ_VERSION 100
+
+struct oq_rpbh_s {
+  uint64_t seed = 0;
+  int d = 0, h = 0;
+  std::vector<int32_t> perm;        // pi, (P x)_j = x_{pi(j)}
+  std::vector<uint32_t> sign_bits;  // bit j%32 of word j/32 set <=> sign_j = -1
+  std::mutex mu;
+  uint16_t* dev_perm[OQ_MAX_DEVICES] = {};   // pi as uint16 [d]
+  uint32_t* dev_signs[OQ_MAX_DEVICES] = {};  // sign words [d/32]
+};
+
+struct oq_codebook_s {
+  int d = 0, bits = 0;
+  std::vector<double> centroids;  // 2^b ascending, exactly antisymmetric
+  std::vector<double> bounds;     // 2^b - 1 midpoints
+  std::vector<uint16_t> lut;      // fp16 bits of RNE(sqrt(d) c_k)
+  int iterations = 0;
+  double distortion = 0.0;
+};
+
+namespace oq {
+
+// Error reporting: store a message for oq_last_error() and return `code`.
+int fail(int code, const char* fmt, ...);
+void clear_error();
+
+// Host planning (oq_host.cpp).
+uint64_t splitmix64_next(uint64_t& state);
+void lloyd_max(int d, int bits, std::vector<double>& centroids, std::vector<double>& bounds, int& iterations,
+               double& distortion);
+uint16_t double_to_fp16_rne(double v);
+
+// Device-side state (oq_host.cpp).
+int current_device(int* dev);
+int rpbh_device_tables(oq_rpbh_t r, const uint16_t** perm, const uint32_t** signs);
+int device_status_word(int** status);
+int sm_count(int* n);
+bool aligned16(const void* p);
+
+// Kernel launchers.
+int launch_rotq(oq_rpbh_t r, oq_codebook_t cb, const void* X, int M, uint8_t* codes, float* norm_f32,
+                uint16_t* norm_bf16, void* stream);
+int launch_cbgemm(int d, oq_codebook_t cb_a, oq_codebook_t cb_w, const uint8_t* a_codes, const float* a_norm, int M,
+                  const uint8_t* w_codes, const uint16_t* w_norm, int N, const uint16_t* bias, int epilogue,
+                  float* Y_f32, uint16_t* Y_bf16, void* stream);
+
+}  // namespace oq

@@ -1,0 +1,190 @@
+/*
+ * orbitquant.h -- C ABI of the B200 (sm_100a) OrbitQuant hot path.
+ *
+ * OrbitQuant quantizes both operands of a linear layer in one shared rotated,
+ * normalised basis: activations are rotated online by the randomized
+ * permuted block-Hadamard (RPBH) transform, split into norm and direction,
+ * and the direction is coded against a data-free Lloyd-Max codebook; weights
+ * went through the same steps offline; the layer multiplies the codes and
+ * rescales by both norms.  Sources are cited by page title and section:
+ *
+ *   [OQ]  "OrbitQuant: Data-Agnostic Quantization for Image and Video
+ *          Diffusion Transformers" -- the method.
+ *   [TQ]  "TurboQuant: Online Vector Quantization with Near-optimal
+ *          Distortion Rate" (slide deck) -- f_d and Lloyd-Max origins.
+ *
+ * Conventions for every entry point
+ *   - Return value: OQ_OK (0) or one of the OQ_ERR_* codes below.  Argument
+ *     errors are detected on the host before anything is launched, and
+ *     oq_last_error() then returns a message (thread-local).
+ *   - Device buffers are plain device pointers owned by the caller; they must
+ *     be 16-byte aligned (OQ_ERR_ALIGN otherwise).  No entry point frees or
+ *     keeps a caller buffer.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *     stream).  Kernel launches are asynchronous on that stream.
+ *   - Handles (oq_rpbh_t, oq_codebook_t) are created on the host and own
+ *     small device tables.  Tables are uploaded to the current device when
+ *     the handle is created (if a device is present) and lazily, once, to any
+ *     other device the handle is used on; that lazy first use allocates and
+ *     copies synchronously, so make it outside any stream capture.
+ *   - Device-side failures (a bounded wait in a kernel that gave up) are
+ *     recorded in a per-device status word; read and clear it with
+ *     oq_get_device_status().
+ *   - Layouts: bf16 tensors are row-major uint16 bit patterns.  Packed codes
+ *     of a row form a little-endian bit stream, code i in bits [i*b, (i+1)*b)
+ *     (4 bits: element 2j in the low nibble of byte j; 6 bits: four codes in
+ *     three bytes); each row is d*b/8 bytes.
+ */
+#ifndef ORBITQUANT_H
+#define ORBITQUANT_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define OQ_API __attribute__((visibility("default")))
+#else
+#define OQ_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+enum {
+  OQ_OK = 0,
+  OQ_ERR_ARG = 1,          /* null handle/pointer, bad size, mismatched handles */
+  OQ_ERR_UNSUPPORTED = 2,  /* valid for the method but not for these kernels */
+  OQ_ERR_ALIGN = 3,        /* a device pointer is not 16-byte aligned */
+  OQ_ERR_CUDA = 4,         /* a CUDA runtime call failed (message has the name) */
+  OQ_ERR_TIMEOUT = 5,      /* a kernel's bounded wait gave up (device status) */
+  OQ_ERR_NOMEM = 6         /* host or device allocation of a handle table failed */
+};
+
+enum { OQ_EPI_NONE = 0, OQ_EPI_GELU = 1 };
+
+typedef struct oq_rpbh_s* oq_rpbh_t;
+typedef struct oq_codebook_s* oq_codebook_t;
+
+/* Version of this ABI (major*100 + minor). */
+OQ_API int oq_version(void);
+
+/* Message for the last error returned on this host thread ("" if none). */
+OQ_API const char* oq_last_error(void);
+
+/* Reads and clears the device status word of the current device after
+ * synchronising `stream`.  Returns OQ_OK, OQ_ERR_TIMEOUT, or OQ_ERR_CUDA. */
+OQ_API int oq_get_device_status(void* stream);
+
+/* ---------------------------------------------------------------------------
+ * RPBH rotation  Pi_d = blkdiag(H_h D_1, ..., H_h D_{d/h}) P_pi
+ * [OQ] Methodology, "Randomized Permuted Block-Hadamard (RPBH) Rotation".
+ *
+ * seed  : the fixed random draw ("drawn once per dimension").  SplitMix64
+ *         with state = seed; pi by Fisher-Yates (i = d-1..1,
+ *         j = next() mod (i+1), swap), then d signs: sign_j = -1 when the top
+ *         bit of next() is set.
+ * d     : dimension, >= 1.  The kernels need d % 32 == 0 and d <= 16384.
+ * block : h, a power of two dividing d; 0 picks the page's rule (largest
+ *         power of two dividing d).  The kernels support 32 <= h <= 1024.
+ * H_h is the Sylvester-order Walsh-Hadamard matrix scaled by 1/sqrt(h), so
+ * Pi_d is orthogonal; (P x)_j = x_{pi(j)}; the signs act before H.
+ * Errors: OQ_ERR_ARG (d < 1, bad block, null out), OQ_ERR_NOMEM.
+ * ------------------------------------------------------------------------- */
+OQ_API int oq_make_rpbh(uint64_t seed, int d, int block, oq_rpbh_t* out);
+
+/* d and h of a handle.  Either output may be NULL. */
+OQ_API int oq_rpbh_info(oq_rpbh_t r, int* d, int* block);
+
+/* Copies pi (int32[d], host) and the sign bits (uint32[ceil(d/32)], host;
+ * bit j%32 of word j/32 set <=> sign_j = -1).  Either output may be NULL. */
+OQ_API int oq_rpbh_export(oq_rpbh_t r, int32_t* perm, uint32_t* sign_bits);
+
+OQ_API void oq_free_rpbh(oq_rpbh_t r);
+
+/* ---------------------------------------------------------------------------
+ * Lloyd-Max codebook C^(d,b) for the sphere marginal
+ *   f_d(t) = Gamma(d/2) / (sqrt(pi) Gamma((d-1)/2)) (1 - t^2)^((d-3)/2)
+ * [OQ] "Theoretical Basis" (f_d, codebook, q_hat) and "Data-Agnostic
+ * Codebook"; [TQ] slides 14-16.  Built on the host with no data: Lloyd
+ * iteration (midpoint boundaries, conditional-mean centroids) from
+ * linspace(-a, a, 2^b), a = min(3/sqrt(d), 0.9), integrals by composite
+ * Gauss-Legendre in theta = asin(t); stops when max|delta c| sqrt(d) < 1e-13
+ * or after 200000 iterations; centroids then made exactly antisymmetric.
+ * d >= 3, 1 <= bits <= 8 (kernels: bits <= 6).
+ * ------------------------------------------------------------------------- */
+OQ_API int oq_build_codebook(int d, int bits, oq_codebook_t* out);
+
+/* d and bits of a handle.  Either output may be NULL. */
+OQ_API int oq_codebook_info(oq_codebook_t cb, int* d, int* bits);
+
+/* Copies (host) centroids double[2^b] ascending, bounds double[2^b-1]
+ * (midpoints), the dequantisation table lut_fp16 uint16[2^b] = fp16 bits of
+ * round-to-nearest-even(sqrt(d) * c_k), the Lloyd iteration count and the
+ * per-coordinate distortion int (t - q(t))^2 f_d.  Any output may be NULL. */
+OQ_API int oq_codebook_export(oq_codebook_t cb, double* centroids, double* bounds, uint16_t* lut_fp16,
+                       int* iterations, double* distortion);
+
+OQ_API void oq_free_codebook(oq_codebook_t cb);
+
+/* ---------------------------------------------------------------------------
+ * Online activation quantization  ([OQ] "Online Activation Quantization")
+ *   x' = Pi_d x ;  s = ||x'||_2 ;  codes = q_hat(x' / (s + eps)),  eps = 1e-12
+ * q_hat(t) = argmin_c |t - c| over C^(d,b); a t exactly on a boundary takes
+ * the lower centroid.
+ * X     : device bf16 [M][d] (row-major, rows contiguous).
+ * codes : device uint8 [M][d*b/8], packed as described at the top.
+ * norms : device float [M], s per row (the norm of x' equals that of x).
+ * M >= 0 (M == 0 launches nothing).  d must match both handles.
+ * ------------------------------------------------------------------------- */
+OQ_API int oq_quantize_act(oq_rpbh_t r, oq_codebook_t cb, const void* X, int M, uint8_t* codes, float* norms,
+                    void* stream);
+
+/* ---------------------------------------------------------------------------
+ * Offline weight quantization  ([OQ] "Offline Weight Quantization")
+ *   w' = Pi_d w ;  r' = ||w'||_2 ;  codes = q_hat(w' / (r' + eps))
+ * r' is stored in bf16 (round to nearest even), step 4 of that section.
+ * W     : device bf16 [N][d]; codes: device uint8 [N][d*b/8];
+ * norms_bf16 : device bf16 [N].
+ * ------------------------------------------------------------------------- */
+OQ_API int oq_quantize_weight(oq_rpbh_t r, oq_codebook_t cb, const void* W, int N, uint8_t* codes, void* norms_bf16,
+                       void* stream);
+
+/* ---------------------------------------------------------------------------
+ * Codebook linear on codes  ([OQ] "Online Activation Quantization", last
+ * paragraph: W^' x^' ~= W Pi^T Pi x = W x, no inverse rotation)
+ *   y[m][n] = s_m r'_n sum_k v_a[ca[m][k]] v_w[cw[n][k]]  (+ bias_n) (-> GELU)
+ * with v = lut_fp16 / sqrt(d) of each codebook.  Accumulation is fp32 on the
+ * tensor cores (fp16 x fp16 products).
+ * d           : common inner dimension; cb_a and cb_w must both have it.
+ * a_codes     : device uint8 [M][d*ba/8];  a_norm : device float [M].
+ * w_codes     : device uint8 [N][d*bw/8];  w_norm : device bf16 [N].
+ * bias        : device bf16 [N] or NULL.
+ * epilogue    : OQ_EPI_NONE or OQ_EPI_GELU (exact erf form).
+ * Y_f32       : device float [M][N] or NULL; Y_bf16: device bf16 [M][N] or
+ *               NULL (at least one).  Row stride N elements.
+ * Needs d % 64 == 0, N % 16 == 0, bits in {2, 4, 6} for both operands.
+ * ------------------------------------------------------------------------- */
+OQ_API int oq_linear_codes(int d, oq_codebook_t cb_a, oq_codebook_t cb_w, const uint8_t* a_codes, const float* a_norm,
+                    int M, const uint8_t* w_codes, const void* w_norm, int N, const void* bias, int epilogue,
+                    float* Y_f32, void* Y_bf16, void* stream);
+
+/* Bytes of workspace oq_linear needs for M rows: the activation codes
+ * (M*d*bits_a/8, rounded up to 256) plus the norms (4*M). */
+OQ_API size_t oq_linear_workspace_bytes(int M, int d, int bits_a);
+
+/* ---------------------------------------------------------------------------
+ * Full layer: oq_quantize_act of X into `workspace`, then oq_linear_codes.
+ * X : device bf16 [M][d].  workspace: device, >= oq_linear_workspace_bytes.
+ * The rotation handle must be the one the weights were quantized with (the
+ * shared rotation that cancels in the product).
+ * ------------------------------------------------------------------------- */
+OQ_API int oq_linear(oq_rpbh_t r, oq_codebook_t cb_a, oq_codebook_t cb_w, const void* X, int M, const uint8_t* w_codes,
+              const void* w_norm, int N, const void* bias, int epilogue, float* Y_f32, void* Y_bf16,
+              void* workspace, size_t workspace_bytes, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* ORBITQUANT_H */

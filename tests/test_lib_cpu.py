@@ -1,0 +1,108 @@
+"""C-ABI library on the CPU: it loads, exports every declared symbol, and its
+host planning (RPBH draw, Lloyd-Max codebook, fp16 table, argument checks)
+agrees with the oracle.  No kernel is launched here."""
+
+import ctypes
+import math
+import os
+import re
+
+import numpy as np
+import pytest
+
+from oracle import codebook as ocb
+from oracle import rpbh as orpbh
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def oq():
+    from calibration_free_rotated_b200 import build
+    build.build()
+    from calibration_free_rotated_b200 import orbitquant
+    return orbitquant
+
+
+def _declared_symbols():
+    src = open(os.path.join(ROOT, "include", "orbitquant.h")).read()
+    return sorted(set(re.findall(r"OQ_API\s+[\w\s\*]+?\b(oq_\w+)\s*\(", src)))
+
+
+def test_every_declared_symbol_is_exported(oq):
+    names = _declared_symbols()
+    assert len(names) >= 16
+    lib = oq.lib()
+    for n in names:
+        assert hasattr(lib, n), n
+
+
+def test_version_and_empty_error(oq):
+    assert oq.lib().oq_version() >= 100
+
+
+@pytest.mark.parametrize("seed,d,block", [(0, 256, 64), (0, 3072, 128), (7, 1536, 0), (123, 96, 32), (0, 8960, 128)])
+def test_rpbh_draw_matches_oracle(oq, seed, d, block):
+    r = oq.Rpbh(seed, d, block)
+    perm, signs = r.export()
+    operm, osigns = orpbh.draw_permutation_and_signs(seed, d)
+    assert np.array_equal(perm.astype(np.int64), operm)
+    bits = np.array([(signs[j >> 5] >> (j & 31)) & 1 for j in range(d)])
+    assert np.array_equal(bits == 1, osigns < 0)
+    assert r.block == (block or orpbh.default_block(d))
+
+
+@pytest.mark.parametrize("d,bits", [(3, 2), (64, 4), (256, 4), (3072, 4), (3072, 2), (3072, 6), (8960, 4),
+                                    (1536, 6), (12288, 4), (12288, 2)])
+def test_codebook_matches_oracle(oq, codebooks, d, bits):
+    lib_cb = oq.Codebook(d, bits).export()
+    ref = codebooks(d, bits)
+    sd = math.sqrt(d)
+    assert np.max(np.abs(lib_cb["centroids"] - ref["centroids"])) * sd < 1e-10
+    assert np.max(np.abs(lib_cb["boundaries"] - ref["boundaries"])) * sd < 1e-10
+    assert np.array_equal(lib_cb["centroids"], -lib_cb["centroids"][::-1])
+    assert abs(lib_cb["distortion"] / ref["distortion"] - 1) < 1e-9
+    # the declared fp16 table, bit for bit
+    lut = ocb.fp16_lut(ref["centroids"], d).view(np.uint16)
+    assert np.array_equal(lib_cb["lut_fp16"], lut)
+
+
+def test_argument_errors_without_gpu(oq):
+    lib = oq.lib()
+    h = ctypes.c_void_p()
+    assert lib.oq_make_rpbh(0, 0, 0, ctypes.byref(h)) == oq.OQ_ERR_ARG
+    assert lib.oq_make_rpbh(0, 96, 64, ctypes.byref(h)) == oq.OQ_ERR_ARG       # 64 does not divide 96
+    assert b"power of two" in lib.oq_last_error()
+    assert lib.oq_build_codebook(2, 4, ctypes.byref(h)) == oq.OQ_ERR_ARG
+    assert lib.oq_build_codebook(64, 9, ctypes.byref(h)) == oq.OQ_ERR_ARG
+    r = oq.Rpbh(0, 256, 64)
+    cb = oq.Codebook(256, 4)
+    cb8 = oq.Codebook(256, 8)
+    cb_other = oq.Codebook(512, 4)
+    # mismatched d, too many bits, NULL buffers: rejected before any launch
+    assert lib.oq_quantize_act(r.handle, cb_other.handle, None, 4, None, None, None) == oq.OQ_ERR_ARG
+    assert lib.oq_quantize_act(r.handle, cb8.handle, None, 4, None, None, None) == oq.OQ_ERR_UNSUPPORTED
+    assert lib.oq_quantize_act(r.handle, cb.handle, None, 4, None, None, None) == oq.OQ_ERR_ARG
+    assert lib.oq_quantize_act(r.handle, cb.handle, None, 0, None, None, None) == oq.OQ_OK  # M == 0: nothing
+    assert lib.oq_quantize_act(r.handle, cb.handle, ctypes.c_void_p(8), 4, ctypes.c_void_p(16),
+                               ctypes.c_void_p(16), None) == oq.OQ_ERR_ALIGN
+    r_small = oq.Rpbh(0, 48, 16)
+    cb48 = oq.Codebook(48, 4)
+    assert lib.oq_quantize_act(r_small.handle, cb48.handle, None, 4, None, None, None) == oq.OQ_ERR_UNSUPPORTED
+    # GEMM constraints
+    cb2 = oq.Codebook(256, 2)
+    cb3 = oq.Codebook(256, 3)
+    args = (None, None, 4, None, None, 32, None, 0, ctypes.c_void_p(16), None, None)
+    assert lib.oq_linear_codes(256, cb.handle, cb3.handle, *args) == oq.OQ_ERR_UNSUPPORTED
+    assert lib.oq_linear_codes(256, cb.handle, cb2.handle, None, None, 4, None, None, 30, None, 0,
+                               ctypes.c_void_p(16), None, None) == oq.OQ_ERR_UNSUPPORTED   # N % 16
+    assert lib.oq_linear_codes(256, cb.handle, cb2.handle, None, None, 4, None, None, 32, None, 7,
+                               ctypes.c_void_p(16), None, None) == oq.OQ_ERR_ARG           # epilogue
+    assert lib.oq_linear_codes(256, cb.handle, cb2.handle, None, None, 4, None, None, 32, None, 0,
+                               None, None, None) == oq.OQ_ERR_ARG                          # no output
+
+
+def test_workspace_bytes(oq):
+    assert oq.workspace_bytes(4608, 3072, 4) == 4608 * 3072 // 2 + 4 * 4608
+    assert oq.workspace_bytes(3, 64, 6) == 256 + 12
+    assert oq.workspace_bytes(0, 64, 4) == 0

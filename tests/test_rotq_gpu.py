@@ -1,0 +1,181 @@
+"""Parity of the rotate+quantize kernel (oq_quantize_act / oq_quantize_weight)
+against the fp64 oracle, through the C ABI.
+
+Rule (stated with the workload): codes are bit-exact except entries whose
+normalised rotated value t lies within 1e-5 of a decision boundary; those are
+counted and reported, and every mismatch must lie inside that band.  The
+oracle decides in fp64, the kernel in fp32, so the only disagreements are
+decisions within fp32 rounding of a boundary.  Norms: rel 1e-6 (fp32
+activations); bf16 weight norms exact or one bf16 ulp.
+"""
+
+import math
+
+import numpy as np
+import pytest
+import torch
+
+from calibration_free_rotated_b200 import inputs
+from oracle import quantize as oqz
+from oracle import rpbh as orpbh
+
+pytestmark = pytest.mark.gpu
+
+BAND = 1e-5
+
+
+@pytest.fixture(scope="module")
+def oq():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    from calibration_free_rotated_b200 import build
+    build.build()
+    from calibration_free_rotated_b200 import orbitquant
+    return orbitquant
+
+
+_handles = {}
+
+
+def _lib_handles(oq, seed, d, h, bits):
+    key = (seed, d, h, bits)
+    if key not in _handles:
+        _handles[key] = (oq.Rpbh(seed, d, h), oq.Codebook(d, bits))
+    return _handles[key]
+
+
+def _to_dev(bits_u16):
+    return torch.from_numpy(np.ascontiguousarray(bits_u16).view(np.int16)).cuda().view(torch.bfloat16)
+
+
+def _check_rows(oq, codebooks, X_bits, d, h, bits, seed=0, weight=False, rows=None, report=None):
+    """Runs the kernel on all of X_bits; checks rows `rows` (default all) against the oracle."""
+    r, cb = _lib_handles(oq, seed, d, h, bits)
+    X = _to_dev(X_bits)
+    if weight:
+        codes, norms = oq.quantize_weight(r, cb, X)
+    else:
+        codes, norms = oq.quantize_act(r, cb, X)
+    torch.cuda.synchronize()
+    oq.device_status()
+    rows = np.arange(X_bits.shape[0]) if rows is None else np.asarray(rows)
+    codes_np = codes.cpu().numpy()[rows]
+    if weight:
+        norms_np = norms.cpu().view(torch.int16).numpy().view(np.uint16)[rows]
+    else:
+        norms_np = norms.cpu().numpy()[rows]
+    perm, signs = orpbh.draw_permutation_and_signs(seed, d)
+    ref = codebooks(d, bits)
+    xs = inputs.bf16_bits_to_f64(X_bits[rows])
+    if weight:
+        ref_codes, r16, r_exact, T = oqz.quantize_weight_rows(xs, perm, signs, h, ref["centroids"])
+    else:
+        ref_codes, s, T = oqz.quantize_rows(xs, perm, signs, h, ref["centroids"])
+    got = oqz.unpack_codes(codes_np, bits, d)
+    mismatch = got != ref_codes
+    band = oqz.boundary_distance(T, ref["boundaries"]) < BAND
+    outside = mismatch & ~band
+    assert not np.any(outside), f"{int(outside.sum())} code mismatches outside the 1e-5 band"
+    if report is not None:
+        report.append((int(mismatch.sum()), int(band.sum()), mismatch.size))
+    if weight:
+        ref_bits = oqz.bf16_bits(r16)
+        diff = np.abs(norms_np.astype(np.int32) - ref_bits.astype(np.int32))
+        assert np.all(diff <= 1), "bf16 row norms differ by more than one ulp"
+    else:
+        rel = np.abs(norms_np - s) / np.maximum(s, 1e-30)
+        assert np.all((s == 0) == (norms_np == 0))
+        assert np.max(rel) < 1e-6
+    return got, mismatch
+
+
+@pytest.mark.parametrize("bits", [4, 2, 6])
+def test_single_linear_workload_act_and_weight(oq, codebooks, bits):
+    # X[64 x 256] with 3 outlier channels x20, W[256 x 256]; block 64, seed 0
+    X = inputs.activations(1, 64, 256)
+    W = inputs.weights(1, inputs.T_W, 256, 256)
+    _check_rows(oq, codebooks, X, 256, 64, bits)
+    _check_rows(oq, codebooks, W, 256, 64, bits, weight=True)
+
+
+@pytest.mark.parametrize("d,h", [(256, 64), (1536, 128), (3072, 128), (3072, 256), (8960, 128), (12288, 128),
+                                 (1024, 1024), (512, 32), (1536, 512)])
+@pytest.mark.parametrize("bits", [2, 4, 6])
+def test_sweep_shapes_with_ragged_tail(oq, codebooks, d, h, bits):
+    # several stages and CTAs, M not a multiple of the rows per stage, sparse tail rows
+    M = 300 if d >= 8192 else 1000
+    X = inputs.sweep_activations(M, d)
+    rep = []
+    _check_rows(oq, codebooks, X, d, h, bits, report=rep)
+    mism, inband, total = rep[0]
+    assert mism <= inband
+
+
+@pytest.mark.parametrize("bits", [1, 3, 5])
+def test_odd_bit_widths(oq, codebooks, bits):
+    X = inputs.sweep_activations(400, 1536)
+    _check_rows(oq, codebooks, X, 1536, 128, bits)
+
+
+def test_edge_rows(oq, codebooks):
+    d, h = 3072, 128
+    rng = np.random.default_rng(0)
+    x = rng.standard_normal((37, d))
+    x[0] = 0.0                                  # zero row
+    x[1] = 0.0
+    x[1, 5] = -3.0                              # one-hot
+    x[2] = 1.0                                  # constant row
+    x[3] *= 1e-18                               # tiny (squares still normal in fp32)
+    x[4] *= 1e15                                # large (squared norm still finite in fp32)
+    x[5, :] = 0.0
+    x[5, :2] = [1.0, 1.0]                       # two-hot
+    X = inputs.to_bf16_bits(x)
+    got, _ = _check_rows(oq, codebooks, X, d, h, 4)
+    assert np.all(got[0] == 7)                  # t = 0 takes the lower middle centroid
+    _check_rows(oq, codebooks, X[:1], d, h, 4)  # M = 1
+    _check_rows(oq, codebooks, X, d, h, 4, weight=True)
+
+
+def test_empty_batch(oq):
+    r, cb = _lib_handles(oq, 0, 256, 64, 4)
+    X = torch.empty((0, 256), dtype=torch.bfloat16, device="cuda")
+    codes, norms = oq.quantize_act(r, cb, X)
+    assert codes.shape == (0, 128)
+    oq.device_status()
+
+
+def test_deterministic(oq):
+    r, cb = _lib_handles(oq, 0, 3072, 128, 4)
+    X = _to_dev(inputs.activations(2, 4608, 3072, rows=(0, 777)))
+    c1, n1 = oq.quantize_act(r, cb, X)
+    c2, n2 = oq.quantize_act(r, cb, X)
+    assert torch.equal(c1, c2) and torch.equal(n1, n2)
+
+
+def test_flux_projection_full_size_sampled(oq, codebooks):
+    # X[4608 x 3072] (log-normal channel scales + 16 outlier channels x50), h = 128,
+    # all rows quantized in one launch, sampled rows checked
+    M, d = 4608, 3072
+    X = inputs.activations(2, M, d)
+    rows = np.linspace(0, M - 1, 48).astype(int)
+    _check_rows(oq, codebooks, X, d, 128, 4, rows=rows)
+    W = inputs.weights(2, inputs.T_W, 9216, d)
+    _check_rows(oq, codebooks, W, d, 128, 4, weight=True, rows=np.linspace(0, 9215, 32).astype(int))
+
+
+def test_wan_ffn_full_size_sampled(oq, codebooks):
+    # X[32760 x 1536] Student-t(3), 6-bit activations; fc2 input width 8960
+    M, d = 32760, 1536
+    X = inputs.activations(4, M, d)
+    rows = np.concatenate([np.linspace(0, M - 1, 40).astype(int), [M - 1]])
+    _check_rows(oq, codebooks, X, d, 128, 6, rows=rows)
+    W2 = inputs.weights(4, inputs.T_W2, 1536, 8960)
+    _check_rows(oq, codebooks, W2, 8960, 128, 4, weight=True, rows=np.linspace(0, 1535, 24).astype(int))
+
+
+def test_sweep_largest_full_size_sampled(oq, codebooks):
+    # 65536 x 12288 bf16 (1.6 GB), the largest sweep point; sparse tail included
+    M, d = 65536, 12288
+    X = inputs.sweep_activations(M, d)
+    rows = np.concatenate([np.linspace(0, M - 1, 24).astype(int), np.arange(M - 8, M)])
+    _check_rows(oq, codebooks, X, d, 256, 2, rows=rows)
