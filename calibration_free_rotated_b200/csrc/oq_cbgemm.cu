@@ -1,9 +1,610 @@
-// Kernel 2 placeholder: the codebook GEMM is added in its own change.
+// Kernel 2: codebook GEMM on packed codes with the norm-rescale epilogue.
+//
+// "OrbitQuant: Data-Agnostic Quantization for Image and Video Diffusion
+// Transformers", Methodology, "Online Activation Quantization" (last
+// paragraph): the shared rotation cancels in the product, so the layer is
+//   y[m][n] = s_m r'_n sum_k C_a[ca[m][k]] C_w[cw[n][k]]  (+ bias_n)
+// computed here as  acc = sum_k LUT_a[ca] LUT_w[cw]  (fp16 operands,
+// LUT = fp16(sqrt(d) c)), y = acc * s_m * r'_n / d + bias_n, optional GELU.
+//
+// sm_100a design (one CTA per SM, persistent over 128 x 256 output tiles):
+//   warp 12      TMA producer: 2-D tensor copies of the packed code tiles
+//                (A: 128 rows, B: 256 rows, 64 codes of K each) into a
+//                4-deep packed ring.
+//   warps 0..7   converters: expand codes through the fp16 LUT (register
+//                byte-permute tables for 2 and 4 bits, a 128-byte shared
+//                table for 6 bits) straight into the canonical K-major
+//                128-byte-swizzled UMMA layout of a 3-deep expanded ring.
+//   warp 13      one thread issues tcgen05.mma (kind::f16, M=128, N=256,
+//                K=16, fp32 accumulate in TMEM); tcgen05.commit frees ring
+//                stages and publishes finished accumulators.
+//   warps 8..11  epilogue: tcgen05.ld of the accumulator (each warp its
+//                32-lane quadrant), rescale, bias, GELU, fp32/bf16 stores.
+// TMEM holds two 128 x 256 fp32 accumulators (all 512 columns) so the
+// epilogue of one tile overlaps the main loop of the next.  Every mbarrier
+// wait is bounded (~1 s); a wait that gives up records OQ_ERR_TIMEOUT,
+// raises an abort flag that makes every role skip its remaining work, and
+// the CTA still reaches its teardown (TMEM is always released).
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cmath>
+#include <cstring>
+
 #include "oq_internal.h"
 
 namespace oq {
-int launch_cbgemm(int, oq_codebook_t, oq_codebook_t, const uint8_t*, const float*, int, const uint8_t*,
-                  const uint16_t*, int, const uint16_t*, int, float*, uint16_t*, void*) {
-  return fail(OQ_ERR_UNSUPPORTED, "codebook GEMM not built yet");
+namespace {
+
+constexpr int BM = 128, BN = 256, BK = 64;
+constexpr int PSTAGES = 4;
+constexpr int ESTAGES = 3;
+constexpr int NUM_CONV_WARPS = 8;
+constexpr int EPI_WARP0 = 8;
+constexpr int TMA_WARP = 12;
+constexpr int MMA_WARP = 13;
+constexpr int NUM_THREADS = 14 * 32;
+constexpr int TMEM_COLS = 512;
+constexpr unsigned long long kWaitLimitNs = 1000000000ull;
+
+constexpr int EXP_A_BYTES = BM * BK * 2;  // 16 KB
+constexpr int EXP_B_BYTES = BN * BK * 2;  // 32 KB
+
+struct GemmArgs {
+  const float* a_norm;
+  const uint16_t* w_norm;
+  const uint16_t* bias;
+  float* y32;
+  uint16_t* y16;
+  int* status;
+  int M, N, K;
+  int tiles_m, num_tiles;
+  int epilogue;
+  float inv_d;
+  uint32_t lut_a[32];  // 64 fp16 entries, two per word (entry 2i in the low half)
+  uint32_t lut_w[32];
+};
+
+template <int BITS>
+struct PackedTile {
+  static constexpr int kRowBytes = BK * BITS / 8;
+};
+
+// ---- shared memory plan (offsets from a 1024-aligned base) -------------------
+template <int BA, int BW>
+struct Smem {
+  static constexpr int kPkA = BM * PackedTile<BA>::kRowBytes;
+  static constexpr int kPkB = BN * PackedTile<BW>::kRowBytes;
+  static constexpr int kExpA = 0;
+  static constexpr int kExpB = kExpA + ESTAGES * EXP_A_BYTES;
+  static constexpr int kPackA = kExpB + ESTAGES * EXP_B_BYTES;
+  static constexpr int kPackB = kPackA + PSTAGES * ((kPkA + 127) / 128 * 128);
+  static constexpr int kLut = kPackB + PSTAGES * ((kPkB + 127) / 128 * 128);
+  static constexpr int kBars = kLut + 256;
+  // barriers: pk_full[P], pk_empty[P], ex_full[E], ex_empty[E], acc_full[2], acc_empty[2]
+  static constexpr int kNumBars = 2 * PSTAGES + 2 * ESTAGES + 4;
+  static constexpr int kMisc = kBars + kNumBars * 8;  // tmem base, abort flag
+  static constexpr int kTotal = kMisc + 16;
+  static constexpr int kAlloc = kTotal + 1024;  // room to align the base
+};
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
+
+__device__ __forceinline__ unsigned long long global_ns() {
+  unsigned long long t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Bounded wait; on give-up records the status, raises the CTA abort flag.
+__device__ bool wait_bounded(uint32_t bar, uint32_t parity, volatile int* abort_flag, int* status) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const unsigned long long t0 = global_ns();
+  while (true) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if (*abort_flag) return false;
+    if (global_ns() - t0 > kWaitLimitNs) {
+      atomicExch(status, OQ_ERR_TIMEOUT);
+      *abort_flag = 1;
+      return false;
+    }
+  }
+}
+
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
+}
+
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, int x, int y, uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::"r"(
+          dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar)
+      : "memory");
+}
+
+// UMMA shared-memory descriptor: K-major, 128-byte swizzle, 8-row groups 1024 B apart.
+__device__ __forceinline__ uint64_t umma_desc_sw128(uint32_t addr) {
+  uint64_t d = 0;
+  d |= (uint64_t)((addr & 0x3FFFFu) >> 4);
+  d |= (uint64_t)1 << 16;             // leading byte offset (unused for this layout)
+  d |= (uint64_t)(1024 >> 4) << 32;   // stride byte offset
+  d |= (uint64_t)1 << 46;             // descriptor version for sm_100
+  d |= (uint64_t)2 << 61;             // SWIZZLE_128B
+  return d;
+}
+
+// Instruction descriptor: D f32, A/B f16, both K-major, M = 128, N = 256.
+constexpr uint32_t kIdesc = (1u << 4) | (0u << 7) | (0u << 10) | ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
+
+__device__ __forceinline__ void umma_f16(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem_d),
+      "l"(adesc), "l"(bdesc), "r"(kIdesc), "r"(accumulate)
+      : "memory");
+}
+
+__device__ __forceinline__ void umma_commit(uint32_t bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar) : "memory");
+}
+
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
+  uint32_t d;
+  asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(sel));
+  return d;
+}
+
+// ---- code -> fp16 expansion ---------------------------------------------------
+// A 16-entry fp16 table as byte planes: lo[q] holds the low bytes of entries
+// 4q..4q+3, hi[q] the high bytes.
+struct Lut16 {
+  uint32_t lo[4], hi[4];
+};
+
+__device__ __forceinline__ Lut16 make_lut16(const uint32_t* words) {
+  Lut16 t;
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const uint32_t w0 = words[2 * q], w1 = words[2 * q + 1];  // entries 4q..4q+3
+    t.lo[q] = prmt(w0, w1, 0x6420);
+    t.hi[q] = prmt(w0, w1, 0x7531);
+  }
+  return t;
+}
+
+// Four 4-bit codes (x bits 0..15) -> two fp16x2 words.
+__device__ __forceinline__ void expand4_nib(uint32_t x, const Lut16& t, uint32_t& w0, uint32_t& w1) {
+  const uint32_t sel = x & 0x7777u;                         // entry within a group of 8
+  const uint32_t sel2 = ((x >> 1) & 0x4444u) | 0x3210u;     // which group (bit 3)
+  const uint32_t lo = prmt(prmt(t.lo[0], t.lo[1], sel), prmt(t.lo[2], t.lo[3], sel), sel2);
+  const uint32_t hi = prmt(prmt(t.hi[0], t.hi[1], sel), prmt(t.hi[2], t.hi[3], sel), sel2);
+  w0 = prmt(lo, hi, 0x5140);
+  w1 = prmt(lo, hi, 0x7362);
+}
+
+// Eight codes -> uint4 of eight fp16 (element 0 in the low half of .x).
+template <int BITS>
+__device__ __forceinline__ uint4 expand8(uint64_t packed, const Lut16& t16, uint32_t q0, uint32_t q1,
+                                         const uint16_t* lut_smem) {
+  uint4 r;
+  if constexpr (BITS == 4) {
+    const uint32_t w = (uint32_t)packed;
+    expand4_nib(w & 0xFFFFu, t16, r.x, r.y);
+    expand4_nib(w >> 16, t16, r.z, r.w);
+  } else if constexpr (BITS == 2) {
+    // selector bytes (2c0, 2c0+1, 2c1, 2c1+1) pick two fp16 from the 4-entry table {q1:q0}
+    const uint32_t w = (uint32_t)packed;
+    uint32_t o[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const uint32_t z = (w >> (4 * i)) & 0xFu;
+      const uint32_t sel = 0x1010u + (z & 3u) * 0x22u + (z & 0xCu) * 0x880u;
+      o[i] = prmt(q0, q1, sel);
+    }
+    r = make_uint4(o[0], o[1], o[2], o[3]);
+  } else {  // 6 bits: shared 64-entry table
+    uint32_t o[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const uint32_t c0 = (uint32_t)(packed >> (12 * i)) & 63u;
+      const uint32_t c1 = (uint32_t)(packed >> (12 * i + 6)) & 63u;
+      o[i] = (uint32_t)lut_smem[c0] | ((uint32_t)lut_smem[c1] << 16);
+    }
+    r = make_uint4(o[0], o[1], o[2], o[3]);
+  }
+  return r;
+}
+
+template <int BITS>
+__device__ __forceinline__ uint64_t load_chunk(const uint8_t* tile, int row, int c) {
+  constexpr int RB = PackedTile<BITS>::kRowBytes;
+  if constexpr (BITS == 4) {
+    return *reinterpret_cast<const uint32_t*>(tile + row * RB + 4 * c);
+  } else if constexpr (BITS == 2) {
+    return *reinterpret_cast<const uint16_t*>(tile + row * RB + 2 * c);
+  } else {
+    const int off = row * RB + 6 * c;
+    const int base = off & ~3;
+    const uint64_t lo = *reinterpret_cast<const uint32_t*>(tile + base);
+    const uint64_t hi = *reinterpret_cast<const uint32_t*>(tile + base + 4);
+    return ((hi << 32) | lo) >> (8 * (off - base));
+  }
+}
+
+// Offset of (row, 16-byte chunk c) in a K-major 128-byte-swizzled tile of 64 fp16 per row.
+__device__ __forceinline__ uint32_t sw128_offset(int row, int c) {
+  return (uint32_t)((row >> 3) * 1024 + (row & 7) * 128 + ((c ^ (row & 7)) << 4));
+}
+
+__device__ __forceinline__ float bf16_to_f32(uint16_t v) { return __uint_as_float((uint32_t)v << 16); }
+
+__device__ __forceinline__ uint16_t f32_to_bf16_rn(float f) {
+  uint32_t u = __float_as_uint(f);
+  if ((u & 0x7F800000u) == 0x7F800000u) return (uint16_t)((u >> 16) | ((u & 0xFFFFu) ? 0x40u : 0u));
+  u += 0x7FFFu + ((u >> 16) & 1u);
+  return (uint16_t)(u >> 16);
+}
+
+template <int BA, int BW>
+__global__ void __launch_bounds__(NUM_THREADS, 1)
+    cbgemm_kernel(const __grid_constant__ GemmArgs args, const __grid_constant__ CUtensorMap map_a,
+                  const __grid_constant__ CUtensorMap map_b) {
+  using S = Smem<BA, BW>;
+  extern __shared__ unsigned char smem_raw[];
+  unsigned char* smem = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+  const uint32_t sbase = smem_u32(smem);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S::kBars);
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + S::kMisc);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + S::kMisc + 4);
+  uint16_t* lut_a_s = reinterpret_cast<uint16_t*>(smem + S::kLut);
+  uint16_t* lut_w_s = lut_a_s + 64;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  auto bar = [&](int i) { return smem_u32(&bars[i]); };
+  const int PK_FULL = 0, PK_EMPTY = PSTAGES, EX_FULL = 2 * PSTAGES, EX_EMPTY = 2 * PSTAGES + ESTAGES,
+            ACC_FULL = 2 * PSTAGES + 2 * ESTAGES, ACC_EMPTY = ACC_FULL + 2;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < PSTAGES; ++s) {
+      mbar_init(bar(PK_FULL + s), 1);
+      mbar_init(bar(PK_EMPTY + s), NUM_CONV_WARPS);
+    }
+    for (int s = 0; s < ESTAGES; ++s) {
+      mbar_init(bar(EX_FULL + s), NUM_CONV_WARPS);
+      mbar_init(bar(EX_EMPTY + s), 1);
+    }
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(bar(ACC_FULL + s), 1);
+      mbar_init(bar(ACC_EMPTY + s), 4);
+    }
+    *abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (threadIdx.x < 64) {
+    lut_a_s[threadIdx.x] = (uint16_t)(args.lut_a[threadIdx.x >> 1] >> (16 * (threadIdx.x & 1)));
+    lut_w_s[threadIdx.x] = (uint16_t)(args.lut_w[threadIdx.x >> 1] >> (16 * (threadIdx.x & 1)));
+  }
+  if (warp == MMA_WARP) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_holder)),
+                 "r"(TMEM_COLS)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_holder;
+
+  const int KB = args.K / BK;
+  const int num_tiles = args.num_tiles;
+
+  if (warp == TMA_WARP) {
+    if (lane == 0) {
+      constexpr uint32_t bytes = S::kPkA + S::kPkB;
+      uint32_t pc = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
+        const int m0 = (t % args.tiles_m) * BM, n0 = (t / args.tiles_m) * BN;
+        for (int kb = 0; kb < KB; ++kb, ++pc) {
+          const int s = pc % PSTAGES;
+          const uint32_t ph = (pc / PSTAGES) & 1u;
+          if (!wait_bounded(bar(PK_EMPTY + s), ph ^ 1u, abort_flag, args.status)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(bar(PK_FULL + s), bytes);
+          tma_load_2d(sbase + S::kPackA + s * ((S::kPkA + 127) / 128 * 128), &map_a,
+                      kb * PackedTile<BA>::kRowBytes, m0, bar(PK_FULL + s));
+          tma_load_2d(sbase + S::kPackB + s * ((S::kPkB + 127) / 128 * 128), &map_b,
+                      kb * PackedTile<BW>::kRowBytes, n0, bar(PK_FULL + s));
+        }
+      }
+    }
+  } else if (warp < NUM_CONV_WARPS) {
+    // ---- converters ----
+    Lut16 ta, tw;
+    uint32_t qa0 = args.lut_a[0], qa1 = args.lut_a[1], qw0 = args.lut_w[0], qw1 = args.lut_w[1];
+    if constexpr (BA == 4) ta = make_lut16(args.lut_a);
+    if constexpr (BW == 4) tw = make_lut16(args.lut_w);
+    const int ct = threadIdx.x;  // 0..255
+    uint32_t pc = 0;
+    bool ok = true;
+    for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
+      for (int kb = 0; kb < KB; ++kb, ++pc) {
+        const int ps = pc % PSTAGES, es = pc % ESTAGES;
+        const uint32_t pph = (pc / PSTAGES) & 1u, eph = (pc / ESTAGES) & 1u;
+        if (!wait_bounded(bar(PK_FULL + ps), pph, abort_flag, args.status) ||
+            !wait_bounded(bar(EX_EMPTY + es), eph ^ 1u, abort_flag, args.status)) {
+          ok = false;
+          break;
+        }
+        const uint8_t* pa = smem + S::kPackA + ps * ((S::kPkA + 127) / 128 * 128);
+        const uint8_t* pb = smem + S::kPackB + ps * ((S::kPkB + 127) / 128 * 128);
+        unsigned char* ea = smem + S::kExpA + es * EXP_A_BYTES;
+        unsigned char* eb = smem + S::kExpB + es * EXP_B_BYTES;
+#pragma unroll
+        for (int i = 0; i < (BM * 8) / (NUM_CONV_WARPS * 32); ++i) {
+          const int ci = ct + i * NUM_CONV_WARPS * 32;
+          const int row = ci >> 3, c = ci & 7;
+          const uint4 v = expand8<BA>(load_chunk<BA>(pa, row, c), ta, qa0, qa1, lut_a_s);
+          *reinterpret_cast<uint4*>(ea + sw128_offset(row, c)) = v;
+        }
+#pragma unroll
+        for (int i = 0; i < (BN * 8) / (NUM_CONV_WARPS * 32); ++i) {
+          const int ci = ct + i * NUM_CONV_WARPS * 32;
+          const int row = ci >> 3, c = ci & 7;
+          const uint4 v = expand8<BW>(load_chunk<BW>(pb, row, c), tw, qw0, qw1, lut_w_s);
+          *reinterpret_cast<uint4*>(eb + sw128_offset(row, c)) = v;
+        }
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        __syncwarp();
+        if (lane == 0) {
+          mbar_arrive(bar(PK_EMPTY + ps));
+          mbar_arrive(bar(EX_FULL + es));
+        }
+      }
+    }
+  } else if (warp == MMA_WARP) {
+    if (lane == 0) {
+      uint32_t ec = 0, lt = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x, ++lt) {
+        const int acc = lt & 1;
+        const uint32_t aph = (lt >> 1) & 1u;
+        if (!wait_bounded(bar(ACC_EMPTY + acc), aph ^ 1u, abort_flag, args.status)) break;
+        tc_fence_after();
+        const uint32_t tmem_d = tmem_base + (uint32_t)(acc * BN);
+        for (int kb = 0; kb < KB; ++kb, ++ec) {
+          const int es = ec % ESTAGES;
+          const uint32_t eph = (ec / ESTAGES) & 1u;
+          if (!wait_bounded(bar(EX_FULL + es), eph, abort_flag, args.status)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a_addr = sbase + S::kExpA + es * EXP_A_BYTES;
+          const uint32_t b_addr = sbase + S::kExpB + es * EXP_B_BYTES;
+#pragma unroll
+          for (int k = 0; k < BK / 16; ++k) {
+            umma_f16(tmem_d, umma_desc_sw128(a_addr + 32 * k), umma_desc_sw128(b_addr + 32 * k),
+                     (kb > 0 || k > 0) ? 1u : 0u);
+          }
+          umma_commit(bar(EX_EMPTY + es));
+        }
+        if (!ok) break;
+        umma_commit(bar(ACC_FULL + acc));
+      }
+    }
+  } else if (warp >= EPI_WARP0 && warp < EPI_WARP0 + 4) {
+    // ---- epilogue ----
+    const int quad = warp & 3;  // TMEM lanes 32*quad .. 32*quad+31
+    uint32_t lt = 0;
+    for (int t = blockIdx.x; t < num_tiles; t += gridDim.x, ++lt) {
+      const int acc = lt & 1;
+      const uint32_t aph = (lt >> 1) & 1u;
+      const bool got = wait_bounded(bar(ACC_FULL + acc), aph, abort_flag, args.status);
+      __syncwarp();
+      if (__any_sync(0xFFFFFFFFu, !got)) break;
+      tc_fence_after();
+      const int m0 = (t % args.tiles_m) * BM, n0 = (t / args.tiles_m) * BN;
+      const int row = m0 + quad * 32 + lane;
+      const bool row_ok = row < args.M;
+      const float a_scale = row_ok ? args.a_norm[row] * args.inv_d : 0.0f;
+      const uint32_t taddr = tmem_base + ((uint32_t)(quad * 32) << 16) + (uint32_t)(acc * BN);
+#pragma unroll 1
+      for (int c0 = 0; c0 < BN; c0 += 32) {
+        uint32_t v[32];
+        __syncwarp();
+        asm volatile(
+            "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, "
+            "%14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+            : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7]),
+              "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]), "=r"(v[15]),
+              "=r"(v[16]), "=r"(v[17]), "=r"(v[18]), "=r"(v[19]), "=r"(v[20]), "=r"(v[21]), "=r"(v[22]),
+              "=r"(v[23]), "=r"(v[24]), "=r"(v[25]), "=r"(v[26]), "=r"(v[27]), "=r"(v[28]), "=r"(v[29]),
+              "=r"(v[30]), "=r"(v[31])
+            : "r"(taddr + (uint32_t)c0));
+        asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+        const int nb = n0 + c0;
+        if (row_ok && nb < args.N) {
+        float y[32];
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+          const int n = min(nb + j, args.N - 1);
+          float val = __uint_as_float(v[j]) * a_scale * bf16_to_f32(args.w_norm[n]);
+          if (args.bias) val += bf16_to_f32(args.bias[n]);
+          if (args.epilogue == OQ_EPI_GELU) val = 0.5f * val * (1.0f + erff(val * 0.70710678118654752f));
+          y[j] = val;
+        }
+        const bool full = nb + 32 <= args.N;
+        if (args.y32) {
+          float* dst = args.y32 + (size_t)row * args.N + nb;
+          if (full) {
+#pragma unroll
+            for (int j = 0; j < 32; j += 4) *reinterpret_cast<float4*>(dst + j) = make_float4(y[j], y[j + 1], y[j + 2], y[j + 3]);
+          } else {
+            for (int j = 0; j < args.N - nb; ++j) dst[j] = y[j];
+          }
+        }
+        if (args.y16) {
+          uint16_t* dst = args.y16 + (size_t)row * args.N + nb;
+          if (full) {
+#pragma unroll
+            for (int j = 0; j < 32; j += 8) {
+              uint4 p;
+              p.x = f32_to_bf16_rn(y[j]) | ((uint32_t)f32_to_bf16_rn(y[j + 1]) << 16);
+              p.y = f32_to_bf16_rn(y[j + 2]) | ((uint32_t)f32_to_bf16_rn(y[j + 3]) << 16);
+              p.z = f32_to_bf16_rn(y[j + 4]) | ((uint32_t)f32_to_bf16_rn(y[j + 5]) << 16);
+              p.w = f32_to_bf16_rn(y[j + 6]) | ((uint32_t)f32_to_bf16_rn(y[j + 7]) << 16);
+              *reinterpret_cast<uint4*>(dst + j) = p;
+            }
+          } else {
+            for (int j = 0; j < args.N - nb; ++j) dst[j] = f32_to_bf16_rn(y[j]);
+          }
+        }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(ACC_EMPTY + acc));
+    }
+  }
+
+  // teardown: every role is done (or gave up); release TMEM
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == MMA_WARP) {
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(TMEM_COLS) : "memory");
+  }
+}
+
+// ---- host side ----------------------------------------------------------------
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+int get_encode_fn(EncodeTiledFn* fn) {
+  static EncodeTiledFn cached = nullptr;
+  if (!cached) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    cudaError_t e = cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q);
+    if (e != cudaSuccess || q != cudaDriverEntryPointSuccess || !p)
+      return fail(OQ_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable (%s)", cudaGetErrorString(e));
+    cached = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  *fn = cached;
+  return OQ_OK;
+}
+
+// 2-D map over packed codes: [rows][row_bytes] uint8, box = (64 codes, box_rows).
+int make_code_map(CUtensorMap* map, const void* base, int rows, int row_bytes, int box_bytes, int box_rows) {
+  EncodeTiledFn enc;
+  if (int rc = get_encode_fn(&enc)) return rc;
+  cuuint64_t dims[2] = {(cuuint64_t)row_bytes, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)row_bytes};
+  cuuint32_t box[2] = {(cuuint32_t)box_bytes, (cuuint32_t)box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(OQ_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+  return OQ_OK;
+}
+
+using GemmKernel = void (*)(GemmArgs, CUtensorMap, CUtensorMap);
+
+template <int BA, int BW>
+int launch_t(GemmArgs& a, const uint8_t* a_codes, const uint8_t* w_codes, int nsm, cudaStream_t stream) {
+  CUtensorMap ma, mb;
+  if (int rc = make_code_map(&ma, a_codes, a.M, a.K * BA / 8, BK * BA / 8, BM)) return rc;
+  if (int rc = make_code_map(&mb, w_codes, a.N, a.K * BW / 8, BK * BW / 8, BN)) return rc;
+  GemmKernel k = cbgemm_kernel<BA, BW>;
+  const int smem = Smem<BA, BW>::kAlloc;
+  cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return fail(OQ_ERR_CUDA, "cudaFuncSetAttribute(GEMM): %s", cudaGetErrorString(e));
+  const int grid = std::min(a.num_tiles, nsm);
+  k<<<grid, NUM_THREADS, smem, stream>>>(a, ma, mb);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return fail(OQ_ERR_CUDA, "GEMM launch: %s", cudaGetErrorString(e));
+  return OQ_OK;
+}
+
+}  // namespace
+
+int launch_cbgemm(int d, oq_codebook_t cb_a, oq_codebook_t cb_w, const uint8_t* a_codes, const float* a_norm, int M,
+                  const uint8_t* w_codes, const uint16_t* w_norm, int N, const uint16_t* bias, int epilogue,
+                  float* Y_f32, uint16_t* Y_bf16, void* stream) {
+  int* status;
+  if (int rc = device_status_word(&status)) return rc;
+  int nsm;
+  if (int rc = sm_count(&nsm)) return rc;
+  GemmArgs a;
+  memset(&a, 0, sizeof(a));
+  a.a_norm = a_norm;
+  a.w_norm = w_norm;
+  a.bias = bias;
+  a.y32 = Y_f32;
+  a.y16 = Y_bf16;
+  a.status = status;
+  a.M = M;
+  a.N = N;
+  a.K = d;
+  a.tiles_m = (M + BM - 1) / BM;
+  a.num_tiles = a.tiles_m * ((N + BN - 1) / BN);
+  a.epilogue = epilogue;
+  a.inv_d = (float)(1.0 / (double)d);
+  for (int i = 0; i < 32; ++i) {
+    auto entry = [](oq_codebook_t cb, int k) -> uint32_t {
+      return k < (int)cb->lut.size() ? cb->lut[k] : 0u;
+    };
+    a.lut_a[i] = entry(cb_a, 2 * i) | (entry(cb_a, 2 * i + 1) << 16);
+    a.lut_w[i] = entry(cb_w, 2 * i) | (entry(cb_w, 2 * i + 1) << 16);
+  }
+  cudaStream_t s = (cudaStream_t)stream;
+  const int ba = cb_a->bits, bw = cb_w->bits;
+#define OQ_GEMM_CASE(X, Y) \
+  if (ba == X && bw == Y) return launch_t<X, Y>(a, a_codes, w_codes, nsm, s);
+  OQ_GEMM_CASE(4, 4)
+  OQ_GEMM_CASE(4, 2)
+  OQ_GEMM_CASE(6, 4)
+  OQ_GEMM_CASE(2, 2)
+  OQ_GEMM_CASE(2, 4)
+  OQ_GEMM_CASE(4, 6)
+  OQ_GEMM_CASE(6, 6)
+  OQ_GEMM_CASE(6, 2)
+  OQ_GEMM_CASE(2, 6)
+#undef OQ_GEMM_CASE
+  return fail(OQ_ERR_UNSUPPORTED, "no GEMM kernel for bits a=%d w=%d", ba, bw);
+}
+
 }  // namespace oq

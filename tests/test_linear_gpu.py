@@ -1,0 +1,243 @@
+"""Parity of the codebook GEMM (oq_linear_codes) and the full layer
+(oq_linear) against the fp64 oracle, through the C ABI.
+
+Rule: ||Y_gpu - Y_oracle||_F / ||Y_oracle||_F <= 2e-3 on the same codes and
+norms.  The codes and norms come from the oracle (quantized on the CPU) and
+are uploaded; the oracle sums in fp64 on the same declared fp16 dequant
+table the kernel multiplies.  For oq_linear the GPU quantizes X itself; its
+codes may differ from the oracle's only inside the 1e-5 boundary band, so the
+same bound applies.
+"""
+
+import math
+
+import numpy as np
+import pytest
+import torch
+
+from calibration_free_rotated_b200 import inputs
+from oracle import linear as olin
+from oracle import quantize as oqz
+from oracle import rpbh as orpbh
+
+pytestmark = pytest.mark.gpu
+
+TOL = 2e-3
+
+
+@pytest.fixture(scope="module")
+def oq():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    from calibration_free_rotated_b200 import build
+    build.build()
+    from calibration_free_rotated_b200 import orbitquant
+    return orbitquant
+
+
+_cb = {}
+
+
+def _lib_cb(oq, d, bits):
+    if (d, bits) not in _cb:
+        _cb[(d, bits)] = oq.Codebook(d, bits)
+    return _cb[(d, bits)]
+
+
+def _dev_u8(a):
+    return torch.from_numpy(np.ascontiguousarray(a)).cuda()
+
+
+def _dev_bf16(bits_u16):
+    return torch.from_numpy(np.ascontiguousarray(bits_u16).view(np.int16)).cuda().view(torch.bfloat16)
+
+
+def _oracle_weight(codebooks, W_bits, d, h, bits, seed=0):
+    perm, signs = orpbh.draw_permutation_and_signs(seed, d)
+    cw, r16, _, _ = oqz.quantize_weight_rows(inputs.bf16_bits_to_f64(W_bits), perm, signs, h,
+                                             codebooks(d, bits)["centroids"])
+    return cw, r16
+
+
+def _oracle_act(codebooks, X_bits, d, h, bits, seed=0):
+    perm, signs = orpbh.draw_permutation_and_signs(seed, d)
+    ca, s, _ = oqz.quantize_rows(inputs.bf16_bits_to_f64(X_bits), perm, signs, h, codebooks(d, bits)["centroids"])
+    return ca, s
+
+
+def _rel_fro(y, ref):
+    return float(np.linalg.norm(y - ref) / np.linalg.norm(ref))
+
+
+def _run_codes(oq, codebooks, ca, s, cw, r16, d, ba, bw, bias_bits=None, epilogue="none", want_bf16=False):
+    cb_a, cb_w = _lib_cb(oq, d, ba), _lib_cb(oq, d, bw)
+    a_codes = _dev_u8(oqz.pack_codes(ca, ba))
+    a_norm = torch.from_numpy(s.astype(np.float32)).cuda()
+    w_codes = _dev_u8(oqz.pack_codes(cw, bw))
+    w_norm = _dev_bf16(oqz.bf16_bits(r16))
+    bias = None if bias_bits is None else _dev_bf16(bias_bits)
+    y32, y16 = oq.linear_codes(d, cb_a, cb_w, a_codes, a_norm, w_codes, w_norm, bias=bias, epilogue=epilogue,
+                               want_bf16=want_bf16)
+    torch.cuda.synchronize()
+    oq.device_status()
+    ref = olin.linear_from_codes(ca, s, cw, r16, codebooks(d, ba)["centroids"], codebooks(d, bw)["centroids"], d,
+                                 bias=None if bias_bits is None else inputs.bf16_bits_to_f64(bias_bits),
+                                 gelu=(epilogue == "gelu"))
+    return y32.cpu().double().numpy(), (None if y16 is None else y16.float().cpu().double().numpy()), ref
+
+
+@pytest.mark.parametrize("ba,bw", [(4, 4), (4, 2), (6, 4), (2, 2), (6, 6), (2, 4)])
+def test_codes_gemm_small_ragged(oq, codebooks, ba, bw):
+    # several tiles in both M and N, M and N tails (M=200, N=272), K = 256
+    d, h, M, N = 256, 64, 200, 272
+    rng = np.random.default_rng(ba * 10 + bw)
+    X = inputs.to_bf16_bits(rng.standard_normal((M, d)))
+    W = inputs.to_bf16_bits(rng.standard_normal((N, d)) * 0.02)
+    ca, s = _oracle_act(codebooks, X, d, h, ba)
+    cw, r16 = _oracle_weight(codebooks, W, d, h, bw)
+    y, _, ref = _run_codes(oq, codebooks, ca, s, cw, r16, d, ba, bw)
+    assert _rel_fro(y, ref) <= TOL
+
+
+def test_codes_gemm_single_linear_workload(oq, codebooks):
+    # X[64 x 256] (3 outlier channels x20), W[256 x 256]; block 64; W4A4
+    d, h = 256, 64
+    X = inputs.activations(1, 64, d)
+    W = inputs.weights(1, inputs.T_W, 256, d)
+    ca, s = _oracle_act(codebooks, X, d, h, 4)
+    cw, r16 = _oracle_weight(codebooks, W, d, h, 4)
+    y, _, ref = _run_codes(oq, codebooks, ca, s, cw, r16, d, 4, 4)
+    assert _rel_fro(y, ref) <= TOL
+    # and the elementwise view: every output close in absolute terms
+    assert np.max(np.abs(y - ref)) <= 5e-3 * np.max(np.abs(ref))
+
+
+@pytest.mark.parametrize("epilogue", ["none", "gelu"])
+def test_codes_gemm_bias_gelu_and_bf16_output(oq, codebooks, epilogue):
+    d, h, M, N = 512, 128, 130, 256 + 48
+    rng = np.random.default_rng(5)
+    X = inputs.to_bf16_bits(rng.standard_normal((M, d)) * 3)
+    W = inputs.to_bf16_bits(rng.standard_normal((N, d)) * 0.05)
+    bias = inputs.to_bf16_bits(rng.standard_normal(N) * 0.5)
+    ca, s = _oracle_act(codebooks, X, d, h, 4)
+    cw, r16 = _oracle_weight(codebooks, W, d, h, 4)
+    y, y16, ref = _run_codes(oq, codebooks, ca, s, cw, r16, d, 4, 4, bias_bits=bias, epilogue=epilogue,
+                             want_bf16=True)
+    assert _rel_fro(y, ref) <= TOL
+    # bf16 output is the fp32 output rounded to nearest even
+    y_as_bf16 = torch.from_numpy(y.astype(np.float32)).to(torch.bfloat16).double().numpy()
+    assert np.array_equal(y16, y_as_bf16)
+
+
+def test_codes_gemm_long_k(oq, codebooks):
+    # K = 12288 (FLUX fc2 input width), 2-bit weights, 4-bit activations
+    d, h, M, N = 12288, 128, 150, 272
+    rng = np.random.default_rng(11)
+    X = inputs.to_bf16_bits(rng.standard_normal((M, d)))
+    W = inputs.to_bf16_bits(rng.standard_normal((N, d)) * 0.02)
+    ca, s = _oracle_act(codebooks, X, d, h, 4)
+    cw, r16 = _oracle_weight(codebooks, W, d, h, 2)
+    y, _, ref = _run_codes(oq, codebooks, ca, s, cw, r16, d, 4, 2)
+    assert _rel_fro(y, ref) <= TOL
+
+
+def test_zero_rows_give_bias_only(oq, codebooks):
+    d, h, M, N = 256, 64, 8, 32
+    rng = np.random.default_rng(2)
+    X = np.zeros((M, d))
+    X[1] = rng.standard_normal(d)
+    W = inputs.to_bf16_bits(rng.standard_normal((N, d)) * 0.02)
+    bias = inputs.to_bf16_bits(rng.standard_normal(N))
+    ca, s = _oracle_act(codebooks, inputs.to_bf16_bits(X), d, h, 4)
+    cw, r16 = _oracle_weight(codebooks, W, d, h, 4)
+    y, _, ref = _run_codes(oq, codebooks, ca, s, cw, r16, d, 4, 4, bias_bits=bias)
+    assert np.array_equal(y[0], inputs.bf16_bits_to_f64(bias).astype(np.float32).astype(np.float64))
+    assert _rel_fro(y, ref) <= TOL
+
+
+def _full_layer(oq, X_bits, W_bits, d, h, ba, bw, bias_bits=None, epilogue="none", want_bf16=False):
+    r = oq.Rpbh(0, d, h)
+    cb_a, cb_w = _lib_cb(oq, d, ba), _lib_cb(oq, d, bw)
+    W = _dev_bf16(W_bits)
+    w_codes, w_norm = oq.quantize_weight(r, cb_w, W)
+    X = _dev_bf16(X_bits)
+    bias = None if bias_bits is None else _dev_bf16(bias_bits)
+    y32, y16 = oq.linear(r, cb_a, cb_w, X, w_codes, w_norm, bias=bias, epilogue=epilogue, want_bf16=want_bf16)
+    torch.cuda.synchronize()
+    oq.device_status()
+    return y32, y16
+
+
+def test_flux_projection_full_size(oq, codebooks):
+    # X[4608 x 3072], fused QKV W[9216 x 3072] + bias, block 128, W4A4.
+    # GEMM on oracle codes (all rows), checked on sampled rows; then the full layer.
+    M, N, d, h = 4608, 9216, 3072, 128
+    X = inputs.activations(2, M, d)
+    W = inputs.weights(2, inputs.T_W, N, d)
+    bias = inputs.bias(2, N)
+    ca, s = _oracle_act(codebooks, X, d, h, 4)
+    cw, r16 = _oracle_weight(codebooks, W, d, h, 4)
+    rows = np.linspace(0, M - 1, 40).astype(int)
+    cb_a, cb_w = _lib_cb(oq, d, 4), _lib_cb(oq, d, 4)
+    y32, _ = oq.linear_codes(d, cb_a, cb_w, _dev_u8(oqz.pack_codes(ca, 4)), torch.from_numpy(s.astype(np.float32)).cuda(),
+                             _dev_u8(oqz.pack_codes(cw, 4)), _dev_bf16(oqz.bf16_bits(r16)), bias=_dev_bf16(bias))
+    torch.cuda.synchronize()
+    oq.device_status()
+    cents = codebooks(d, 4)["centroids"]
+    ref = olin.linear_from_codes(ca[rows], s[rows], cw, r16, cents, cents, d, bias=inputs.bf16_bits_to_f64(bias))
+    y = y32.cpu().double().numpy()[rows]
+    assert _rel_fro(y, ref) <= TOL
+    # full layer: the GPU quantizes X and W itself
+    y32, _ = _full_layer(oq, X, W, d, h, 4, 4, bias_bits=bias)
+    y = y32.cpu().double().numpy()[rows]
+    assert _rel_fro(y, ref) <= TOL
+    # the method's own W4A4 error against the unquantized product (not a parity bound):
+    # about 0.24 on these outlier-heavy rows, well below the size of the output
+    exact = inputs.bf16_bits_to_f64(X[rows]) @ inputs.bf16_bits_to_f64(W).T + inputs.bf16_bits_to_f64(bias)
+    assert _rel_fro(y, exact) < 0.5
+
+
+def test_flux_mlp_pair_w2a4(oq, codebooks):
+    # fc1 [12288 x 3072] -> GELU -> fc2 [3072 x 12288], W2A4, block 128; sampled rows.
+    M, d1, d2, h = 4608, 3072, 12288, 128
+    X = inputs.activations(3, M, d1)
+    W1 = inputs.weights(3, inputs.T_W, d2, d1)
+    W2 = inputs.weights(3, inputs.T_W2, d1, d2)
+    rows = np.linspace(0, M - 1, 16).astype(int)
+    y1, h1 = _full_layer(oq, X, W1, d1, h, 4, 2, epilogue="gelu", want_bf16=True)
+    ca, s = _oracle_act(codebooks, X[rows], d1, h, 4)
+    cw1, r1 = _oracle_weight(codebooks, W1, d1, h, 2)
+    ref1 = olin.linear_from_codes(ca, s, cw1, r1, codebooks(d1, 4)["centroids"], codebooks(d1, 2)["centroids"], d1,
+                                  gelu=True)
+    assert _rel_fro(y1.cpu().double().numpy()[rows], ref1) <= TOL
+    # fc2 on the oracle's own bf16 fc1 output (each layer judged on its own inputs)
+    h1_oracle = inputs.to_bf16_bits(ref1)
+    ca2, s2 = _oracle_act(codebooks, h1_oracle, d2, h, 4)
+    cw2, r2 = _oracle_weight(codebooks, W2, d2, h, 2)
+    y2, _ = _full_layer(oq, h1_oracle, W2, d2, h, 4, 2)
+    ref2 = olin.linear_from_codes(ca2, s2, cw2, r2, codebooks(d2, 4)["centroids"], codebooks(d2, 2)["centroids"], d2)
+    assert _rel_fro(y2.cpu().double().numpy(), ref2) <= TOL
+
+
+def test_wan_ffn_w4a6_sampled(oq, codebooks):
+    # X[32760 x 1536] Student-t(3), fc1 W[8960 x 1536] with 6-bit activations: M tail tile
+    M, d, N, h = 32760, 1536, 8960, 128
+    X = inputs.activations(4, M, d)
+    W1 = inputs.weights(4, inputs.T_W, N, d)
+    y1, _ = _full_layer(oq, X, W1, d, h, 6, 4, epilogue="gelu")
+    rows = np.concatenate([np.linspace(0, M - 1, 20).astype(int), [M - 1]])
+    ca, s = _oracle_act(codebooks, X[rows], d, h, 6)
+    cw, r16 = _oracle_weight(codebooks, W1, d, h, 4)
+    ref = olin.linear_from_codes(ca, s, cw, r16, codebooks(d, 6)["centroids"], codebooks(d, 4)["centroids"], d,
+                                 gelu=True)
+    assert _rel_fro(y1.cpu().double().numpy()[rows], ref) <= TOL
+
+
+def test_empty_shapes(oq):
+    cb = _lib_cb(oq, 256, 4)
+    a = torch.empty((0, 128), dtype=torch.uint8, device="cuda")
+    w = torch.zeros((32, 128), dtype=torch.uint8, device="cuda")
+    y32, _ = oq.linear_codes(256, cb, cb, a, torch.empty(0, device="cuda"), w,
+                             torch.ones(32, dtype=torch.bfloat16, device="cuda"))
+    assert y32.shape == (0, 32)
+    oq.device_status()
