@@ -1,0 +1,385 @@
+"""Benchmark of the OrbitQuant hot path on B200: one step = RPBH rotate +
+Lloyd-Max quantize of the activations, then the codebook W4A4 GEMM with the
+norm-rescale + bias epilogue, on the FLUX-like attention projection
+(X[4608 x 3072] bf16, fused QKV W[9216 x 3072], block 128, W4A4).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Prints ONE JSON line (rank 0).  Multi-GPU (torchrun, one rank per GPU): every
+rank runs its own copy of the workload (the path is row-parallel with no
+exchange), timing is the max over ranks, value is the whole-job throughput.
+`--impl reference` times the CPU oracle (plain fp64 NumPy) on a bounded sample
+of the same workload; it is the deliberately slow program the ratio divides by.
+"""
+
+import argparse
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "RPBH+Lloyd-Max act-quant GB/s (frac of HBM); codebook W4A4 linear TFLOP/s"
+UNIT = "TFLOP/s"
+WORKLOAD = dict(workload="flux_attention_qkv_projection", M=4608, K=3072, N=9216, block=128, bits_w=4, bits_a=4,
+                seed=0, bias=True, out="bf16")
+N_SETS = 4
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def algorithmic(M, K, N, ba, bw):
+    """Per-launch algorithmic work: act-quant bytes (read bf16 X, write codes and
+    fp32 norms) and GEMM flops 2MNK."""
+    aq_bytes = M * K * 2 + M * K * ba / 8 + 4 * M
+    gemm_flops = 2.0 * M * N * K
+    return aq_bytes, gemm_flops
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return FALLBACK_PEAKS, "fallback"
+
+
+def profiled_traffic(kernel_file, summary_name):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken on
+    the current source of that kernel (matching sha256), else None."""
+    import hashlib
+    path = os.path.join(ROOT, "profiles", summary_name)
+    src = os.path.join(ROOT, "calibration_free_rotated_b200", "csrc", kernel_file)
+    if not (os.path.exists(path) and os.path.exists(src)):
+        return None
+    sha = hashlib.sha256(open(src, "rb").read()).hexdigest()
+    vals = {}
+    for line in open(path):
+        if ":" in line:
+            k, v = line.split(":", 1)
+            vals[k.strip().strip("-* ").lower()] = v.strip().strip("`")
+    if vals.get("source_sha256") != sha:
+        return None
+    try:
+        return float(vals["traffic_bytes_per_launch"])
+    except (KeyError, ValueError):
+        return None
+
+
+class ClockSampler:
+    """Samples SM clock and clock-event reasons through NVML while running."""
+
+    REASONS = {
+        0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap", 0x8: "hw_slowdown",
+        0x10: "sync_boost", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+        0x100: "display_clock_setting",
+    }
+
+    def __init__(self, device_index):
+        self.samples, self.reasons, self.max_mhz = [], set(), None
+        self._stop = threading.Event()
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self._nv = pynvml
+            self._h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+        except Exception:
+            self._nv = None
+
+    def _poll(self):
+        nv = self._nv
+        while True:
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM))
+                r = nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+                for bit, name in self.REASONS.items():
+                    if r & bit:
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            if self._stop.wait(0.005):
+                break
+
+    def __enter__(self):
+        if self._nv is not None:
+            self._t = threading.Thread(target=self._poll, daemon=True)
+            self._t.start()
+        return self
+
+    def __exit__(self, *exc):
+        if self._nv is not None:
+            self._stop.set()
+            self._t.join()
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons), "samples": 0}
+        return {"sm_mhz": float(statistics.median(self.samples)), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons - {"gpu_idle"}), "samples": len(self.samples)}
+
+
+def dist_setup():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def reduce_max(values, world):
+    """Max over ranks of a list of floats (identity when world == 1)."""
+    if world == 1:
+        return list(values)
+    import torch
+    import torch.distributed as dist
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor(values, dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return t.cpu().tolist()
+
+
+def whole_job_value(units_per_rank, world, max_seconds):
+    return units_per_rank * world / max_seconds
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle arm (reference arm and cpu_baseline)
+# ---------------------------------------------------------------------------
+def oracle_sample(rows, W_state=None):
+    """Times the oracle on `rows` activation rows of the workload: act-quant +
+    fp64 linear against precomputed oracle weight codes (offline step, untimed)."""
+    from calibration_free_rotated_b200 import inputs
+    from oracle import codebook as ocb
+    from oracle import linear as olin
+    from oracle import quantize as oqz
+    from oracle import rpbh as orpbh
+    w = WORKLOAD
+    M, K, N, h = w["M"], w["K"], w["N"], w["block"]
+    if W_state is None:
+        perm, signs = orpbh.draw_permutation_and_signs(w["seed"], K)
+        cb = ocb.lloyd_max(K, 4)
+        Wb = inputs.weights(2, inputs.T_W, N, K)
+        cw, r16, _, _ = oqz.quantize_weight_rows(inputs.bf16_bits_to_f64(Wb), perm, signs, h, cb["centroids"])
+        bias = inputs.bf16_bits_to_f64(inputs.bias(2, N))
+        W_state = dict(perm=perm, signs=signs, cb=cb, cw=cw, r16=r16, bias=bias)
+    X = inputs.bf16_bits_to_f64(inputs.activations(2, M, K, rows=(0, rows)))
+    st = W_state
+    t0 = time.perf_counter()
+    ca, s, _ = oqz.quantize_rows(X, st["perm"], st["signs"], h, st["cb"]["centroids"])
+    y = olin.linear_from_codes(ca, s, st["cw"], st["r16"], st["cb"]["centroids"], st["cb"]["centroids"], K,
+                               bias=st["bias"])
+    dt = time.perf_counter() - t0
+    assert np.isfinite(y).all()
+    return dt, W_state
+
+
+def cpu_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = max((i.get("num_threads", 1) for i in threadpool_info()), default=1)
+        return int(n)
+    except Exception:
+        return os.cpu_count()
+
+
+def run_reference(args, world, rank):
+    if rank != 0:
+        return 0
+    w = WORKLOAD
+    rows = 256
+    _, flops = algorithmic(rows, w["K"], w["N"], w["bits_a"], w["bits_w"])
+    dt, st = oracle_sample(rows)
+    for _ in range(max(0, args.warmup - 1)):
+        oracle_sample(rows, st)
+    times = [oracle_sample(rows, st)[0] for _ in range(args.steps)]
+    total = sum(times)
+    value = flops * args.steps / total / 1e12
+    sample = f"{rows} of {w['M']} activation rows per step (act-quant + fp64 linear vs all {w['N']} outputs)"
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * total / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": dict(w, l2="n/a (CPU)", sample_rows=rows),
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cpu_threads(), "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ---------------------------------------------------------------------------
+# GPU arm
+# ---------------------------------------------------------------------------
+def run_ours(args, world, rank, local):
+    import torch
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device (no CPU fallback)")
+    torch.cuda.set_device(local)
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    from calibration_free_rotated_b200 import build
+    build.build()
+    from calibration_free_rotated_b200 import inputs
+    from calibration_free_rotated_b200 import orbitquant as oq
+
+    w = WORKLOAD
+    M, K, N, h = w["M"], w["K"], w["N"], w["block"]
+    dev = torch.device("cuda", local)
+    stream = torch.cuda.current_stream()
+    r = oq.Rpbh(w["seed"], K, h)
+    cb = oq.Codebook(K, 4)
+
+    def dev_bf16(bits):
+        return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).to(dev).view(torch.bfloat16)
+
+    X0 = dev_bf16(inputs.activations(2, M, K))
+    W0 = dev_bf16(inputs.weights(2, inputs.T_W, N, K))
+    bias = dev_bf16(inputs.bias(2, N))
+    # offline weight quantization (not part of the step)
+    wc0, wn = oq.quantize_weight(r, cb, W0)
+    del W0
+    sets = []
+    for i in range(N_SETS):
+        sets.append(dict(
+            X=X0.clone(), wc=wc0.clone(),
+            codes=torch.empty((M, K * 4 // 8), dtype=torch.uint8, device=dev),
+            norms=torch.empty((M,), dtype=torch.float32, device=dev),
+            Y=torch.empty((M, N), dtype=torch.bfloat16, device=dev)))
+    torch.cuda.synchronize()
+
+    def step(i, ev=None):
+        s = sets[i % N_SETS]
+        if ev is not None:
+            ev[0].record(stream)
+        oq.quantize_act(r, cb, s["X"], s["codes"], s["norms"], stream=stream)
+        if ev is not None:
+            ev[1].record(stream)
+        oq.linear_codes(K, cb, cb, s["codes"], s["norms"], s["wc"], wn, bias=bias, out_bf16=s["Y"],
+                        want_f32=False, want_bf16=True, stream=stream)
+        if ev is not None:
+            ev[2].record(stream)
+
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize()
+    oq.device_status()
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(torch.cuda.current_device()) as clk:
+        start.record(stream)
+        for i in range(args.steps):
+            step(i, evs[i])
+        end.record(stream)
+        torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    oq.device_status()
+    total_s = start.elapsed_time(end) / 1e3
+    k1 = [e[0].elapsed_time(e[1]) / 1e3 for e in evs]
+    k2 = [e[1].elapsed_time(e[2]) / 1e3 for e in evs]
+    total_s, k1_avg, k2_avg = reduce_max([total_s, sum(k1) / len(k1), sum(k2) / len(k2)], world)
+
+    aq_bytes, flops = algorithmic(M, K, N, 4, 4)
+    value = whole_job_value(flops * args.steps, world, total_s) / 1e12
+
+    # end to end through the public oq_linear call with host buffers
+    Xh = torch.empty((M, K), dtype=torch.bfloat16, pin_memory=True)
+    Xh.copy_(X0.cpu())
+    Yh = torch.empty((M, N), dtype=torch.bfloat16, pin_memory=True)
+    ws = torch.empty((oq.workspace_bytes(M, K, 4),), dtype=torch.uint8, device=dev)
+    Xd = torch.empty_like(X0)
+    Yd = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+
+    def e2e_step():
+        Xd.copy_(Xh, non_blocking=True)
+        oq.linear(r, cb, cb, Xd, wc0, wn, bias=bias, out_bf16=Yd, want_f32=False, want_bf16=True, workspace=ws,
+                  stream=stream)
+        Yh.copy_(Yd, non_blocking=True)
+
+    for _ in range(max(1, args.warmup)):
+        e2e_step()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for _ in range(args.steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_s = reduce_max([e0.elapsed_time(e1) / 1e3], world)[0]
+    oq.device_status()
+    e2e_value = whole_job_value(flops * args.steps, world, e2e_s) / 1e12
+
+    peaks, peak_kind = load_peaks()
+    gemm_tflops = flops / k2_avg / 1e12
+    aq_gbs = aq_bytes / k1_avg / 1e9
+    gemm_traffic = profiled_traffic("oq_cbgemm.cu", "cbgemm_flux_qkv_w4a4.md")
+    aq_traffic = profiled_traffic("oq_rotq.cu", "rotq_flux_qkv_act_w4.md")
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": 1e3 * total_s / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f16 (tensor operands, f32 accumulate; f32 rotate)",
+        "data": "synthetic",
+        "config": dict(w, parallelism=f"replicated weights, rows per rank (dp{world})",
+                       l2=f"{N_SETS} rotating input/weight/output sets (~{N_SETS * 127} MB) > 126 MB L2"),
+        "roofline": {"bound": "tensor", "kernel": "cbgemm_kernel", "achieved": gemm_tflops,
+                     "peak": peaks["bf16_tflops"], "unit": "TFLOP/s", "frac": gemm_tflops / peaks["bf16_tflops"],
+                     "traffic": gemm_traffic, "peak_source": f"{peak_kind} bf16 burst (f16 same rate)",
+                     "algorithmic_per_launch": flops},
+        "roofline_act_quant": {"bound": "hbm", "kernel": "rotq_kernel", "achieved": aq_gbs,
+                               "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": aq_gbs / peaks["hbm_gbs"],
+                               "traffic": aq_traffic, "peak_source": f"{peak_kind} copy bandwidth",
+                               "algorithmic_per_launch": aq_bytes},
+        "kernel_ms": {"rotq_kernel": 1e3 * k1_avg, "cbgemm_kernel": 1e3 * k2_avg},
+        "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": M * K * 2, "d2h_bytes_per_step": M * N * 2},
+        "gpu_launches": 2 * args.steps,
+        "clocks": clk.summary(),
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        rows = 2048
+        _, st = oracle_sample(8)
+        dt, _ = oracle_sample(rows, st)
+        _, sflops = algorithmic(rows, K, N, 4, 4)
+        line["cpu_baseline"] = {"value": sflops / dt / 1e12, "unit": UNIT, "cores": cpu_threads(), "kind": "oracle",
+                                "sample": f"{rows} of {M} activation rows (act-quant + fp64 linear vs all {N} "
+                                          "outputs); weights quantized beforehand, untimed"}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    world, rank, local = dist_setup()
+    if args.impl == "reference":
+        return run_reference(args, world, rank)
+    return run_ours(args, world, rank, local)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

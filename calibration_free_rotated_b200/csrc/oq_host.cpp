@@ -474,8 +474,8 @@ static int check_linear_args(int d, oq_codebook_t cb_a, oq_codebook_t cb_w, int 
   auto ok_bits = [](int b) { return b == 2 || b == 4 || b == 6; };
   if (!ok_bits(cb_a->bits) || !ok_bits(cb_w->bits))
     return fail(OQ_ERR_UNSUPPORTED, "the GEMM needs bits in {2,4,6} (a=%d, w=%d)", cb_a->bits, cb_w->bits);
-  if (!Y_f32 && !Y_bf16) return fail(OQ_ERR_ARG, "at least one of Y_f32 / Y_bf16 is needed");
   if (M == 0 || N == 0) return OQ_OK;
+  if (!Y_f32 && !Y_bf16) return fail(OQ_ERR_ARG, "at least one of Y_f32 / Y_bf16 is needed");
   if (!w_codes || !w_norm) return fail(OQ_ERR_ARG, "NULL weight buffer");
   if (!aligned16(w_codes) || !aligned16(w_norm) || (bias && !aligned16(bias)) || (Y_f32 && !aligned16(Y_f32)) ||
       (Y_bf16 && !aligned16(Y_bf16)))

@@ -100,6 +100,8 @@ def test_argument_errors_without_gpu(oq):
                                ctypes.c_void_p(16), None, None) == oq.OQ_ERR_ARG           # epilogue
     assert lib.oq_linear_codes(256, cb.handle, cb2.handle, None, None, 4, None, None, 32, None, 0,
                                None, None, None) == oq.OQ_ERR_ARG                          # no output
+    assert lib.oq_linear_codes(256, cb.handle, cb2.handle, None, None, 0, None, None, 32, None, 0,
+                               None, None, None) == oq.OQ_OK                               # M == 0
 
 
 def test_workspace_bytes(oq):
