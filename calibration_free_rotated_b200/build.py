@@ -15,7 +15,7 @@ import sys
 HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "liborbitquant.so")
-SOURCES = ["oq_host.cpp", "oq_rotq.cu", "oq_cbgemm.cu"]
+SOURCES = ["oq_host.cpp", "oq_rotq.cu", "oq_cbgemm.cu", "oq_noalloc.cu"]
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",
     "-lineinfo", "-O3", "-std=c++17",

@@ -236,6 +236,15 @@ int device_status_word(int** status) {
   return OQ_OK;
 }
 
+int device_status_word_if_present(int** status) {
+  int dev;
+  if (int rc = current_device(&dev)) return rc;
+  std::lock_guard<std::mutex> lk(g_dev_mu);
+  if (!g_status[dev]) return OQ_ERR_ARG;
+  *status = g_status[dev];
+  return OQ_OK;
+}
+
 int sm_count(int* n) {
   int dev;
   if (int rc = current_device(&dev)) return rc;

@@ -46,6 +46,7 @@ uint16_t double_to_fp16_rne(double v);
 int current_device(int* dev);
 int rpbh_device_tables(oq_rpbh_t r, const uint16_t** perm, const uint32_t** signs);
 int device_status_word(int** status);
+int device_status_word_if_present(int** status);  // never allocates
 int sm_count(int* n);
 bool aligned16(const void* p);
 

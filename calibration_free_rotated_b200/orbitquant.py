@@ -45,7 +45,10 @@ _SIGS = {
     "oq_linear_workspace_bytes": (_c_size_t, [_c_int, _c_int, _c_int]),
     "oq_linear": (_c_int, [_c_void_p, _c_void_p, _c_void_p, _c_void_p, _c_int, _c_void_p, _c_void_p, _c_int,
                            _c_void_p, _c_int, _c_void_p, _c_void_p, _c_void_p, _c_size_t, _c_void_p]),
+    "oq_linear_noalloc": (_c_int, [_c_void_p, _c_void_p, _c_void_p, _c_void_p, _c_int, _c_void_p, _c_void_p,
+                                   _c_int, _c_void_p, _c_int, _c_void_p, _c_void_p, _c_void_p]),
 }
+NOALLOC_SCRATCH_BYTES = 32 << 20
 for _name, (_res, _args) in _SIGS.items():
     _fn = getattr(_lib, _name)
     _fn.restype = _res
@@ -203,3 +206,15 @@ def linear(rpbh: Rpbh, cb_a: Codebook, cb_w: Codebook, X, w_codes, w_norm, bias=
 def device_status(stream=None):
     """Raises OQError if a kernel's bounded wait gave up since the last call."""
     _check(_lib.oq_get_device_status(_stream(stream)))
+
+
+def linear_noalloc(rpbh: Rpbh, cb_a: Codebook, cb_w: Codebook, X, w_codes, w_norm, bias=None, epilogue="none",
+                   out_f32=None, out_bf16=None, stream=None):
+    """oq_linear_noalloc: the full layer with the library's static scratch
+    instead of a workspace.  Outputs must be passed in (this call is for code
+    that cannot allocate)."""
+    M, N = X.shape[0], w_codes.shape[0]
+    _check(_lib.oq_linear_noalloc(rpbh.handle, cb_a.handle, cb_w.handle, _ptr(X), M, _ptr(w_codes), _ptr(w_norm),
+                                  N, _ptr(bias), EPILOGUES[epilogue], _ptr(out_f32), _ptr(out_bf16),
+                                  _stream(stream)))
+    return out_f32, out_bf16

@@ -183,6 +183,42 @@ OQ_API int oq_linear(oq_rpbh_t r, oq_codebook_t cb_a, oq_codebook_t cb_w, const 
               const void* w_norm, int N, const void* bias, int epilogue, float* Y_f32, void* Y_bf16,
               void* workspace, size_t workspace_bytes, void* stream);
 
+/* ---------------------------------------------------------------------------
+ * oq_linear without a workspace, for callers that cannot allocate.
+ * The OrbitQuant pages have no counterpart for this entry point.
+ *
+ * Some callers run where they may not allocate device memory and have no
+ * buffer of their own to lend (an inference engine's execute callback that
+ * owns every allocation, a latency-critical loop that cannot take the
+ * implicit synchronisation of cudaMalloc).  This call does exactly what
+ * oq_linear does, but keeps the activation codes and norms in a fixed static
+ * device array of OQ_NOALLOC_SCRATCH_BYTES instead of a caller workspace.
+ *   - It allocates nothing: no cudaMalloc/cudaFree, no allocating library
+ *     routine.  The static array is held by every GPU that loads the library
+ *     until the process exits.
+ *   - Size limit: oq_linear_workspace_bytes(M, d, bits_a) must not exceed
+ *     OQ_NOALLOC_SCRATCH_BYTES (32 MiB); larger calls return
+ *     OQ_ERR_UNSUPPORTED before launching anything.
+ *   - Preconditions (checked; OQ_ERR_ARG otherwise, never an allocation): the
+ *     rotation handle was created with this device current, and the device
+ *     already has the library's status word (any earlier launching call on
+ *     the device, or oq_get_device_status(), creates it).
+ *   - The first call on a device looks up the array's device address with
+ *     cudaGetSymbolAddress (with that device current) and caches it; make
+ *     that first call before any stream capture.
+ *   - All calls share the one array, which keeps the last call's contents;
+ *     nothing in it has to start at zero (the quantize kernel rewrites the
+ *     codes and norms of all M rows before the GEMM reads them).  Calls that
+ *     overlap on the GPU (different streams, or several host threads) race on
+ *     the array: serialise them.
+ * Arguments, layouts and errors are otherwise those of oq_linear.
+ * ------------------------------------------------------------------------- */
+#define OQ_NOALLOC_SCRATCH_BYTES (32u << 20)
+
+OQ_API int oq_linear_noalloc(oq_rpbh_t r, oq_codebook_t cb_a, oq_codebook_t cb_w, const void* X, int M,
+                             const uint8_t* w_codes, const void* w_norm, int N, const void* bias, int epilogue,
+                             float* Y_f32, void* Y_bf16, void* stream);
+
 #ifdef __cplusplus
 }
 #endif
