@@ -365,6 +365,37 @@ def run_ours(args, world, rank, local):
     return 0
 
 
+def run_profile_case(args):
+    """Launches one kernel on a given shape, for ncu captures (prints a short JSON,
+    not the contract line).  Data: device-side random bf16 rows / random codes."""
+    import torch
+    from calibration_free_rotated_b200 import build
+    build.build()
+    from calibration_free_rotated_b200 import orbitquant as oq
+    torch.manual_seed(0)
+    M, d, N = args.rows, args.d, args.n
+    if args.profile == "rotq":
+        r = oq.Rpbh(0, d, args.block)
+        cb = oq.Codebook(d, args.bits_a)
+        X = torch.randn(M, d, device="cuda").to(torch.bfloat16)
+        codes, norms = oq.quantize_act(r, cb, X)
+        run = lambda: oq.quantize_act(r, cb, X, codes, norms)
+    else:
+        cba, cbw = oq.Codebook(d, args.bits_a), oq.Codebook(d, args.bits_w)
+        a = torch.randint(0, 256, (M, d * args.bits_a // 8), dtype=torch.uint8, device="cuda")
+        w = torch.randint(0, 256, (N, d * args.bits_w // 8), dtype=torch.uint8, device="cuda")
+        an = torch.rand(M, device="cuda")
+        wn = torch.rand(N, device="cuda").to(torch.bfloat16)
+        y = torch.empty(M, N, device="cuda", dtype=torch.bfloat16)
+        run = lambda: oq.linear_codes(d, cba, cbw, a, an, w, wn, out_bf16=y, want_f32=False, want_bf16=True)
+    for _ in range(args.warmup + args.steps):
+        run()
+    torch.cuda.synchronize()
+    oq.device_status()
+    print(json.dumps({"profile": args.profile, "rows": M, "d": d, "n": N, "launches": args.warmup + args.steps}))
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -372,7 +403,16 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--profile", choices=["rotq", "gemm"], help="launch one kernel only (for ncu captures)")
+    ap.add_argument("--rows", type=int, default=4608)
+    ap.add_argument("--d", type=int, default=3072)
+    ap.add_argument("--n", type=int, default=9216)
+    ap.add_argument("--block", type=int, default=128)
+    ap.add_argument("--bits-a", type=int, default=4)
+    ap.add_argument("--bits-w", type=int, default=4)
     args = ap.parse_args()
+    if args.profile:
+        return run_profile_case(args)
     if args.warmup < 3:
         args.warmup = 3
     world, rank, local = dist_setup()

@@ -8,17 +8,17 @@
 // LUT = fp16(sqrt(d) c)), y = acc * s_m * r'_n / d + bias_n, optional GELU.
 //
 // sm_100a design (one CTA per SM, persistent over 128 x 256 output tiles):
-//   warp 12      TMA producer: 2-D tensor copies of the packed code tiles
+//   warp 20      TMA producer: 2-D tensor copies of the packed code tiles
 //                (A: 128 rows, B: 256 rows, 64 codes of K each) into a
 //                4-deep packed ring.
-//   warps 0..7   converters: expand codes through the fp16 LUT (register
+//   warps 0..15  converters: expand codes through the fp16 LUT (register
 //                byte-permute tables for 2 and 4 bits, a 128-byte shared
 //                table for 6 bits) straight into the canonical K-major
 //                128-byte-swizzled UMMA layout of a 3-deep expanded ring.
-//   warp 13      one thread issues tcgen05.mma (kind::f16, M=128, N=256,
+//   warp 21      one thread issues tcgen05.mma (kind::f16, M=128, N=256,
 //                K=16, fp32 accumulate in TMEM); tcgen05.commit frees ring
 //                stages and publishes finished accumulators.
-//   warps 8..11  epilogue: tcgen05.ld of the accumulator (each warp its
+//   warps 16..19 epilogue: tcgen05.ld of the accumulator (each warp its
 //                32-lane quadrant), rescale, bias, GELU, fp32/bf16 stores.
 // TMEM holds two 128 x 256 fp32 accumulators (all 512 columns) so the
 // epilogue of one tile overlaps the main loop of the next.  Every mbarrier
@@ -40,11 +40,12 @@ namespace {
 constexpr int BM = 128, BN = 256, BK = 64;
 constexpr int PSTAGES = 4;
 constexpr int ESTAGES = 3;
-constexpr int NUM_CONV_WARPS = 8;
-constexpr int EPI_WARP0 = 8;
-constexpr int TMA_WARP = 12;
-constexpr int MMA_WARP = 13;
-constexpr int NUM_THREADS = 14 * 32;
+constexpr int NUM_CONV_WARPS = 16;
+constexpr int NUM_CONV = NUM_CONV_WARPS * 32;
+constexpr int EPI_WARP0 = 16;
+constexpr int TMA_WARP = 20;
+constexpr int MMA_WARP = 21;
+constexpr int NUM_THREADS = 22 * 32;
 constexpr int TMEM_COLS = 512;
 constexpr unsigned long long kWaitLimitNs = 1000000000ull;
 
@@ -243,15 +244,14 @@ __device__ __forceinline__ uint4 expand8(uint64_t packed, const Lut16& t16, uint
   return r;
 }
 
+// Eight packed codes starting at byte offset `off` of a packed tile (8*BITS bits).
 template <int BITS>
-__device__ __forceinline__ uint64_t load_chunk(const uint8_t* tile, int row, int c) {
-  constexpr int RB = PackedTile<BITS>::kRowBytes;
+__device__ __forceinline__ uint64_t load_chunk(const uint8_t* tile, int off) {
   if constexpr (BITS == 4) {
-    return *reinterpret_cast<const uint32_t*>(tile + row * RB + 4 * c);
+    return *reinterpret_cast<const uint32_t*>(tile + off);
   } else if constexpr (BITS == 2) {
-    return *reinterpret_cast<const uint16_t*>(tile + row * RB + 2 * c);
+    return *reinterpret_cast<const uint16_t*>(tile + off);
   } else {
-    const int off = row * RB + 6 * c;
     const int base = off & ~3;
     const uint64_t lo = *reinterpret_cast<const uint32_t*>(tile + base);
     const uint64_t hi = *reinterpret_cast<const uint32_t*>(tile + base + 4);
@@ -350,11 +350,21 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     }
   } else if (warp < NUM_CONV_WARPS) {
     // ---- converters ----
+    // Thread ct owns chunk (row, c) = (ct/8 + 64 i, ct % 8) of every stage: A rows
+    // i = 0..1, B rows i = 0..3.  Row & 7 does not depend on i, so each chunk's
+    // swizzled store offset and packed load offset are a per-thread base plus a
+    // compile-time stride.
     Lut16 ta, tw;
     uint32_t qa0 = args.lut_a[0], qa1 = args.lut_a[1], qw0 = args.lut_w[0], qw1 = args.lut_w[1];
     if constexpr (BA == 4) ta = make_lut16(args.lut_a);
     if constexpr (BW == 4) tw = make_lut16(args.lut_w);
-    const int ct = threadIdx.x;  // 0..255
+    const int ct = threadIdx.x;  // 0..NUM_CONV-1
+    const int r0 = ct >> 3, c = ct & 7;
+    const uint32_t st_off = sw128_offset(r0, c);
+    constexpr int RB_A = PackedTile<BA>::kRowBytes, RB_B = PackedTile<BW>::kRowBytes;
+    const int ld_a = r0 * RB_A + c * BA, ld_b = r0 * RB_B + c * BW;  // 8 codes = BITS bytes
+    constexpr int ROWS_PER_PASS = NUM_CONV / 8;                     // 64
+    constexpr int ST_STRIDE = ROWS_PER_PASS / 8 * 1024;             // 8192 bytes
     uint32_t pc = 0;
     bool ok = true;
     for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
@@ -368,28 +378,24 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         }
         const uint8_t* pa = smem + S::kPackA + ps * ((S::kPkA + 127) / 128 * 128);
         const uint8_t* pb = smem + S::kPackB + ps * ((S::kPkB + 127) / 128 * 128);
-        unsigned char* ea = smem + S::kExpA + es * EXP_A_BYTES;
-        unsigned char* eb = smem + S::kExpB + es * EXP_B_BYTES;
+        unsigned char* ea = smem + S::kExpA + es * EXP_A_BYTES + st_off;
+        unsigned char* eb = smem + S::kExpB + es * EXP_B_BYTES + st_off;
+        uint64_t ra[BM / ROWS_PER_PASS], rb[BN / ROWS_PER_PASS];
 #pragma unroll
-        for (int i = 0; i < (BM * 8) / (NUM_CONV_WARPS * 32); ++i) {
-          const int ci = ct + i * NUM_CONV_WARPS * 32;
-          const int row = ci >> 3, c = ci & 7;
-          const uint4 v = expand8<BA>(load_chunk<BA>(pa, row, c), ta, qa0, qa1, lut_a_s);
-          *reinterpret_cast<uint4*>(ea + sw128_offset(row, c)) = v;
-        }
+        for (int i = 0; i < BM / ROWS_PER_PASS; ++i) ra[i] = load_chunk<BA>(pa, ld_a + i * ROWS_PER_PASS * RB_A);
 #pragma unroll
-        for (int i = 0; i < (BN * 8) / (NUM_CONV_WARPS * 32); ++i) {
-          const int ci = ct + i * NUM_CONV_WARPS * 32;
-          const int row = ci >> 3, c = ci & 7;
-          const uint4 v = expand8<BW>(load_chunk<BW>(pb, row, c), tw, qw0, qw1, lut_w_s);
-          *reinterpret_cast<uint4*>(eb + sw128_offset(row, c)) = v;
-        }
+        for (int i = 0; i < BN / ROWS_PER_PASS; ++i) rb[i] = load_chunk<BW>(pb, ld_b + i * ROWS_PER_PASS * RB_B);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(PK_EMPTY + ps));  // packed stage fully read by this warp
+#pragma unroll
+        for (int i = 0; i < BM / ROWS_PER_PASS; ++i)
+          *reinterpret_cast<uint4*>(ea + i * ST_STRIDE) = expand8<BA>(ra[i], ta, qa0, qa1, lut_a_s);
+#pragma unroll
+        for (int i = 0; i < BN / ROWS_PER_PASS; ++i)
+          *reinterpret_cast<uint4*>(eb + i * ST_STRIDE) = expand8<BW>(rb[i], tw, qw0, qw1, lut_w_s);
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
         __syncwarp();
-        if (lane == 0) {
-          mbar_arrive(bar(PK_EMPTY + ps));
-          mbar_arrive(bar(EX_FULL + es));
-        }
+        if (lane == 0) mbar_arrive(bar(EX_FULL + es));
       }
     }
   } else if (warp == MMA_WARP) {
@@ -440,56 +446,44 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       const float a_scale = row_ok ? args.a_norm[row] * args.inv_d : 0.0f;
       const uint32_t taddr = tmem_base + ((uint32_t)(quad * 32) << 16) + (uint32_t)(acc * BN);
 #pragma unroll 1
-      for (int c0 = 0; c0 < BN; c0 += 32) {
-        uint32_t v[32];
+      for (int c0 = 0; c0 < BN; c0 += 16) {
+        uint32_t v[16];
         __syncwarp();
         asm volatile(
-            "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, "
-            "%14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+            "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, "
+            "%14, %15}, [%16];"
             : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7]),
-              "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]), "=r"(v[15]),
-              "=r"(v[16]), "=r"(v[17]), "=r"(v[18]), "=r"(v[19]), "=r"(v[20]), "=r"(v[21]), "=r"(v[22]),
-              "=r"(v[23]), "=r"(v[24]), "=r"(v[25]), "=r"(v[26]), "=r"(v[27]), "=r"(v[28]), "=r"(v[29]),
-              "=r"(v[30]), "=r"(v[31])
+              "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]), "=r"(v[15])
             : "r"(taddr + (uint32_t)c0));
         asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
         const int nb = n0 + c0;
-        if (row_ok && nb < args.N) {
-        float y[32];
+        if (row_ok && nb < args.N) {  // N % 16 == 0: a 16-column group is all in or all out
+          float y[16];
 #pragma unroll
-        for (int j = 0; j < 32; ++j) {
-          const int n = min(nb + j, args.N - 1);
-          float val = __uint_as_float(v[j]) * a_scale * bf16_to_f32(args.w_norm[n]);
-          if (args.bias) val += bf16_to_f32(args.bias[n]);
-          if (args.epilogue == OQ_EPI_GELU) val = 0.5f * val * (1.0f + erff(val * 0.70710678118654752f));
-          y[j] = val;
-        }
-        const bool full = nb + 32 <= args.N;
-        if (args.y32) {
-          float* dst = args.y32 + (size_t)row * args.N + nb;
-          if (full) {
-#pragma unroll
-            for (int j = 0; j < 32; j += 4) *reinterpret_cast<float4*>(dst + j) = make_float4(y[j], y[j + 1], y[j + 2], y[j + 3]);
-          } else {
-            for (int j = 0; j < args.N - nb; ++j) dst[j] = y[j];
+          for (int j = 0; j < 16; ++j) {
+            const int n = nb + j;
+            float val = __uint_as_float(v[j]) * a_scale * bf16_to_f32(args.w_norm[n]);
+            if (args.bias) val += bf16_to_f32(args.bias[n]);
+            if (args.epilogue == OQ_EPI_GELU) val = 0.5f * val * (1.0f + erff(val * 0.70710678118654752f));
+            y[j] = val;
           }
-        }
-        if (args.y16) {
-          uint16_t* dst = args.y16 + (size_t)row * args.N + nb;
-          if (full) {
+          if (args.y32) {
+            float4* dst = reinterpret_cast<float4*>(args.y32 + (size_t)row * args.N + nb);
 #pragma unroll
-            for (int j = 0; j < 32; j += 8) {
+            for (int j = 0; j < 16; j += 4) dst[j / 4] = make_float4(y[j], y[j + 1], y[j + 2], y[j + 3]);
+          }
+          if (args.y16) {
+            uint4* dst = reinterpret_cast<uint4*>(args.y16 + (size_t)row * args.N + nb);
+#pragma unroll
+            for (int j = 0; j < 16; j += 8) {
               uint4 p;
               p.x = f32_to_bf16_rn(y[j]) | ((uint32_t)f32_to_bf16_rn(y[j + 1]) << 16);
               p.y = f32_to_bf16_rn(y[j + 2]) | ((uint32_t)f32_to_bf16_rn(y[j + 3]) << 16);
               p.z = f32_to_bf16_rn(y[j + 4]) | ((uint32_t)f32_to_bf16_rn(y[j + 5]) << 16);
               p.w = f32_to_bf16_rn(y[j + 6]) | ((uint32_t)f32_to_bf16_rn(y[j + 7]) << 16);
-              *reinterpret_cast<uint4*>(dst + j) = p;
+              dst[j / 8] = p;
             }
-          } else {
-            for (int j = 0; j < args.N - nb; ++j) dst[j] = f32_to_bf16_rn(y[j]);
           }
-        }
         }
       }
       tc_fence_before();
