@@ -37,9 +37,8 @@
 namespace oq {
 namespace {
 
-constexpr int BM = 128, BN = 256, BK = 64;
+constexpr int BM = 128, BN = 256, BK = 64;  // per-CTA A rows, tile N, K step
 constexpr int PSTAGES = 4;
-constexpr int ESTAGES = 3;
 constexpr int NUM_CONV_WARPS = 16;
 constexpr int NUM_CONV = NUM_CONV_WARPS * 32;
 constexpr int EPI_WARP0 = 16;
@@ -50,7 +49,6 @@ constexpr int TMEM_COLS = 512;
 constexpr unsigned long long kWaitLimitNs = 1000000000ull;
 
 constexpr int EXP_A_BYTES = BM * BK * 2;  // 16 KB
-constexpr int EXP_B_BYTES = BN * BK * 2;  // 32 KB
 
 struct GemmArgs {
   const float* a_norm;
@@ -73,18 +71,26 @@ struct PackedTile {
 };
 
 // ---- shared memory plan (offsets from a 1024-aligned base) -------------------
-template <int BA, int BW>
+// PAIR: two CTAs of a cluster share one 256 x 256 tile (cta_group::2); each holds
+// 128 rows of A and 128 of the 256 B rows.  Otherwise one CTA owns 128 x 256.
+template <int BA, int BW, bool PAIR>
 struct Smem {
+  static constexpr int kBnCta = PAIR ? BN / 2 : BN;
+  static constexpr int kEStages = PAIR ? 5 : 3;
+  static constexpr int kExpBBytes = kBnCta * BK * 2;
   static constexpr int kPkA = BM * PackedTile<BA>::kRowBytes;
-  static constexpr int kPkB = BN * PackedTile<BW>::kRowBytes;
+  static constexpr int kPkB = kBnCta * PackedTile<BW>::kRowBytes;
+  static constexpr int kPkAStride = (kPkA + 127) / 128 * 128;
+  static constexpr int kPkBStride = (kPkB + 127) / 128 * 128;
   static constexpr int kExpA = 0;
-  static constexpr int kExpB = kExpA + ESTAGES * EXP_A_BYTES;
-  static constexpr int kPackA = kExpB + ESTAGES * EXP_B_BYTES;
-  static constexpr int kPackB = kPackA + PSTAGES * ((kPkA + 127) / 128 * 128);
-  static constexpr int kLut = kPackB + PSTAGES * ((kPkB + 127) / 128 * 128);
-  static constexpr int kBars = kLut + 256;
+  static constexpr int kExpB = kExpA + kEStages * EXP_A_BYTES;
+  static constexpr int kPackA = kExpB + kEStages * kExpBBytes;
+  static constexpr int kPackB = kPackA + PSTAGES * kPkAStride;
+  static constexpr int kLut = kPackB + PSTAGES * kPkBStride;
+  static constexpr int kEpi = kLut + 256;                 // 4 warps x (r'[256], bias[256]) floats
+  static constexpr int kBars = kEpi + 4 * 2 * BN * 4;
   // barriers: pk_full[P], pk_empty[P], ex_full[E], ex_empty[E], acc_full[2], acc_empty[2]
-  static constexpr int kNumBars = 2 * PSTAGES + 2 * ESTAGES + 4;
+  static constexpr int kNumBars = 2 * PSTAGES + 2 * kEStages + 4;
   static constexpr int kMisc = kBars + kNumBars * 8;  // tmem base, abort flag
   static constexpr int kTotal = kMisc + 16;
   static constexpr int kAlloc = kTotal + 1024;  // room to align the base
@@ -127,6 +133,53 @@ __device__ bool wait_bounded(uint32_t bar, uint32_t parity, volatile int* abort_
   }
 }
 
+__device__ __forceinline__ bool mbar_try_wait_cluster(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Bounded wait with cluster-scope acquire (barriers that the peer CTA arrives on).
+__device__ bool wait_bounded_cluster(uint32_t bar, uint32_t parity, volatile int* abort_flag, int* status) {
+  if (mbar_try_wait_cluster(bar, parity)) return true;
+  const unsigned long long t0 = global_ns();
+  while (true) {
+    if (mbar_try_wait_cluster(bar, parity)) return true;
+    if (*abort_flag) return false;
+    if (global_ns() - t0 > kWaitLimitNs) {
+      atomicExch(status, OQ_ERR_TIMEOUT);
+      *abort_flag = 1;
+      return false;
+    }
+  }
+}
+
+__device__ __forceinline__ uint32_t cluster_ctarank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+
+// Arrive on the barrier at the same shared offset in CTA `rank` of the cluster.
+// Callers order their shared-memory writes first (fence.proxy.async for data the
+// tensor cores read, tcgen05.fence for TMEM reads); the arrive itself keeps the
+// default semantics, which avoids a cluster-wide memory fence per call.
+__device__ __forceinline__ void mbar_arrive_cluster(uint32_t bar, uint32_t rank) {
+  uint32_t remote;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(bar), "r"(rank));
+  asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(remote) : "memory");
+}
+
+__device__ __forceinline__ void cluster_sync() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
 __device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
   asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
 }
@@ -158,20 +211,46 @@ __device__ __forceinline__ uint64_t umma_desc_sw128(uint32_t addr) {
   return d;
 }
 
-// Instruction descriptor: D f32, A/B f16, both K-major, M = 128, N = 256.
-constexpr uint32_t kIdesc = (1u << 4) | (0u << 7) | (0u << 10) | ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
-
-__device__ __forceinline__ void umma_f16(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem_d),
-      "l"(adesc), "l"(bdesc), "r"(kIdesc), "r"(accumulate)
-      : "memory");
+// Instruction descriptor: D f32, A/B f16, both K-major, N = 256, M = 128 (one CTA)
+// or 256 (CTA pair).
+template <int MMA_M>
+__host__ __device__ constexpr uint32_t idesc_f16() {
+  return (1u << 4) | (0u << 7) | (0u << 10) | ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(MMA_M >> 4) << 24);
 }
 
+template <bool PAIR>
+__device__ __forceinline__ void umma_f16(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uint32_t accumulate) {
+  if constexpr (PAIR) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem_d),
+        "l"(adesc), "l"(bdesc), "r"(idesc_f16<256>()), "r"(accumulate)
+        : "memory");
+  } else {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem_d),
+        "l"(adesc), "l"(bdesc), "r"(idesc_f16<128>()), "r"(accumulate)
+        : "memory");
+  }
+}
+
+// Arrives on `bar` (same offset) in every CTA of the pair, or locally, once all
+// MMAs issued so far by this thread have completed.
+template <bool PAIR>
 __device__ __forceinline__ void umma_commit(uint32_t bar) {
-  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar) : "memory");
+  if constexpr (PAIR) {
+    const uint16_t mask = 0x3;
+    asm volatile(
+        "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(
+            bar),
+        "h"(mask)
+        : "memory");
+  } else {
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar) : "memory");
+  }
 }
 
 __device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
@@ -273,11 +352,15 @@ __device__ __forceinline__ uint16_t f32_to_bf16_rn(float f) {
   return (uint16_t)(u >> 16);
 }
 
-template <int BA, int BW>
+template <int BA, int BW, bool PAIR>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     cbgemm_kernel(const __grid_constant__ GemmArgs args, const __grid_constant__ CUtensorMap map_a,
                   const __grid_constant__ CUtensorMap map_b) {
-  using S = Smem<BA, BW>;
+  using S = Smem<BA, BW, PAIR>;
+  constexpr int ESTAGES = S::kEStages;
+  constexpr int BN_CTA = S::kBnCta;
+  constexpr int TILE_M = PAIR ? 2 * BM : BM;
+  constexpr uint32_t NCTA = PAIR ? 2 : 1;
   extern __shared__ unsigned char smem_raw[];
   unsigned char* smem = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
   const uint32_t sbase = smem_u32(smem);
@@ -288,6 +371,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   uint16_t* lut_w_s = lut_a_s + 64;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = PAIR ? cluster_ctarank() : 0u;   // 0 = leader (issues the MMAs)
+  const int unit = PAIR ? (int)(blockIdx.x >> 1) : (int)blockIdx.x;
+  const int nunits = PAIR ? (int)(gridDim.x >> 1) : (int)gridDim.x;
   auto bar = [&](int i) { return smem_u32(&bars[i]); };
   const int PK_FULL = 0, PK_EMPTY = PSTAGES, EX_FULL = 2 * PSTAGES, EX_EMPTY = 2 * PSTAGES + ESTAGES,
             ACC_FULL = 2 * PSTAGES + 2 * ESTAGES, ACC_EMPTY = ACC_FULL + 2;
@@ -298,12 +384,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       mbar_init(bar(PK_EMPTY + s), NUM_CONV_WARPS);
     }
     for (int s = 0; s < ESTAGES; ++s) {
-      mbar_init(bar(EX_FULL + s), NUM_CONV_WARPS);
+      mbar_init(bar(EX_FULL + s), NUM_CONV_WARPS * NCTA);  // converters of both CTAs
       mbar_init(bar(EX_EMPTY + s), 1);
     }
     for (int s = 0; s < 2; ++s) {
       mbar_init(bar(ACC_FULL + s), 1);
-      mbar_init(bar(ACC_EMPTY + s), 4);
+      mbar_init(bar(ACC_EMPTY + s), 4 * NCTA);            // epilogue warps of both CTAs
     }
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -313,13 +399,20 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     lut_w_s[threadIdx.x] = (uint16_t)(args.lut_w[threadIdx.x >> 1] >> (16 * (threadIdx.x & 1)));
   }
   if (warp == MMA_WARP) {
-    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_holder)),
-                 "r"(TMEM_COLS)
-                 : "memory");
-    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    if constexpr (PAIR) {
+      asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_holder)),
+                   "r"(TMEM_COLS)
+                   : "memory");
+      asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+    } else {
+      asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_holder)),
+                   "r"(TMEM_COLS)
+                   : "memory");
+      asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
   }
   tc_fence_before();
-  __syncthreads();
+  if constexpr (PAIR) cluster_sync(); else __syncthreads();   // barriers initialised in both CTAs
   tc_fence_after();
   const uint32_t tmem_base = *tmem_holder;
 
@@ -331,8 +424,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       constexpr uint32_t bytes = S::kPkA + S::kPkB;
       uint32_t pc = 0;
       bool ok = true;
-      for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
-        const int m0 = (t % args.tiles_m) * BM, n0 = (t / args.tiles_m) * BN;
+      for (int t = unit; t < num_tiles && ok; t += nunits) {
+        const int m0 = (t % args.tiles_m) * TILE_M + (int)rank * BM;
+        const int n0 = (t / args.tiles_m) * BN + (int)rank * BN_CTA;
         for (int kb = 0; kb < KB; ++kb, ++pc) {
           const int s = pc % PSTAGES;
           const uint32_t ph = (pc / PSTAGES) & 1u;
@@ -341,19 +435,18 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             break;
           }
           mbar_arrive_expect_tx(bar(PK_FULL + s), bytes);
-          tma_load_2d(sbase + S::kPackA + s * ((S::kPkA + 127) / 128 * 128), &map_a,
-                      kb * PackedTile<BA>::kRowBytes, m0, bar(PK_FULL + s));
-          tma_load_2d(sbase + S::kPackB + s * ((S::kPkB + 127) / 128 * 128), &map_b,
-                      kb * PackedTile<BW>::kRowBytes, n0, bar(PK_FULL + s));
+          tma_load_2d(sbase + S::kPackA + s * S::kPkAStride, &map_a, kb * PackedTile<BA>::kRowBytes, m0,
+                      bar(PK_FULL + s));
+          tma_load_2d(sbase + S::kPackB + s * S::kPkBStride, &map_b, kb * PackedTile<BW>::kRowBytes, n0,
+                      bar(PK_FULL + s));
         }
       }
     }
   } else if (warp < NUM_CONV_WARPS) {
     // ---- converters ----
-    // Thread ct owns chunk (row, c) = (ct/8 + 64 i, ct % 8) of every stage: A rows
-    // i = 0..1, B rows i = 0..3.  Row & 7 does not depend on i, so each chunk's
-    // swizzled store offset and packed load offset are a per-thread base plus a
-    // compile-time stride.
+    // Thread ct owns chunk (row, c) = (ct/8 + 64 i, ct % 8) of every stage.  Row & 7
+    // does not depend on i, so each chunk's swizzled store offset and packed load
+    // offset are a per-thread base plus a compile-time stride.
     Lut16 ta, tw;
     uint32_t qa0 = args.lut_a[0], qa1 = args.lut_a[1], qw0 = args.lut_w[0], qw1 = args.lut_w[1];
     if constexpr (BA == 4) ta = make_lut16(args.lut_a);
@@ -367,7 +460,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     constexpr int ST_STRIDE = ROWS_PER_PASS / 8 * 1024;             // 8192 bytes
     uint32_t pc = 0;
     bool ok = true;
-    for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
+    for (int t = unit; t < num_tiles && ok; t += nunits) {
       for (int kb = 0; kb < KB; ++kb, ++pc) {
         const int ps = pc % PSTAGES, es = pc % ESTAGES;
         const uint32_t pph = (pc / PSTAGES) & 1u, eph = (pc / ESTAGES) & 1u;
@@ -376,74 +469,92 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           ok = false;
           break;
         }
-        const uint8_t* pa = smem + S::kPackA + ps * ((S::kPkA + 127) / 128 * 128);
-        const uint8_t* pb = smem + S::kPackB + ps * ((S::kPkB + 127) / 128 * 128);
+        const uint8_t* pa = smem + S::kPackA + ps * S::kPkAStride;
+        const uint8_t* pb = smem + S::kPackB + ps * S::kPkBStride;
         unsigned char* ea = smem + S::kExpA + es * EXP_A_BYTES + st_off;
-        unsigned char* eb = smem + S::kExpB + es * EXP_B_BYTES + st_off;
-        uint64_t ra[BM / ROWS_PER_PASS], rb[BN / ROWS_PER_PASS];
+        unsigned char* eb = smem + S::kExpB + es * S::kExpBBytes + st_off;
+        uint64_t ra[BM / ROWS_PER_PASS], rb[BN_CTA / ROWS_PER_PASS];
 #pragma unroll
         for (int i = 0; i < BM / ROWS_PER_PASS; ++i) ra[i] = load_chunk<BA>(pa, ld_a + i * ROWS_PER_PASS * RB_A);
 #pragma unroll
-        for (int i = 0; i < BN / ROWS_PER_PASS; ++i) rb[i] = load_chunk<BW>(pb, ld_b + i * ROWS_PER_PASS * RB_B);
+        for (int i = 0; i < BN_CTA / ROWS_PER_PASS; ++i) rb[i] = load_chunk<BW>(pb, ld_b + i * ROWS_PER_PASS * RB_B);
         __syncwarp();
         if (lane == 0) mbar_arrive(bar(PK_EMPTY + ps));  // packed stage fully read by this warp
 #pragma unroll
         for (int i = 0; i < BM / ROWS_PER_PASS; ++i)
           *reinterpret_cast<uint4*>(ea + i * ST_STRIDE) = expand8<BA>(ra[i], ta, qa0, qa1, lut_a_s);
 #pragma unroll
-        for (int i = 0; i < BN / ROWS_PER_PASS; ++i)
+        for (int i = 0; i < BN_CTA / ROWS_PER_PASS; ++i)
           *reinterpret_cast<uint4*>(eb + i * ST_STRIDE) = expand8<BW>(rb[i], tw, qw0, qw1, lut_w_s);
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
         __syncwarp();
-        if (lane == 0) mbar_arrive(bar(EX_FULL + es));
+        if (lane == 0) {
+          if constexpr (PAIR) mbar_arrive_cluster(bar(EX_FULL + es), 0);  // the leader's barrier
+          else mbar_arrive(bar(EX_FULL + es));
+        }
       }
     }
   } else if (warp == MMA_WARP) {
-    if (lane == 0) {
+    if (lane == 0 && rank == 0) {
       uint32_t ec = 0, lt = 0;
       bool ok = true;
-      for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x, ++lt) {
+      for (int t = unit; t < num_tiles && ok; t += nunits, ++lt) {
         const int acc = lt & 1;
         const uint32_t aph = (lt >> 1) & 1u;
-        if (!wait_bounded(bar(ACC_EMPTY + acc), aph ^ 1u, abort_flag, args.status)) break;
+        const bool got = PAIR ? wait_bounded_cluster(bar(ACC_EMPTY + acc), aph ^ 1u, abort_flag, args.status)
+                              : wait_bounded(bar(ACC_EMPTY + acc), aph ^ 1u, abort_flag, args.status);
+        if (!got) break;
         tc_fence_after();
         const uint32_t tmem_d = tmem_base + (uint32_t)(acc * BN);
         for (int kb = 0; kb < KB; ++kb, ++ec) {
           const int es = ec % ESTAGES;
           const uint32_t eph = (ec / ESTAGES) & 1u;
-          if (!wait_bounded(bar(EX_FULL + es), eph, abort_flag, args.status)) {
+          const bool full = PAIR ? wait_bounded_cluster(bar(EX_FULL + es), eph, abort_flag, args.status)
+                                 : wait_bounded(bar(EX_FULL + es), eph, abort_flag, args.status);
+          if (!full) {
             ok = false;
             break;
           }
           tc_fence_after();
           const uint32_t a_addr = sbase + S::kExpA + es * EXP_A_BYTES;
-          const uint32_t b_addr = sbase + S::kExpB + es * EXP_B_BYTES;
+          const uint32_t b_addr = sbase + S::kExpB + es * S::kExpBBytes;
 #pragma unroll
           for (int k = 0; k < BK / 16; ++k) {
-            umma_f16(tmem_d, umma_desc_sw128(a_addr + 32 * k), umma_desc_sw128(b_addr + 32 * k),
-                     (kb > 0 || k > 0) ? 1u : 0u);
+            umma_f16<PAIR>(tmem_d, umma_desc_sw128(a_addr + 32 * k), umma_desc_sw128(b_addr + 32 * k),
+                           (kb > 0 || k > 0) ? 1u : 0u);
           }
-          umma_commit(bar(EX_EMPTY + es));
+          umma_commit<PAIR>(bar(EX_EMPTY + es));
         }
         if (!ok) break;
-        umma_commit(bar(ACC_FULL + acc));
+        umma_commit<PAIR>(bar(ACC_FULL + acc));
       }
     }
   } else if (warp >= EPI_WARP0 && warp < EPI_WARP0 + 4) {
-    // ---- epilogue ----
+    // ---- epilogue: this CTA's 128 accumulator rows ----
     const int quad = warp & 3;  // TMEM lanes 32*quad .. 32*quad+31
     uint32_t lt = 0;
-    for (int t = blockIdx.x; t < num_tiles; t += gridDim.x, ++lt) {
+    for (int t = unit; t < num_tiles; t += nunits, ++lt) {
       const int acc = lt & 1;
       const uint32_t aph = (lt >> 1) & 1u;
       const bool got = wait_bounded(bar(ACC_FULL + acc), aph, abort_flag, args.status);
       __syncwarp();
       if (__any_sync(0xFFFFFFFFu, !got)) break;
       tc_fence_after();
-      const int m0 = (t % args.tiles_m) * BM, n0 = (t / args.tiles_m) * BN;
+      const int m0 = (t % args.tiles_m) * TILE_M + (int)rank * BM, n0 = (t / args.tiles_m) * BN;
       const int row = m0 + quad * 32 + lane;
       const bool row_ok = row < args.M;
       const float a_scale = row_ok ? args.a_norm[row] * args.inv_d : 0.0f;
+      // this tile's column factors r'_n and bias_n, loaded once per warp
+      float* col_r = reinterpret_cast<float*>(smem + S::kEpi) + quad * 2 * BN;
+      float* col_b = col_r + BN;
+#pragma unroll
+      for (int j = 0; j < BN / 32; ++j) {
+        const int n = n0 + lane + 32 * j;
+        const bool in = n < args.N;
+        col_r[lane + 32 * j] = in ? bf16_to_f32(args.w_norm[n]) : 0.0f;
+        col_b[lane + 32 * j] = (in && args.bias) ? bf16_to_f32(args.bias[n]) : 0.0f;
+      }
+      __syncwarp();
       const uint32_t taddr = tmem_base + ((uint32_t)(quad * 32) << 16) + (uint32_t)(acc * BN);
 #pragma unroll 1
       for (int c0 = 0; c0 < BN; c0 += 16) {
@@ -461,9 +572,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           float y[16];
 #pragma unroll
           for (int j = 0; j < 16; ++j) {
-            const int n = nb + j;
-            float val = __uint_as_float(v[j]) * a_scale * bf16_to_f32(args.w_norm[n]);
-            if (args.bias) val += bf16_to_f32(args.bias[n]);
+            float val = fmaf(__uint_as_float(v[j]) * a_scale, col_r[c0 + j], col_b[c0 + j]);
             if (args.epilogue == OQ_EPI_GELU) val = 0.5f * val * (1.0f + erff(val * 0.70710678118654752f));
             y[j] = val;
           }
@@ -487,17 +596,24 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         }
       }
       tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(bar(ACC_EMPTY + acc));
+      __syncwarp();  // also: every lane is done reading this tile's column factors
+      if (lane == 0) {
+        if constexpr (PAIR) mbar_arrive_cluster(bar(ACC_EMPTY + acc), 0);  // the leader's barrier
+        else mbar_arrive(bar(ACC_EMPTY + acc));
+      }
     }
   }
 
-  // teardown: every role is done (or gave up); release TMEM
+  // teardown: every role of both CTAs is done (or gave up); release TMEM
+  __syncwarp();
   tc_fence_before();
-  __syncthreads();
+  if constexpr (PAIR) cluster_sync(); else __syncthreads();
   tc_fence_after();
   if (warp == MMA_WARP) {
-    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(TMEM_COLS) : "memory");
+    if constexpr (PAIR)
+      asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(TMEM_COLS) : "memory");
+    else
+      asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(TMEM_COLS) : "memory");
   }
 }
 
@@ -537,20 +653,54 @@ int make_code_map(CUtensorMap* map, const void* base, int rows, int row_bytes, i
 
 using GemmKernel = void (*)(GemmArgs, CUtensorMap, CUtensorMap);
 
-template <int BA, int BW>
+template <int BA, int BW, bool PAIR>
 int launch_t(GemmArgs& a, const uint8_t* a_codes, const uint8_t* w_codes, int nsm, cudaStream_t stream) {
+  using S = Smem<BA, BW, PAIR>;
   CUtensorMap ma, mb;
   if (int rc = make_code_map(&ma, a_codes, a.M, a.K * BA / 8, BK * BA / 8, BM)) return rc;
-  if (int rc = make_code_map(&mb, w_codes, a.N, a.K * BW / 8, BK * BW / 8, BN)) return rc;
-  GemmKernel k = cbgemm_kernel<BA, BW>;
-  const int smem = Smem<BA, BW>::kAlloc;
+  if (int rc = make_code_map(&mb, w_codes, a.N, a.K * BW / 8, BK * BW / 8, S::kBnCta)) return rc;
+  GemmKernel k = cbgemm_kernel<BA, BW, PAIR>;
+  const int smem = S::kAlloc;
   cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return fail(OQ_ERR_CUDA, "cudaFuncSetAttribute(GEMM): %s", cudaGetErrorString(e));
-  const int grid = std::min(a.num_tiles, nsm);
-  k<<<grid, NUM_THREADS, smem, stream>>>(a, ma, mb);
-  e = cudaGetLastError();
+  const int tile_m = PAIR ? 2 * BM : BM;
+  a.tiles_m = (a.M + tile_m - 1) / tile_m;
+  a.num_tiles = a.tiles_m * ((a.N + BN - 1) / BN);
+  cudaLaunchConfig_t cfg;
+  memset(&cfg, 0, sizeof(cfg));
+  cudaLaunchAttribute attr[1];
+  cfg.blockDim = dim3(NUM_THREADS, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  int units = std::min(a.num_tiles, nsm);
+  if (PAIR) {
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cfg.gridDim = dim3(2 * std::min(a.num_tiles, nsm / 2), 1, 1);
+    int max_clusters = 0;
+    e = cudaOccupancyMaxActiveClusters(&max_clusters, k, &cfg);
+    if (e != cudaSuccess) return fail(OQ_ERR_CUDA, "cluster occupancy query: %s", cudaGetErrorString(e));
+    if (max_clusters < 1) return fail(OQ_ERR_UNSUPPORTED, "no CTA pair of the GEMM fits on this device");
+    units = std::min(a.num_tiles, max_clusters);
+    cfg.gridDim = dim3(2 * units, 1, 1);
+  } else {
+    cfg.gridDim = dim3(units, 1, 1);
+  }
+  e = cudaLaunchKernelEx(&cfg, k, a, ma, mb);
   if (e != cudaSuccess) return fail(OQ_ERR_CUDA, "GEMM launch: %s", cudaGetErrorString(e));
   return OQ_OK;
+}
+
+template <int BA, int BW>
+int launch_pick(GemmArgs& a, const uint8_t* a_codes, const uint8_t* w_codes, int nsm, cudaStream_t stream) {
+  // CTA pairs halve the operand expansion per tensor-core flop; one CTA suffices
+  // when a single 128-row tile covers M.
+  if (a.M > BM) return launch_t<BA, BW, true>(a, a_codes, w_codes, nsm, stream);
+  return launch_t<BA, BW, false>(a, a_codes, w_codes, nsm, stream);
 }
 
 }  // namespace
@@ -573,8 +723,6 @@ int launch_cbgemm(int d, oq_codebook_t cb_a, oq_codebook_t cb_w, const uint8_t* 
   a.M = M;
   a.N = N;
   a.K = d;
-  a.tiles_m = (M + BM - 1) / BM;
-  a.num_tiles = a.tiles_m * ((N + BN - 1) / BN);
   a.epilogue = epilogue;
   a.inv_d = (float)(1.0 / (double)d);
   for (int i = 0; i < 32; ++i) {
@@ -587,7 +735,7 @@ int launch_cbgemm(int d, oq_codebook_t cb_a, oq_codebook_t cb_w, const uint8_t* 
   cudaStream_t s = (cudaStream_t)stream;
   const int ba = cb_a->bits, bw = cb_w->bits;
 #define OQ_GEMM_CASE(X, Y) \
-  if (ba == X && bw == Y) return launch_t<X, Y>(a, a_codes, w_codes, nsm, s);
+  if (ba == X && bw == Y) return launch_pick<X, Y>(a, a_codes, w_codes, nsm, s);
   OQ_GEMM_CASE(4, 4)
   OQ_GEMM_CASE(4, 2)
   OQ_GEMM_CASE(6, 4)
