@@ -118,17 +118,20 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 
-// Bounded wait; on give-up records the status, raises the CTA abort flag.
+// Bounded wait; on give-up records the status, raises the CTA abort flag.  The
+// clock and the abort flag are read only every 64 polls.
 __device__ bool wait_bounded(uint32_t bar, uint32_t parity, volatile int* abort_flag, int* status) {
   if (mbar_try_wait(bar, parity)) return true;
   const unsigned long long t0 = global_ns();
-  while (true) {
+  for (uint32_t i = 1;; ++i) {
     if (mbar_try_wait(bar, parity)) return true;
-    if (*abort_flag) return false;
-    if (global_ns() - t0 > kWaitLimitNs) {
-      atomicExch(status, OQ_ERR_TIMEOUT);
-      *abort_flag = 1;
-      return false;
+    if ((i & 63u) == 0) {
+      if (*abort_flag) return false;
+      if (global_ns() - t0 > kWaitLimitNs) {
+        atomicExch(status, OQ_ERR_TIMEOUT);
+        *abort_flag = 1;
+        return false;
+      }
     }
   }
 }
@@ -149,13 +152,15 @@ __device__ __forceinline__ bool mbar_try_wait_cluster(uint32_t bar, uint32_t par
 __device__ bool wait_bounded_cluster(uint32_t bar, uint32_t parity, volatile int* abort_flag, int* status) {
   if (mbar_try_wait_cluster(bar, parity)) return true;
   const unsigned long long t0 = global_ns();
-  while (true) {
+  for (uint32_t i = 1;; ++i) {
     if (mbar_try_wait_cluster(bar, parity)) return true;
-    if (*abort_flag) return false;
-    if (global_ns() - t0 > kWaitLimitNs) {
-      atomicExch(status, OQ_ERR_TIMEOUT);
-      *abort_flag = 1;
-      return false;
+    if ((i & 63u) == 0) {
+      if (*abort_flag) return false;
+      if (global_ns() - t0 > kWaitLimitNs) {
+        atomicExch(status, OQ_ERR_TIMEOUT);
+        *abort_flag = 1;
+        return false;
+      }
     }
   }
 }
@@ -262,6 +267,23 @@ __device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
   return d;
 }
 
+__device__ __forceinline__ uint32_t lds_u32(uint32_t addr) {
+  uint32_t v;
+  asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(addr));
+  return v;
+}
+
+__device__ __forceinline__ uint32_t lds_u16(uint32_t addr) {
+  uint16_t v;
+  asm volatile("ld.shared.u16 %0, [%1];" : "=h"(v) : "r"(addr));
+  return v;
+}
+
+__device__ __forceinline__ void sts_v4(uint32_t addr, uint4 v) {
+  asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
+               : "memory");
+}
+
 // ---- code -> fp16 expansion ---------------------------------------------------
 // A 16-entry fp16 table as byte planes: lo[q] holds the low bytes of entries
 // 4q..4q+3, hi[q] the high bytes.
@@ -293,7 +315,7 @@ __device__ __forceinline__ void expand4_nib(uint32_t x, const Lut16& t, uint32_t
 // Eight codes -> uint4 of eight fp16 (element 0 in the low half of .x).
 template <int BITS>
 __device__ __forceinline__ uint4 expand8(uint64_t packed, const Lut16& t16, uint32_t q0, uint32_t q1,
-                                         const uint16_t* lut_smem) {
+                                         uint32_t lut_smem) {
   uint4 r;
   if constexpr (BITS == 4) {
     const uint32_t w = (uint32_t)packed;
@@ -316,25 +338,25 @@ __device__ __forceinline__ uint4 expand8(uint64_t packed, const Lut16& t16, uint
     for (int i = 0; i < 4; ++i) {
       const uint32_t c0 = (uint32_t)(packed >> (12 * i)) & 63u;
       const uint32_t c1 = (uint32_t)(packed >> (12 * i + 6)) & 63u;
-      o[i] = (uint32_t)lut_smem[c0] | ((uint32_t)lut_smem[c1] << 16);
+      o[i] = lds_u16(lut_smem + 2 * c0) | (lds_u16(lut_smem + 2 * c1) << 16);
     }
     r = make_uint4(o[0], o[1], o[2], o[3]);
   }
   return r;
 }
 
-// Eight packed codes starting at byte offset `off` of a packed tile (8*BITS bits).
+// Eight packed codes starting at shared address `addr` (8*BITS bits).
 template <int BITS>
-__device__ __forceinline__ uint64_t load_chunk(const uint8_t* tile, int off) {
+__device__ __forceinline__ uint64_t load_chunk(uint32_t addr) {
   if constexpr (BITS == 4) {
-    return *reinterpret_cast<const uint32_t*>(tile + off);
+    return lds_u32(addr);
   } else if constexpr (BITS == 2) {
-    return *reinterpret_cast<const uint16_t*>(tile + off);
+    return lds_u16(addr);
   } else {
-    const int base = off & ~3;
-    const uint64_t lo = *reinterpret_cast<const uint32_t*>(tile + base);
-    const uint64_t hi = *reinterpret_cast<const uint32_t*>(tile + base + 4);
-    return ((hi << 32) | lo) >> (8 * (off - base));
+    const uint32_t base = addr & ~3u;
+    const uint64_t lo = lds_u32(base);
+    const uint64_t hi = lds_u32(base + 4);
+    return ((hi << 32) | lo) >> (8 * (addr - base));
   }
 }
 
@@ -345,11 +367,11 @@ __device__ __forceinline__ uint32_t sw128_offset(int row, int c) {
 
 __device__ __forceinline__ float bf16_to_f32(uint16_t v) { return __uint_as_float((uint32_t)v << 16); }
 
-__device__ __forceinline__ uint16_t f32_to_bf16_rn(float f) {
-  uint32_t u = __float_as_uint(f);
-  if ((u & 0x7F800000u) == 0x7F800000u) return (uint16_t)((u >> 16) | ((u & 0xFFFFu) ? 0x40u : 0u));
-  u += 0x7FFFu + ((u >> 16) & 1u);
-  return (uint16_t)(u >> 16);
+// Two floats -> bf16x2 (lo in the low half), round to nearest even.
+__device__ __forceinline__ uint32_t bf16x2_rn(float lo, float hi) {
+  uint32_t r;
+  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
 }
 
 template <int BA, int BW, bool PAIR>
@@ -469,23 +491,22 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           ok = false;
           break;
         }
-        const uint8_t* pa = smem + S::kPackA + ps * S::kPkAStride;
-        const uint8_t* pb = smem + S::kPackB + ps * S::kPkBStride;
-        unsigned char* ea = smem + S::kExpA + es * EXP_A_BYTES + st_off;
-        unsigned char* eb = smem + S::kExpB + es * S::kExpBBytes + st_off;
+        const uint32_t pa = sbase + S::kPackA + ps * S::kPkAStride + ld_a;
+        const uint32_t pb = sbase + S::kPackB + ps * S::kPkBStride + ld_b;
+        const uint32_t ea = sbase + S::kExpA + es * EXP_A_BYTES + st_off;
+        const uint32_t eb = sbase + S::kExpB + es * S::kExpBBytes + st_off;
         uint64_t ra[BM / ROWS_PER_PASS], rb[BN_CTA / ROWS_PER_PASS];
 #pragma unroll
-        for (int i = 0; i < BM / ROWS_PER_PASS; ++i) ra[i] = load_chunk<BA>(pa, ld_a + i * ROWS_PER_PASS * RB_A);
+        for (int i = 0; i < BM / ROWS_PER_PASS; ++i) ra[i] = load_chunk<BA>(pa + i * ROWS_PER_PASS * RB_A);
 #pragma unroll
-        for (int i = 0; i < BN_CTA / ROWS_PER_PASS; ++i) rb[i] = load_chunk<BW>(pb, ld_b + i * ROWS_PER_PASS * RB_B);
+        for (int i = 0; i < BN_CTA / ROWS_PER_PASS; ++i) rb[i] = load_chunk<BW>(pb + i * ROWS_PER_PASS * RB_B);
         __syncwarp();
         if (lane == 0) mbar_arrive(bar(PK_EMPTY + ps));  // packed stage fully read by this warp
 #pragma unroll
-        for (int i = 0; i < BM / ROWS_PER_PASS; ++i)
-          *reinterpret_cast<uint4*>(ea + i * ST_STRIDE) = expand8<BA>(ra[i], ta, qa0, qa1, lut_a_s);
+        for (int i = 0; i < BM / ROWS_PER_PASS; ++i) sts_v4(ea + i * ST_STRIDE, expand8<BA>(ra[i], ta, qa0, qa1, sbase + S::kLut));
 #pragma unroll
         for (int i = 0; i < BN_CTA / ROWS_PER_PASS; ++i)
-          *reinterpret_cast<uint4*>(eb + i * ST_STRIDE) = expand8<BW>(rb[i], tw, qw0, qw1, lut_w_s);
+          sts_v4(eb + i * ST_STRIDE, expand8<BW>(rb[i], tw, qw0, qw1, sbase + S::kLut + 128));
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
         __syncwarp();
         if (lane == 0) {
@@ -586,10 +607,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 #pragma unroll
             for (int j = 0; j < 16; j += 8) {
               uint4 p;
-              p.x = f32_to_bf16_rn(y[j]) | ((uint32_t)f32_to_bf16_rn(y[j + 1]) << 16);
-              p.y = f32_to_bf16_rn(y[j + 2]) | ((uint32_t)f32_to_bf16_rn(y[j + 3]) << 16);
-              p.z = f32_to_bf16_rn(y[j + 4]) | ((uint32_t)f32_to_bf16_rn(y[j + 5]) << 16);
-              p.w = f32_to_bf16_rn(y[j + 6]) | ((uint32_t)f32_to_bf16_rn(y[j + 7]) << 16);
+              p.x = bf16x2_rn(y[j], y[j + 1]);
+              p.y = bf16x2_rn(y[j + 2], y[j + 3]);
+              p.z = bf16x2_rn(y[j + 4], y[j + 5]);
+              p.w = bf16x2_rn(y[j + 6], y[j + 7]);
               dst[j / 8] = p;
             }
           }
