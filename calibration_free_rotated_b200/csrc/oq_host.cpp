@@ -207,6 +207,61 @@ uint16_t double_to_fp16_rne(double v) {
 }
 
 // ---------------------------------------------------------------------------
+// Bucket table for the rotate+quantize kernel's centroid search.
+//
+// The kernel forms t (fp32) and y = fma(t, G, C) with C = 1.5*2^23 + off0, so
+// y's low mantissa bits hold q = round(t*G + off0) exactly (one rounding of the
+// exact t*G + C).  Bucket q covers z = t*G + off0 in [q - 1/2, q + 1/2).  G is
+// chosen so that consecutive fp32 boundaries are >= 1.25 buckets apart (at most
+// one boundary per bucket) and no boundary lies within 0.02 bucket of a bucket
+// edge (so a t that rounds to either neighbour at an edge gets the same answer).
+// Entry q: the boundary inside the bucket (or 3e38 if none) with its low b
+// mantissa bits replaced by base_q = #{boundaries below the bucket}; the code
+// is (entry & (2^b - 1)) + (t > entry).  Replacing those bits moves a threshold
+// by fewer than 2^b fp32 ulps (< 4e-6 relative), far inside the 1e-5 boundary
+// band of the parity rule.
+// ---------------------------------------------------------------------------
+void build_qtable(oq_codebook_t cb) {
+  const int L = 1 << cb->bits;
+  std::vector<float> b32(L - 1);
+  for (int k = 0; k < L - 1; ++k) b32[k] = (float)cb->bounds[k];
+  double min_gap = 2.0;
+  for (int k = 0; k + 1 < L - 1; ++k) min_gap = std::fmin(min_gap, (double)b32[k + 1] - (double)b32[k]);
+  float G = (float)(1.25 / min_gap);
+  if (L == 2) G = 4.0f;
+  double off0 = 0.0;
+  for (int attempt = 0; attempt < 100000; ++attempt) {
+    off0 = std::ceil((double)G * 1.001) + 2.0;
+    bool ok = true;
+    for (int k = 0; k < L - 1 && ok; ++k) {
+      const double z = (double)b32[k] * (double)G + off0;
+      const double f = z - std::floor(z);
+      if (std::fabs(f - 0.5) < 0.02) ok = false;
+    }
+    if (ok) break;
+    G = (float)((double)G * 1.0007);
+  }
+  const int Q = 2 * (int)off0 + 2;
+  cb->qtable.assign(Q, 0u);
+  const uint32_t lowmask = (uint32_t)L - 1u;
+  for (int q = 0; q < Q; ++q) {
+    const double lo = q - 0.5, hi = q + 0.5;
+    uint32_t base = 0;
+    float thr = 3.0e38f;
+    for (int k = 0; k < L - 1; ++k) {
+      const double z = (double)b32[k] * (double)G + off0;
+      if (z < lo) ++base;
+      else if (z < hi) thr = b32[k];
+    }
+    uint32_t bits;
+    std::memcpy(&bits, &thr, 4);
+    cb->qtable[q] = (bits & ~lowmask) | base;
+  }
+  cb->qt_scale = G;
+  cb->qt_offset = (float)(12582912.0 + off0);  // 1.5 * 2^23 + off0, exact in fp32
+}
+
+// ---------------------------------------------------------------------------
 // Device state
 // ---------------------------------------------------------------------------
 static std::mutex g_dev_mu;
@@ -276,6 +331,25 @@ static int upload_rpbh(oq_rpbh_t r, int dev) {
   }
   r->dev_perm[dev] = dp;
   r->dev_signs[dev] = ds;
+  return OQ_OK;
+}
+
+int codebook_device_qtable(oq_codebook_t cb, const uint32_t** qtable) {
+  int dev;
+  if (int rc = current_device(&dev)) return rc;
+  std::lock_guard<std::mutex> lk(cb->mu);
+  if (!cb->dev_qtable[dev]) {
+    uint32_t* p = nullptr;
+    const size_t bytes = sizeof(uint32_t) * cb->qtable.size();
+    cudaError_t e = cudaMalloc(&p, bytes);
+    if (e == cudaSuccess) e = cudaMemcpy(p, cb->qtable.data(), bytes, cudaMemcpyHostToDevice);
+    if (e != cudaSuccess) {
+      cudaFree(p);
+      return fail(OQ_ERR_CUDA, "uploading the search table: %s", cudaGetErrorString(e));
+    }
+    cb->dev_qtable[dev] = p;
+  }
+  *qtable = cb->dev_qtable[dev];
   return OQ_OK;
 }
 
@@ -405,6 +479,18 @@ int oq_build_codebook(int d, int bits, oq_codebook_t* out) {
   cb->lut.resize(cb->centroids.size());
   const double sd = std::sqrt((double)d);
   for (size_t k = 0; k < cb->centroids.size(); ++k) cb->lut[k] = double_to_fp16_rne(sd * cb->centroids[k]);
+  build_qtable(cb);
+  // Upload the search table to the current device now when one is present.
+  int ndev = 0;
+  if (cudaGetDeviceCount(&ndev) == cudaSuccess && ndev > 0) {
+    const uint32_t* t;
+    if (int rc = codebook_device_qtable(cb, &t)) {
+      delete cb;
+      return rc;
+    }
+  } else {
+    cudaGetLastError();
+  }
   *out = cb;
   return OQ_OK;
 }
@@ -429,7 +515,17 @@ int oq_codebook_export(oq_codebook_t cb, double* centroids, double* bounds, uint
   return OQ_OK;
 }
 
-void oq_free_codebook(oq_codebook_t cb) { delete cb; }
+void oq_free_codebook(oq_codebook_t cb) {
+  if (!cb) return;
+  int prev = -1;
+  bool have_prev = cudaGetDevice(&prev) == cudaSuccess;
+  for (int dev = 0; dev < OQ_MAX_DEVICES; ++dev) {
+    if (!cb->dev_qtable[dev]) continue;
+    if (cudaSetDevice(dev) == cudaSuccess) cudaFree(cb->dev_qtable[dev]);
+  }
+  if (have_prev) cudaSetDevice(prev);
+  delete cb;
+}
 
 static int check_quant_args(oq_rpbh_t r, oq_codebook_t cb, const void* X, int M, const void* codes,
                             const void* norms) {

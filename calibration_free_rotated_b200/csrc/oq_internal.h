@@ -28,6 +28,11 @@ struct oq_codebook_s {
   std::vector<uint16_t> lut;      // fp16 bits of RNE(sqrt(d) c_k)
   int iterations = 0;
   double distortion = 0.0;
+  // Bucket table for the branchless centroid search (see oq_host.cpp).
+  float qt_scale = 0.0f, qt_offset = 0.0f;
+  std::vector<uint32_t> qtable;
+  std::mutex mu;
+  uint32_t* dev_qtable[OQ_MAX_DEVICES] = {};
 };
 
 namespace oq {
@@ -45,6 +50,8 @@ uint16_t double_to_fp16_rne(double v);
 // Device-side state (oq_host.cpp).
 int current_device(int* dev);
 int rpbh_device_tables(oq_rpbh_t r, const uint16_t** perm, const uint32_t** signs);
+int codebook_device_qtable(oq_codebook_t cb, const uint32_t** qtable);
+void build_qtable(oq_codebook_t cb);
 int device_status_word(int** status);
 int device_status_word_if_present(int** status);  // never allocates
 int sm_count(int* n);

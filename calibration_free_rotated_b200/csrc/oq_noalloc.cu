@@ -61,6 +61,9 @@ extern "C" int oq_linear_noalloc(oq_rpbh_t r, oq_codebook_t cb_a, oq_codebook_t 
   if (!r->dev_perm[dev])
     return oq::fail(OQ_ERR_ARG, "the RPBH handle has no tables on device %d: create it with that device current",
                     dev);
+  if (!cb_a->dev_qtable[dev])
+    return oq::fail(OQ_ERR_ARG,
+                    "the activation codebook has no tables on device %d: build it with that device current", dev);
   int* status = nullptr;
   if (oq::device_status_word_if_present(&status) != OQ_OK)
     return oq::fail(OQ_ERR_ARG,
