@@ -7,24 +7,30 @@
 // computed here as  acc = sum_k LUT_a[ca] LUT_w[cw]  (fp16 operands,
 // LUT = fp16(sqrt(d) c)), y = acc * s_m * r'_n / d + bias_n, optional GELU.
 //
-// sm_100a design (one CTA per SM, persistent over 128 x 256 output tiles):
-//   warp 20      TMA producer: 2-D tensor copies of the packed code tiles
-//                (A: 128 rows, B: 256 rows, 64 codes of K each) into a
-//                4-deep packed ring.
-//   warps 0..15  converters: expand codes through the fp16 LUT (register
-//                byte-permute tables for 2 and 4 bits, a 128-byte shared
-//                table for 6 bits) straight into the canonical K-major
-//                128-byte-swizzled UMMA layout of a 3-deep expanded ring.
-//   warp 21      one thread issues tcgen05.mma (kind::f16, M=128, N=256,
-//                K=16, fp32 accumulate in TMEM); tcgen05.commit frees ring
-//                stages and publishes finished accumulators.
-//   warps 16..19 epilogue: tcgen05.ld of the accumulator (each warp its
-//                32-lane quadrant), rescale, bias, GELU, fp32/bf16 stores.
-// TMEM holds two 128 x 256 fp32 accumulators (all 512 columns) so the
-// epilogue of one tile overlaps the main loop of the next.  Every mbarrier
-// wait is bounded (~1 s); a wait that gives up records OQ_ERR_TIMEOUT,
-// raises an abort flag that makes every role skip its remaining work, and
-// the CTA still reaches its teardown (TMEM is always released).
+// sm_100a design (persistent; tiles of 256 x 256 shared by a CTA pair of a
+// cluster with tcgen05 cta_group::2, or 128 x 256 on one CTA when M <= 128):
+//   warp 20      TMA producer: 2-D tensor copies of the packed code tiles into a
+//                4-deep packed ring (each CTA: 128 rows of A, its B rows).
+//   warps 0..7   A converters: expand activation codes through the fp16 LUT and
+//                write them straight into TMEM with tcgen05.st (warp w owns TMEM
+//                lanes 32 (w % 4) .. +31 = its tile rows, half of K each).
+//   warps 8..15  B converters: expand weight codes into the canonical K-major
+//                128-byte-swizzled UMMA layout in shared memory.
+//                (Both use register byte-permute tables for 2 and 4 bits and a
+//                128-byte shared table for 6 bits.)
+//   warp 21      one thread of the leader CTA issues tcgen05.mma (kind::f16,
+//                A from TMEM, B from shared memory, M = 256 across the pair,
+//                N = 256, K = 16, fp32 accumulate in TMEM); tcgen05.commit
+//                (multicast to both CTAs) frees ring stages and publishes the
+//                finished accumulator.
+//   warps 16..19 epilogue: tcgen05.ld of the accumulator (each warp its 32-lane
+//                quadrant), rescale, bias, GELU, fp32/bf16 stores.
+// Keeping A in TMEM removes A's expanded stores and tensor-core reads from
+// shared memory, whose bandwidth otherwise caps the kernel near 2/3 of the
+// tensor rate.  TMEM: one 256-column fp32 accumulator plus 4 A stages of 32
+// columns.  Every mbarrier wait is bounded (~1 s); a wait that gives up records
+// OQ_ERR_TIMEOUT, raises an abort flag that makes every role skip its remaining
+// work, and the CTA still reaches its teardown (TMEM is always released).
 #include <cuda.h>
 #include <cuda_runtime.h>
 
@@ -38,17 +44,18 @@ namespace oq {
 namespace {
 
 constexpr int BM = 128, BN = 256, BK = 64;  // per-CTA A rows, tile N, K step
-constexpr int PSTAGES = 4;
-constexpr int NUM_CONV_WARPS = 16;
-constexpr int NUM_CONV = NUM_CONV_WARPS * 32;
+constexpr int PSTAGES = 4;                   // packed-code ring
+constexpr int ESTAGES = 4;                   // expanded ring (A in TMEM, B in shared memory)
+constexpr int NUM_A_WARPS = 8;               // warps 0..7
+constexpr int NUM_B_WARPS = 8;               // warps 8..15
+constexpr int NUM_CONV_WARPS = NUM_A_WARPS + NUM_B_WARPS;
 constexpr int EPI_WARP0 = 16;
 constexpr int TMA_WARP = 20;
 constexpr int MMA_WARP = 21;
 constexpr int NUM_THREADS = 22 * 32;
 constexpr int TMEM_COLS = 512;
+constexpr int A_COL0 = BN;                   // A stage s: TMEM columns A_COL0 + 32 s .. + 31
 constexpr unsigned long long kWaitLimitNs = 1000000000ull;
-
-constexpr int EXP_A_BYTES = BM * BK * 2;  // 16 KB
 
 struct GemmArgs {
   const float* a_norm;
@@ -76,24 +83,26 @@ struct PackedTile {
 template <int BA, int BW, bool PAIR>
 struct Smem {
   static constexpr int kBnCta = PAIR ? BN / 2 : BN;
-  static constexpr int kEStages = PAIR ? 5 : 3;
   static constexpr int kExpBBytes = kBnCta * BK * 2;
   static constexpr int kPkA = BM * PackedTile<BA>::kRowBytes;
   static constexpr int kPkB = kBnCta * PackedTile<BW>::kRowBytes;
   static constexpr int kPkAStride = (kPkA + 127) / 128 * 128;
   static constexpr int kPkBStride = (kPkB + 127) / 128 * 128;
-  static constexpr int kExpA = 0;
-  static constexpr int kExpB = kExpA + kEStages * EXP_A_BYTES;
-  static constexpr int kPackA = kExpB + kEStages * kExpBBytes;
+  static constexpr int kExpB = 0;
+  static constexpr int kPackA = kExpB + ESTAGES * kExpBBytes;
   static constexpr int kPackB = kPackA + PSTAGES * kPkAStride;
   static constexpr int kLut = kPackB + PSTAGES * kPkBStride;
   static constexpr int kEpi = kLut + 256;                 // 4 warps x (r'[256], bias[256]) floats
   static constexpr int kBars = kEpi + 4 * 2 * BN * 4;
-  // barriers: pk_full[P], pk_empty[P], ex_full[E], ex_empty[E], acc_full[2], acc_empty[2]
-  static constexpr int kNumBars = 2 * PSTAGES + 2 * kEStages + 4;
+  // barriers: pk_full[P], pk_empty[P], ex_full[E], ex_empty[E], acc_full, acc_empty
+  static constexpr int kNumBars = 2 * PSTAGES + 2 * ESTAGES + 2;
   static constexpr int kMisc = kBars + kNumBars * 8;  // tmem base, abort flag
   static constexpr int kTotal = kMisc + 16;
-  static constexpr int kAlloc = kTotal + 1024;  // room to align the base
+  // Room to align the base, and never less than half an SM's shared memory:
+  // the kernel allocates all 512 TMEM columns, so a second resident CTA would
+  // wait in tcgen05.alloc for the first one to finish.
+  static constexpr int kMinAlloc = 120 * 1024;
+  static constexpr int kAlloc = kTotal + 1024 > kMinAlloc ? kTotal + 1024 : kMinAlloc;
 };
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
@@ -224,20 +233,20 @@ __host__ __device__ constexpr uint32_t idesc_f16() {
 }
 
 template <bool PAIR>
-__device__ __forceinline__ void umma_f16(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uint32_t accumulate) {
+__device__ __forceinline__ void umma_f16_ts(uint32_t tmem_d, uint32_t tmem_a, uint64_t bdesc, uint32_t accumulate) {
   if constexpr (PAIR) {
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
         "setp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem_d),
-        "l"(adesc), "l"(bdesc), "r"(idesc_f16<256>()), "r"(accumulate)
+        "tcgen05.mma.cta_group::2.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(tmem_d),
+        "r"(tmem_a), "l"(bdesc), "r"(idesc_f16<256>()), "r"(accumulate)
         : "memory");
   } else {
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
         "setp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem_d),
-        "l"(adesc), "l"(bdesc), "r"(idesc_f16<128>()), "r"(accumulate)
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(tmem_d),
+        "r"(tmem_a), "l"(bdesc), "r"(idesc_f16<128>()), "r"(accumulate)
         : "memory");
   }
 }
@@ -285,51 +294,88 @@ __device__ __forceinline__ void sts_v4(uint32_t addr, uint4 v) {
 }
 
 // ---- code -> fp16 expansion ---------------------------------------------------
-// A 16-entry fp16 table as byte planes: lo[q] holds the low bytes of entries
-// 4q..4q+3, hi[q] the high bytes.
-struct Lut16 {
-  uint32_t lo[4], hi[4];
+// The codebooks are odd: entry 2^b-1-k is entry k with the sign bit flipped
+// (the host checks this bit pattern before launch). A 4-bit code n is therefore
+// the magnitude entry m = n (n < 8) or m = 15 - n (n >= 8) of the eight
+// negative entries 0..7, negated when n >= 8. The magnitude tables are byte
+// planes: lo0/hi0 hold the low/high bytes of entries 0..3, lo1/hi1 of 4..7.
+struct Lut8 {
+  uint32_t lo0, lo1, hi0, hi1;
 };
 
-__device__ __forceinline__ Lut16 make_lut16(const uint32_t* words) {
-  Lut16 t;
-#pragma unroll
-  for (int q = 0; q < 4; ++q) {
-    const uint32_t w0 = words[2 * q], w1 = words[2 * q + 1];  // entries 4q..4q+3
-    t.lo[q] = prmt(w0, w1, 0x6420);
-    t.hi[q] = prmt(w0, w1, 0x7531);
-  }
+__device__ __forceinline__ Lut8 make_lut8(const uint32_t* words) {
+  Lut8 t;
+  t.lo0 = prmt(words[0], words[1], 0x6420);
+  t.hi0 = prmt(words[0], words[1], 0x7531);
+  t.lo1 = prmt(words[2], words[3], 0x6420);
+  t.hi1 = prmt(words[2], words[3], 0x7531);
   return t;
 }
 
-// Four 4-bit codes (x bits 0..15) -> two fp16x2 words.
-__device__ __forceinline__ void expand4_nib(uint32_t x, const Lut16& t, uint32_t& w0, uint32_t& w1) {
-  const uint32_t sel = x & 0x7777u;                         // entry within a group of 8
-  const uint32_t sel2 = ((x >> 1) & 0x4444u) | 0x3210u;     // which group (bit 3)
-  const uint32_t lo = prmt(prmt(t.lo[0], t.lo[1], sel), prmt(t.lo[2], t.lo[3], sel), sel2);
-  const uint32_t hi = prmt(prmt(t.hi[0], t.hi[1], sel), prmt(t.hi[2], t.hi[3], sel), sel2);
-  w0 = prmt(lo, hi, 0x5140);
-  w1 = prmt(lo, hi, 0x7362);
+// x >> s for a constant s, on the IMAD pipe (which issues alongside the ALU pipe
+// that byte-permutes and logic ops share): high word of x * 2^(32-s).
+template <int S>
+__device__ __forceinline__ uint32_t shr_imad(uint32_t x) {
+  uint32_t r;
+  asm("mul.hi.u32 %0, %1, %2;" : "=r"(r) : "r"(x), "r"(1u << (32 - S)));
+  return r;
+}
+
+__device__ __forceinline__ uint32_t mul_lo(uint32_t x, uint32_t y) {
+  uint32_t r;
+  asm("mul.lo.u32 %0, %1, %2;" : "=r"(r) : "r"(x), "r"(y));
+  return r;
+}
+
+__device__ __forceinline__ uint32_t mul_hi(uint32_t x, uint32_t y) {
+  uint32_t r;
+  asm("mul.hi.u32 %0, %1, %2;" : "=r"(r) : "r"(x), "r"(y));
+  return r;
+}
+
+// Eight 4-bit codes (nibble i of x is code i) -> four fp16x2 words.
+// ALU: 14 ops (byte permutes and logic); 3 multiplies go to the IMAD pipe.
+__device__ __forceinline__ uint4 expand8_nib(uint32_t x, const Lut8& t) {
+  const uint32_t xs = x & 0x88888888u;                           // bit 3 of every code
+  const uint32_t sel = (x ^ mul_hi(xs, 0xE0000000u)) & 0x77777777u;  // m: n ^ 7 where bit 3 is set
+  const uint32_t x4 = mul_lo(x, 16u);  // bit 3 of codes 0, 2, 4, 6 at bit 7 of a byte
+  uint4 r;
+  {
+    const uint32_t lo = prmt(t.lo0, t.lo1, sel);
+    const uint32_t sg = prmt(x4, x, 0xD9C8u);  // 0xFF in byte i where code i >= 8
+    const uint32_t hi = prmt(t.hi0, t.hi1, sel) ^ (sg & 0x80808080u);
+    r.x = prmt(lo, hi, 0x5140u);
+    r.y = prmt(lo, hi, 0x7362u);
+  }
+  {
+    const uint32_t s2 = shr_imad<16>(sel);
+    const uint32_t lo = prmt(t.lo0, t.lo1, s2);
+    const uint32_t sg = prmt(x4, x, 0xFBEAu);  // codes 4..7
+    const uint32_t hi = prmt(t.hi0, t.hi1, s2) ^ (sg & 0x80808080u);
+    r.z = prmt(lo, hi, 0x5140u);
+    r.w = prmt(lo, hi, 0x7362u);
+  }
+  return r;
 }
 
 // Eight codes -> uint4 of eight fp16 (element 0 in the low half of .x).
 template <int BITS>
-__device__ __forceinline__ uint4 expand8(uint64_t packed, const Lut16& t16, uint32_t q0, uint32_t q1,
+__device__ __forceinline__ uint4 expand8(uint64_t packed, const Lut8& t8, uint32_t q0, uint32_t q1,
                                          uint32_t lut_smem) {
   uint4 r;
   if constexpr (BITS == 4) {
-    const uint32_t w = (uint32_t)packed;
-    expand4_nib(w & 0xFFFFu, t16, r.x, r.y);
-    expand4_nib(w >> 16, t16, r.z, r.w);
+    r = expand8_nib((uint32_t)packed, t8);
   } else if constexpr (BITS == 2) {
-    // selector bytes (2c0, 2c0+1, 2c1, 2c1+1) pick two fp16 from the 4-entry table {q1:q0}
+    // Selector nibbles (2c0, 2c0+1, 2c1, 2c1+1) pick two fp16 from the 4-entry table
+    // {q1:q0}.  With z = c0 + 4 c1: sel = 0x1010 + 0x22 z + 0x2178 c1 (no carries
+    // into bit 16; the byte permute reads only the low 16 bits of its selector).
     const uint32_t w = (uint32_t)packed;
     uint32_t o[4];
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-      const uint32_t z = (w >> (4 * i)) & 0xFu;
-      const uint32_t sel = 0x1010u + (z & 3u) * 0x22u + (z & 0xCu) * 0x880u;
-      o[i] = prmt(q0, q1, sel);
+      const uint32_t z = (i == 0 ? w : shr_imad<4>(i == 1 ? w : (i == 2 ? shr_imad<4>(w) : shr_imad<8>(w)))) & 0xFu;
+      const uint32_t c1 = shr_imad<2>(z);
+      o[i] = prmt(q0, q1, c1 * 0x2178u + (z * 0x22u + 0x1010u));
     }
     r = make_uint4(o[0], o[1], o[2], o[3]);
   } else {  // 6 bits: shared 64-entry table
@@ -374,12 +420,32 @@ __device__ __forceinline__ uint32_t bf16x2_rn(float lo, float hi) {
   return r;
 }
 
+// Stores 16 consecutive 32-bit TMEM columns of this thread's lane.
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&v)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
+      "%15, %16};" ::"r"(taddr),
+      "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]), "r"(v[8]), "r"(v[9]),
+      "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15])
+      : "memory");
+}
+
+// Loads 16 consecutive 32-bit TMEM columns of this thread's lane (complete
+// after tcgen05.wait::ld).
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t* v) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, "
+      "%14, %15}, [%16];"
+      : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7]), "=r"(v[8]),
+        "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]), "=r"(v[15])
+      : "r"(taddr));
+}
+
 template <int BA, int BW, bool PAIR>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     cbgemm_kernel(const __grid_constant__ GemmArgs args, const __grid_constant__ CUtensorMap map_a,
                   const __grid_constant__ CUtensorMap map_b) {
   using S = Smem<BA, BW, PAIR>;
-  constexpr int ESTAGES = S::kEStages;
   constexpr int BN_CTA = S::kBnCta;
   constexpr int TILE_M = PAIR ? 2 * BM : BM;
   constexpr uint32_t NCTA = PAIR ? 2 : 1;
@@ -398,7 +464,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   const int nunits = PAIR ? (int)(gridDim.x >> 1) : (int)gridDim.x;
   auto bar = [&](int i) { return smem_u32(&bars[i]); };
   const int PK_FULL = 0, PK_EMPTY = PSTAGES, EX_FULL = 2 * PSTAGES, EX_EMPTY = 2 * PSTAGES + ESTAGES,
-            ACC_FULL = 2 * PSTAGES + 2 * ESTAGES, ACC_EMPTY = ACC_FULL + 2;
+            ACC_FULL = 2 * PSTAGES + 2 * ESTAGES, ACC_EMPTY = ACC_FULL + 1;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < PSTAGES; ++s) {
@@ -409,10 +475,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       mbar_init(bar(EX_FULL + s), NUM_CONV_WARPS * NCTA);  // converters of both CTAs
       mbar_init(bar(EX_EMPTY + s), 1);
     }
-    for (int s = 0; s < 2; ++s) {
-      mbar_init(bar(ACC_FULL + s), 1);
-      mbar_init(bar(ACC_EMPTY + s), 4 * NCTA);            // epilogue warps of both CTAs
-    }
+    mbar_init(bar(ACC_FULL), 1);
+    mbar_init(bar(ACC_EMPTY), 4 * NCTA);                   // epilogue warps of both CTAs
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
@@ -464,46 +528,92 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         }
       }
     }
-  } else if (warp < NUM_CONV_WARPS) {
-    // ---- converters ----
-    // Thread ct owns chunk (row, c) = (ct/8 + 64 i, ct % 8) of every stage.  Row & 7
-    // does not depend on i, so each chunk's swizzled store offset and packed load
-    // offset are a per-thread base plus a compile-time stride.
-    Lut16 ta, tw;
-    uint32_t qa0 = args.lut_a[0], qa1 = args.lut_a[1], qw0 = args.lut_w[0], qw1 = args.lut_w[1];
-    if constexpr (BA == 4) ta = make_lut16(args.lut_a);
-    if constexpr (BW == 4) tw = make_lut16(args.lut_w);
-    const int ct = threadIdx.x;  // 0..NUM_CONV-1
-    const int r0 = ct >> 3, c = ct & 7;
-    const uint32_t st_off = sw128_offset(r0, c);
-    constexpr int RB_A = PackedTile<BA>::kRowBytes, RB_B = PackedTile<BW>::kRowBytes;
-    const int ld_a = r0 * RB_A + c * BA, ld_b = r0 * RB_B + c * BW;  // 8 codes = BITS bytes
-    constexpr int ROWS_PER_PASS = NUM_CONV / 8;                     // 64
-    constexpr int ST_STRIDE = ROWS_PER_PASS / 8 * 1024;             // 8192 bytes
+  } else if (warp < NUM_A_WARPS) {
+    // ---- A converters: row r = 32 (warp % 4) + lane (its TMEM lane), K half hf ----
+    // Each thread expands 4 chunks (32 codes) of its row and stores them as 16
+    // TMEM columns (two fp16 per column, lower K in the low half).
+    Lut8 ta;
+    const uint32_t qa0 = args.lut_a[0], qa1 = args.lut_a[1];
+    if constexpr (BA == 4) ta = make_lut8(args.lut_a);
+    const int q = warp & 3, hf = warp >> 2;
+    const int r = 32 * q + lane;
+    constexpr int RB_A = PackedTile<BA>::kRowBytes;
+    const uint32_t ld_a = (uint32_t)(r * RB_A + hf * 4 * BA);   // 4 chunks = 4 * BA bytes, 8-aligned
+    const uint32_t t_lane = tmem_base + ((uint32_t)(32 * q) << 16) + (uint32_t)(A_COL0 + 16 * hf);
     uint32_t pc = 0;
     bool ok = true;
     for (int t = unit; t < num_tiles && ok; t += nunits) {
       for (int kb = 0; kb < KB; ++kb, ++pc) {
         const int ps = pc % PSTAGES, es = pc % ESTAGES;
         const uint32_t pph = (pc / PSTAGES) & 1u, eph = (pc / ESTAGES) & 1u;
-        if (!wait_bounded(bar(PK_FULL + ps), pph, abort_flag, args.status) ||
-            !wait_bounded(bar(EX_EMPTY + es), eph ^ 1u, abort_flag, args.status)) {
+        const bool got = wait_bounded(bar(PK_FULL + ps), pph, abort_flag, args.status) &&
+                         wait_bounded(bar(EX_EMPTY + es), eph ^ 1u, abort_flag, args.status);
+        __syncwarp();
+        if (__any_sync(0xFFFFFFFFu, !got)) {
           ok = false;
           break;
         }
+        tc_fence_after();  // the MMAs that read this TMEM stage are complete
         const uint32_t pa = sbase + S::kPackA + ps * S::kPkAStride + ld_a;
-        const uint32_t pb = sbase + S::kPackB + ps * S::kPkBStride + ld_b;
-        const uint32_t ea = sbase + S::kExpA + es * EXP_A_BYTES + st_off;
-        const uint32_t eb = sbase + S::kExpB + es * S::kExpBBytes + st_off;
-        uint64_t ra[BM / ROWS_PER_PASS], rb[BN_CTA / ROWS_PER_PASS];
+        uint64_t ra[4];
+        if constexpr (BA == 4) {
+          uint32_t w0, w1, w2, w3;
+          asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(w0), "=r"(w1), "=r"(w2), "=r"(w3) : "r"(pa));
+          ra[0] = w0; ra[1] = w1; ra[2] = w2; ra[3] = w3;
+        } else {
 #pragma unroll
-        for (int i = 0; i < BM / ROWS_PER_PASS; ++i) ra[i] = load_chunk<BA>(pa + i * ROWS_PER_PASS * RB_A);
+          for (int i = 0; i < 4; ++i) ra[i] = load_chunk<BA>(pa + i * BA);
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(PK_EMPTY + ps));  // packed stage read by this warp
+        uint32_t v[16];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const uint4 e = expand8<BA>(ra[i], ta, qa0, qa1, sbase + S::kLut);
+          v[4 * i] = e.x; v[4 * i + 1] = e.y; v[4 * i + 2] = e.z; v[4 * i + 3] = e.w;
+        }
+        tmem_st16(t_lane + (uint32_t)(32 * es), v);
+        asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) {
+          if constexpr (PAIR) mbar_arrive_cluster(bar(EX_FULL + es), 0);  // the leader's barrier
+          else mbar_arrive(bar(EX_FULL + es));
+        }
+      }
+    }
+  } else if (warp < NUM_CONV_WARPS) {
+    // ---- B converters: chunk (row, c) = (ct/8 + 32 i, ct % 8) of every stage ----
+    Lut8 tw;
+    const uint32_t qw0 = args.lut_w[0], qw1 = args.lut_w[1];
+    if constexpr (BW == 4) tw = make_lut8(args.lut_w);
+    const int ct = threadIdx.x - NUM_A_WARPS * 32;  // 0..255
+    const int r0 = ct >> 3, c = ct & 7;
+    const uint32_t st_off = sw128_offset(r0, c);
+    constexpr int RB_B = PackedTile<BW>::kRowBytes;
+    const int ld_b = r0 * RB_B + c * BW;            // 8 codes = BW bytes
+    constexpr int ROWS_PER_PASS = NUM_B_WARPS * 32 / 8;  // 32
+    constexpr int ST_STRIDE = ROWS_PER_PASS / 8 * 1024;  // 4096 bytes
+    uint32_t pc = 0;
+    bool ok = true;
+    for (int t = unit; t < num_tiles && ok; t += nunits) {
+      for (int kb = 0; kb < KB; ++kb, ++pc) {
+        const int ps = pc % PSTAGES, es = pc % ESTAGES;
+        const uint32_t pph = (pc / PSTAGES) & 1u, eph = (pc / ESTAGES) & 1u;
+        const bool got = wait_bounded(bar(PK_FULL + ps), pph, abort_flag, args.status) &&
+                         wait_bounded(bar(EX_EMPTY + es), eph ^ 1u, abort_flag, args.status);
+        __syncwarp();
+        if (__any_sync(0xFFFFFFFFu, !got)) {
+          ok = false;
+          break;
+        }
+        const uint32_t pb = sbase + S::kPackB + ps * S::kPkBStride + ld_b;
+        const uint32_t eb = sbase + S::kExpB + es * S::kExpBBytes + st_off;
+        uint64_t rb[BN_CTA / ROWS_PER_PASS];
 #pragma unroll
         for (int i = 0; i < BN_CTA / ROWS_PER_PASS; ++i) rb[i] = load_chunk<BW>(pb + i * ROWS_PER_PASS * RB_B);
         __syncwarp();
-        if (lane == 0) mbar_arrive(bar(PK_EMPTY + ps));  // packed stage fully read by this warp
-#pragma unroll
-        for (int i = 0; i < BM / ROWS_PER_PASS; ++i) sts_v4(ea + i * ST_STRIDE, expand8<BA>(ra[i], ta, qa0, qa1, sbase + S::kLut));
+        if (lane == 0) mbar_arrive(bar(PK_EMPTY + ps));  // packed stage read by this warp
 #pragma unroll
         for (int i = 0; i < BN_CTA / ROWS_PER_PASS; ++i)
           sts_v4(eb + i * ST_STRIDE, expand8<BW>(rb[i], tw, qw0, qw1, sbase + S::kLut + 128));
@@ -520,13 +630,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       uint32_t ec = 0, lt = 0;
       bool ok = true;
       for (int t = unit; t < num_tiles && ok; t += nunits, ++lt) {
-        const int acc = lt & 1;
-        const uint32_t aph = (lt >> 1) & 1u;
-        const bool got = PAIR ? wait_bounded_cluster(bar(ACC_EMPTY + acc), aph ^ 1u, abort_flag, args.status)
-                              : wait_bounded(bar(ACC_EMPTY + acc), aph ^ 1u, abort_flag, args.status);
+        const uint32_t aph = lt & 1u;
+        const bool got = PAIR ? wait_bounded_cluster(bar(ACC_EMPTY), aph ^ 1u, abort_flag, args.status)
+                              : wait_bounded(bar(ACC_EMPTY), aph ^ 1u, abort_flag, args.status);
         if (!got) break;
         tc_fence_after();
-        const uint32_t tmem_d = tmem_base + (uint32_t)(acc * BN);
         for (int kb = 0; kb < KB; ++kb, ++ec) {
           const int es = ec % ESTAGES;
           const uint32_t eph = (ec / ESTAGES) & 1u;
@@ -537,17 +645,17 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             break;
           }
           tc_fence_after();
-          const uint32_t a_addr = sbase + S::kExpA + es * EXP_A_BYTES;
+          const uint32_t a_tmem = tmem_base + (uint32_t)(A_COL0 + 32 * es);
           const uint32_t b_addr = sbase + S::kExpB + es * S::kExpBBytes;
 #pragma unroll
           for (int k = 0; k < BK / 16; ++k) {
-            umma_f16<PAIR>(tmem_d, umma_desc_sw128(a_addr + 32 * k), umma_desc_sw128(b_addr + 32 * k),
-                           (kb > 0 || k > 0) ? 1u : 0u);
+            umma_f16_ts<PAIR>(tmem_base, a_tmem + 8u * k, umma_desc_sw128(b_addr + 32 * k),
+                              (kb > 0 || k > 0) ? 1u : 0u);
           }
           umma_commit<PAIR>(bar(EX_EMPTY + es));
         }
         if (!ok) break;
-        umma_commit<PAIR>(bar(ACC_FULL + acc));
+        umma_commit<PAIR>(bar(ACC_FULL));
       }
     }
   } else if (warp >= EPI_WARP0 && warp < EPI_WARP0 + 4) {
@@ -555,9 +663,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     const int quad = warp & 3;  // TMEM lanes 32*quad .. 32*quad+31
     uint32_t lt = 0;
     for (int t = unit; t < num_tiles; t += nunits, ++lt) {
-      const int acc = lt & 1;
-      const uint32_t aph = (lt >> 1) & 1u;
-      const bool got = wait_bounded(bar(ACC_FULL + acc), aph, abort_flag, args.status);
+      const uint32_t aph = lt & 1u;
+      const bool got = wait_bounded(bar(ACC_FULL), aph, abort_flag, args.status);
       __syncwarp();
       if (__any_sync(0xFFFFFFFFu, !got)) break;
       tc_fence_after();
@@ -576,26 +683,32 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         col_b[lane + 32 * j] = (in && args.bias) ? bf16_to_f32(args.bias[n]) : 0.0f;
       }
       __syncwarp();
-      const uint32_t taddr = tmem_base + ((uint32_t)(quad * 32) << 16) + (uint32_t)(acc * BN);
+      const uint32_t taddr = tmem_base + ((uint32_t)(quad * 32) << 16);
 #pragma unroll 1
-      for (int c0 = 0; c0 < BN; c0 += 16) {
-        uint32_t v[16];
+      for (int c0 = 0; c0 < BN; c0 += 32) {
+        uint32_t v[32];
         __syncwarp();
-        asm volatile(
-            "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, "
-            "%14, %15}, [%16];"
-            : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7]),
-              "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]), "=r"(v[15])
-            : "r"(taddr + (uint32_t)c0));
+        tmem_ld16(taddr + (uint32_t)c0, v);
+        tmem_ld16(taddr + (uint32_t)c0 + 16u, v + 16);
         asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-        const int nb = n0 + c0;
-        if (row_ok && nb < args.N) {  // N % 16 == 0: a 16-column group is all in or all out
-          float y[16];
 #pragma unroll
-          for (int j = 0; j < 16; ++j) {
-            float val = fmaf(__uint_as_float(v[j]) * a_scale, col_r[c0 + j], col_b[c0 + j]);
-            if (args.epilogue == OQ_EPI_GELU) val = 0.5f * val * (1.0f + erff(val * 0.70710678118654752f));
-            y[j] = val;
+        for (int h = 0; h < 32; h += 16) {
+          const int nb = n0 + c0 + h;
+          if (!row_ok || nb >= args.N) continue;  // N % 16 == 0: a 16-column group is all in or all out
+          float y[16];
+          const float4* cr = reinterpret_cast<const float4*>(col_r + c0 + h);
+          const float4* cb = reinterpret_cast<const float4*>(col_b + c0 + h);
+#pragma unroll
+          for (int j = 0; j < 16; j += 4) {
+            const float4 r4 = cr[j / 4], b4 = cb[j / 4];
+            y[j] = fmaf(__uint_as_float(v[h + j]) * a_scale, r4.x, b4.x);
+            y[j + 1] = fmaf(__uint_as_float(v[h + j + 1]) * a_scale, r4.y, b4.y);
+            y[j + 2] = fmaf(__uint_as_float(v[h + j + 2]) * a_scale, r4.z, b4.z);
+            y[j + 3] = fmaf(__uint_as_float(v[h + j + 3]) * a_scale, r4.w, b4.w);
+          }
+          if (args.epilogue == OQ_EPI_GELU) {
+#pragma unroll
+            for (int j = 0; j < 16; ++j) y[j] = 0.5f * y[j] * (1.0f + erff(y[j] * 0.70710678118654752f));
           }
           if (args.y32) {
             float4* dst = reinterpret_cast<float4*>(args.y32 + (size_t)row * args.N + nb);
@@ -619,8 +732,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       tc_fence_before();
       __syncwarp();  // also: every lane is done reading this tile's column factors
       if (lane == 0) {
-        if constexpr (PAIR) mbar_arrive_cluster(bar(ACC_EMPTY + acc), 0);  // the leader's barrier
-        else mbar_arrive(bar(ACC_EMPTY + acc));
+        if constexpr (PAIR) mbar_arrive_cluster(bar(ACC_EMPTY), 0);  // the leader's barrier
+        else mbar_arrive(bar(ACC_EMPTY));
       }
     }
   }
@@ -706,7 +819,7 @@ int launch_t(GemmArgs& a, const uint8_t* a_codes, const uint8_t* w_codes, int ns
     e = cudaOccupancyMaxActiveClusters(&max_clusters, k, &cfg);
     if (e != cudaSuccess) return fail(OQ_ERR_CUDA, "cluster occupancy query: %s", cudaGetErrorString(e));
     if (max_clusters < 1) return fail(OQ_ERR_UNSUPPORTED, "no CTA pair of the GEMM fits on this device");
-    units = std::min(a.num_tiles, max_clusters);
+    units = std::min(std::min(a.num_tiles, max_clusters), nsm / 2);  // one CTA per SM
     cfg.gridDim = dim3(2 * units, 1, 1);
   } else {
     cfg.gridDim = dim3(units, 1, 1);
@@ -752,6 +865,14 @@ int launch_cbgemm(int d, oq_codebook_t cb_a, oq_codebook_t cb_w, const uint8_t* 
     };
     a.lut_a[i] = entry(cb_a, 2 * i) | (entry(cb_a, 2 * i + 1) << 16);
     a.lut_w[i] = entry(cb_w, 2 * i) | (entry(cb_w, 2 * i + 1) << 16);
+  }
+  // The 4-bit expansion reads only the negative half of each table and flips
+  // the sign bit for the rest.
+  for (oq_codebook_t cb : {cb_a, cb_w}) {
+    const int L = 1 << cb->bits;
+    for (int k = 0; k < L; ++k)
+      if ((uint16_t)cb->lut[L - 1 - k] != (uint16_t)(cb->lut[k] ^ 0x8000u))
+        return fail(OQ_ERR_UNSUPPORTED, "codebook table is not odd (entry %d)", k);
   }
   cudaStream_t s = (cudaStream_t)stream;
   const int ba = cb_a->bits, bw = cb_w->bits;
