@@ -45,7 +45,7 @@ namespace {
 
 constexpr int BM = 128, BN = 256, BK = 64;  // per-CTA A rows, tile N, K step
 constexpr int PSTAGES = 4;                   // packed-code ring
-constexpr int ESTAGES = 4;                   // expanded ring (A in TMEM, B in shared memory)
+constexpr int MAX_ESTAGES = 4;               // expanded ring (A in TMEM, B in shared memory)
 constexpr int NUM_A_WARPS = 8;               // warps 0..7
 constexpr int NUM_B_WARPS = 8;               // warps 8..15
 constexpr int NUM_CONV_WARPS = NUM_A_WARPS + NUM_B_WARPS;
@@ -88,14 +88,20 @@ struct Smem {
   static constexpr int kPkB = kBnCta * PackedTile<BW>::kRowBytes;
   static constexpr int kPkAStride = (kPkA + 127) / 128 * 128;
   static constexpr int kPkBStride = (kPkB + 127) / 128 * 128;
+  // Expanded-B stages: a CTA of a pair holds 16 KB per stage, a lone CTA 32 KB.
+  static constexpr int kES = PAIR ? MAX_ESTAGES : 3;
+  // Output staging for the bulk tensor stores: 128 rows x 128-byte swizzled
+  // blocks of 16 KB (64 bf16 or 32 fp32 columns each).
+  static constexpr int kStageBlocks = PAIR ? 4 : 2;
   static constexpr int kExpB = 0;
-  static constexpr int kPackA = kExpB + ESTAGES * kExpBBytes;
+  static constexpr int kStage = kExpB + kES * kExpBBytes;
+  static constexpr int kPackA = kStage + kStageBlocks * 16384;
   static constexpr int kPackB = kPackA + PSTAGES * kPkAStride;
   static constexpr int kLut = kPackB + PSTAGES * kPkBStride;
   static constexpr int kEpi = kLut + 256;                 // 4 warps x (r'[256], bias[256]) floats
   static constexpr int kBars = kEpi + 4 * 2 * BN * 4;
   // barriers: pk_full[P], pk_empty[P], ex_full[E], ex_empty[E], acc_full, acc_empty
-  static constexpr int kNumBars = 2 * PSTAGES + 2 * ESTAGES + 2;
+  static constexpr int kNumBars = 2 * PSTAGES + 2 * kES + 2;
   static constexpr int kMisc = kBars + kNumBars * 8;  // tmem base, abort flag
   static constexpr int kTotal = kMisc + 16;
   // Room to align the base, and never less than half an SM's shared memory:
@@ -420,6 +426,34 @@ __device__ __forceinline__ uint32_t bf16x2_rn(float lo, float hi) {
   return r;
 }
 
+// Named barrier 1 over the four epilogue warps.
+__device__ __forceinline__ void epi_bar() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+
+// True in every epilogue thread if `p` holds in any of them (named barrier 1).
+__device__ __forceinline__ bool epi_any(bool p) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred a, b;\n\t"
+      "setp.ne.u32 a, %1, 0;\n\t"
+      "bar.red.or.pred b, 1, 128, a;\n\t"
+      "selp.u32 %0, 1, 0, b;\n\t}"
+      : "=r"(r)
+      : "r"((uint32_t)p)
+      : "memory");
+  return r != 0;
+}
+
+// Bulk tensor store of one box from shared memory (clipped to the tensor).
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, uint32_t src, int x, int y) {
+  asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
+                   reinterpret_cast<uint64_t>(map)),
+               "r"(src), "r"(x), "r"(y)
+               : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_read() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+
 // Stores 16 consecutive 32-bit TMEM columns of this thread's lane.
 __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&v)[16]) {
   asm volatile(
@@ -444,7 +478,8 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t* v) {
 template <int BA, int BW, bool PAIR>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     cbgemm_kernel(const __grid_constant__ GemmArgs args, const __grid_constant__ CUtensorMap map_a,
-                  const __grid_constant__ CUtensorMap map_b) {
+                  const __grid_constant__ CUtensorMap map_b, const __grid_constant__ CUtensorMap map_y16,
+                  const __grid_constant__ CUtensorMap map_y32) {
   using S = Smem<BA, BW, PAIR>;
   constexpr int BN_CTA = S::kBnCta;
   constexpr int TILE_M = PAIR ? 2 * BM : BM;
@@ -463,6 +498,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   const int unit = PAIR ? (int)(blockIdx.x >> 1) : (int)blockIdx.x;
   const int nunits = PAIR ? (int)(gridDim.x >> 1) : (int)gridDim.x;
   auto bar = [&](int i) { return smem_u32(&bars[i]); };
+  constexpr int ESTAGES = S::kES;
   const int PK_FULL = 0, PK_EMPTY = PSTAGES, EX_FULL = 2 * PSTAGES, EX_EMPTY = 2 * PSTAGES + ESTAGES,
             ACC_FULL = 2 * PSTAGES + 2 * ESTAGES, ACC_EMPTY = ACC_FULL + 1;
 
@@ -660,21 +696,24 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     }
   } else if (warp >= EPI_WARP0 && warp < EPI_WARP0 + 4) {
     // ---- epilogue: this CTA's 128 accumulator rows ----
+    // TMEM -> registers -> scale, bias, GELU -> swizzled staging -> bulk tensor
+    // stores. The accumulator is released right after its last TMEM read, so the
+    // next tile's MMAs overlap the conversion and the stores. The four warps
+    // take every decision together (named barrier 1), so none can wait on a
+    // barrier that another has left.
     const int quad = warp & 3;  // TMEM lanes 32*quad .. 32*quad+31
+    const int rl = quad * 32 + lane;  // row within the CTA's 128
+    const bool leader = (warp == EPI_WARP0 && lane == 0);
+    const uint32_t stage = sbase + S::kStage;
+    float* col_r = reinterpret_cast<float*>(smem + S::kEpi) + quad * 2 * BN;
+    float* col_b = col_r + BN;
+    const uint32_t taddr = tmem_base + ((uint32_t)(quad * 32) << 16);
     uint32_t lt = 0;
     for (int t = unit; t < num_tiles; t += nunits, ++lt) {
-      const uint32_t aph = lt & 1u;
-      const bool got = wait_bounded(bar(ACC_FULL), aph, abort_flag, args.status);
-      __syncwarp();
-      if (__any_sync(0xFFFFFFFFu, !got)) break;
-      tc_fence_after();
       const int m0 = (t % args.tiles_m) * TILE_M + (int)rank * BM, n0 = (t / args.tiles_m) * BN;
-      const int row = m0 + quad * 32 + lane;
-      const bool row_ok = row < args.M;
-      const float a_scale = row_ok ? args.a_norm[row] * args.inv_d : 0.0f;
-      // this tile's column factors r'_n and bias_n, loaded once per warp
-      float* col_r = reinterpret_cast<float*>(smem + S::kEpi) + quad * 2 * BN;
-      float* col_b = col_r + BN;
+      const int row = m0 + rl;
+      // this tile's factors, fetched while the MMAs run: a_row / d, r'_n and bias_n
+      const float a_scale = row < args.M ? args.a_norm[row] * args.inv_d : 0.0f;
 #pragma unroll
       for (int j = 0; j < BN / 32; ++j) {
         const int n = n0 + lane + 32 * j;
@@ -683,59 +722,80 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         col_b[lane + 32 * j] = (in && args.bias) ? bf16_to_f32(args.bias[n]) : 0.0f;
       }
       __syncwarp();
-      const uint32_t taddr = tmem_base + ((uint32_t)(quad * 32) << 16);
+      const bool got = wait_bounded(bar(ACC_FULL), lt & 1u, abort_flag, args.status);
+      if (epi_any(!got)) break;
+      tc_fence_after();
 #pragma unroll 1
-      for (int c0 = 0; c0 < BN; c0 += 32) {
-        uint32_t v[32];
-        __syncwarp();
-        tmem_ld16(taddr + (uint32_t)c0, v);
-        tmem_ld16(taddr + (uint32_t)c0 + 16u, v + 16);
-        asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-#pragma unroll
-        for (int h = 0; h < 32; h += 16) {
-          const int nb = n0 + c0 + h;
-          if (!row_ok || nb >= args.N) continue;  // N % 16 == 0: a 16-column group is all in or all out
-          float y[16];
-          const float4* cr = reinterpret_cast<const float4*>(col_r + c0 + h);
-          const float4* cb = reinterpret_cast<const float4*>(col_b + c0 + h);
-#pragma unroll
-          for (int j = 0; j < 16; j += 4) {
-            const float4 r4 = cr[j / 4], b4 = cb[j / 4];
-            y[j] = fmaf(__uint_as_float(v[h + j]) * a_scale, r4.x, b4.x);
-            y[j + 1] = fmaf(__uint_as_float(v[h + j + 1]) * a_scale, r4.y, b4.y);
-            y[j + 2] = fmaf(__uint_as_float(v[h + j + 2]) * a_scale, r4.z, b4.z);
-            y[j + 3] = fmaf(__uint_as_float(v[h + j + 3]) * a_scale, r4.w, b4.w);
-          }
-          if (args.epilogue == OQ_EPI_GELU) {
-#pragma unroll
-            for (int j = 0; j < 16; ++j) y[j] = 0.5f * y[j] * (1.0f + erff(y[j] * 0.70710678118654752f));
-          }
-          if (args.y32) {
-            float4* dst = reinterpret_cast<float4*>(args.y32 + (size_t)row * args.N + nb);
-#pragma unroll
-            for (int j = 0; j < 16; j += 4) dst[j / 4] = make_float4(y[j], y[j + 1], y[j + 2], y[j + 3]);
-          }
-          if (args.y16) {
-            uint4* dst = reinterpret_cast<uint4*>(args.y16 + (size_t)row * args.N + nb);
-#pragma unroll
-            for (int j = 0; j < 16; j += 8) {
-              uint4 p;
-              p.x = bf16x2_rn(y[j], y[j + 1]);
-              p.y = bf16x2_rn(y[j + 2], y[j + 3]);
-              p.z = bf16x2_rn(y[j + 4], y[j + 5]);
-              p.w = bf16x2_rn(y[j + 6], y[j + 7]);
-              dst[j / 8] = p;
+      for (int kind = 0; kind < 2; ++kind) {  // 0: bf16 output, 1: fp32 output
+        const bool want = kind == 0 ? args.y16 != nullptr : args.y32 != nullptr;
+        if (!want) continue;
+        const bool last_kind = kind == 1 || args.y32 == nullptr;
+        const int cpb = kind == 0 ? 64 : 32;  // columns per 128-byte block
+        const int pass_cols = S::kStageBlocks * cpb;
+#pragma unroll 1
+        for (int p0 = 0; p0 < BN; p0 += pass_cols) {
+          if (leader) bulk_wait_read();  // the previous stores have read the staging buffer
+          epi_bar();
+#pragma unroll 1
+          for (int c0 = p0; c0 < p0 + pass_cols; c0 += 16) {
+            uint32_t v[16];
+            __syncwarp();
+            tmem_ld16(taddr + (uint32_t)c0, v);
+            asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+            if (last_kind && c0 + 16 == BN) {  // last read of this accumulator
+              tc_fence_before();
+              __syncwarp();
+              if (lane == 0) {
+                if constexpr (PAIR) mbar_arrive_cluster(bar(ACC_EMPTY), 0);  // the leader's barrier
+                else mbar_arrive(bar(ACC_EMPTY));
+              }
             }
+            const int lc = c0 - p0;  // column within the pass
+            const uint32_t blk = stage + (uint32_t)(lc / cpb) * 16384u + (uint32_t)rl * 128u;
+            const int j0 = (lc % cpb) * (kind == 0 ? 2 : 4) / 16;  // first 16-byte chunk of the row
+#pragma unroll
+            for (int q = 0; q < 2; ++q) {  // 8 columns at a time
+              float y[8];
+              const float4 r0 = *reinterpret_cast<const float4*>(col_r + c0 + 8 * q);
+              const float4 r1 = *reinterpret_cast<const float4*>(col_r + c0 + 8 * q + 4);
+              const float4 b0 = *reinterpret_cast<const float4*>(col_b + c0 + 8 * q);
+              const float4 b1 = *reinterpret_cast<const float4*>(col_b + c0 + 8 * q + 4);
+              const float rr[8] = {r0.x, r0.y, r0.z, r0.w, r1.x, r1.y, r1.z, r1.w};
+              const float bb[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+#pragma unroll
+              for (int j = 0; j < 8; ++j) {
+                float val = fmaf(__uint_as_float(v[8 * q + j]) * a_scale, rr[j], bb[j]);
+                if (args.epilogue == OQ_EPI_GELU) val = 0.5f * val * (1.0f + erff(val * 0.70710678118654752f));
+                y[j] = val;
+              }
+              if (kind == 0) {
+                sts_v4(blk + (uint32_t)(((j0 + q) ^ (rl & 7)) << 4),
+                       make_uint4(bf16x2_rn(y[0], y[1]), bf16x2_rn(y[2], y[3]), bf16x2_rn(y[4], y[5]),
+                                  bf16x2_rn(y[6], y[7])));
+              } else {
+                sts_v4(blk + (uint32_t)(((j0 + 2 * q) ^ (rl & 7)) << 4),
+                       make_uint4(__float_as_uint(y[0]), __float_as_uint(y[1]), __float_as_uint(y[2]),
+                                  __float_as_uint(y[3])));
+                sts_v4(blk + (uint32_t)(((j0 + 2 * q + 1) ^ (rl & 7)) << 4),
+                       make_uint4(__float_as_uint(y[4]), __float_as_uint(y[5]), __float_as_uint(y[6]),
+                                  __float_as_uint(y[7])));
+              }
+            }
+          }
+          asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // staging visible to the bulk copies
+          epi_bar();
+          if (leader) {
+            const CUtensorMap* map = kind == 0 ? &map_y16 : &map_y32;
+            for (int b = 0; b < S::kStageBlocks; ++b) {
+              const int x = n0 + p0 + b * cpb;
+              if (x < args.N && m0 < args.M) tma_store_2d(map, stage + (uint32_t)b * 16384u, x, m0);
+            }
+            bulk_commit();
           }
         }
       }
-      tc_fence_before();
-      __syncwarp();  // also: every lane is done reading this tile's column factors
-      if (lane == 0) {
-        if constexpr (PAIR) mbar_arrive_cluster(bar(ACC_EMPTY), 0);  // the leader's barrier
-        else mbar_arrive(bar(ACC_EMPTY));
-      }
     }
+    if (leader) bulk_wait_all();
   }
 
   // teardown: every role of both CTAs is done (or gave up); release TMEM
@@ -785,7 +845,22 @@ int make_code_map(CUtensorMap* map, const void* base, int rows, int row_bytes, i
   return OQ_OK;
 }
 
-using GemmKernel = void (*)(GemmArgs, CUtensorMap, CUtensorMap);
+// Row-major M x N output, written in 128-row boxes of 128 bytes with the
+// 128-byte swizzle that the epilogue's staging layout uses.
+int make_out_map(CUtensorMap* map, void* base, int M, int N, CUtensorMapDataType type, int esize) {
+  EncodeTiledFn enc;
+  if (int rc = get_encode_fn(&enc)) return rc;
+  cuuint64_t dims[2] = {(cuuint64_t)N, (cuuint64_t)M};
+  cuuint64_t strides[1] = {(cuuint64_t)N * (cuuint64_t)esize};
+  cuuint32_t box[2] = {(cuuint32_t)(128 / esize), 128u};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = enc(map, type, 2, base, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                   CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(OQ_ERR_CUDA, "cuTensorMapEncodeTiled (output) failed (%d)", (int)r);
+  return OQ_OK;
+}
+
+using GemmKernel = void (*)(GemmArgs, CUtensorMap, CUtensorMap, CUtensorMap, CUtensorMap);
 
 template <int BA, int BW, bool PAIR>
 int launch_t(GemmArgs& a, const uint8_t* a_codes, const uint8_t* w_codes, int nsm, cudaStream_t stream) {
@@ -793,6 +868,13 @@ int launch_t(GemmArgs& a, const uint8_t* a_codes, const uint8_t* w_codes, int ns
   CUtensorMap ma, mb;
   if (int rc = make_code_map(&ma, a_codes, a.M, a.K * BA / 8, BK * BA / 8, BM)) return rc;
   if (int rc = make_code_map(&mb, w_codes, a.N, a.K * BW / 8, BK * BW / 8, S::kBnCta)) return rc;
+  CUtensorMap my16, my32;
+  memset(&my16, 0, sizeof(my16));
+  memset(&my32, 0, sizeof(my32));
+  if (a.y16)
+    if (int rc = make_out_map(&my16, a.y16, a.M, a.N, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2)) return rc;
+  if (a.y32)
+    if (int rc = make_out_map(&my32, a.y32, a.M, a.N, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4)) return rc;
   GemmKernel k = cbgemm_kernel<BA, BW, PAIR>;
   const int smem = S::kAlloc;
   cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
@@ -824,7 +906,7 @@ int launch_t(GemmArgs& a, const uint8_t* a_codes, const uint8_t* w_codes, int ns
   } else {
     cfg.gridDim = dim3(units, 1, 1);
   }
-  e = cudaLaunchKernelEx(&cfg, k, a, ma, mb);
+  e = cudaLaunchKernelEx(&cfg, k, a, ma, mb, my16, my32);
   if (e != cudaSuccess) return fail(OQ_ERR_CUDA, "GEMM launch: %s", cudaGetErrorString(e));
   return OQ_OK;
 }
