@@ -38,17 +38,18 @@
 #include <cmath>
 #include <cstring>
 
+#include <type_traits>
+
 #include "oq_internal.h"
 
 namespace oq {
 namespace {
 
 constexpr int BM = 128, BN = 256, BK = 64;  // per-CTA A rows, tile N, K step
-constexpr int PSTAGES = 4;                   // packed-code ring
-constexpr int MAX_ESTAGES = 4;               // expanded ring (A in TMEM, B in shared memory)
-constexpr int NUM_A_WARPS = 8;               // warps 0..7
-constexpr int NUM_B_WARPS = 8;               // warps 8..15
-constexpr int NUM_CONV_WARPS = NUM_A_WARPS + NUM_B_WARPS;
+constexpr int NUM_GROUPS = 4;                // converter groups; group g expands k-steps g, g+4, ...
+constexpr int GROUP_WARPS = 4;               // one warp per SM sub-partition and TMEM lane quarter
+constexpr int NUM_CONV_WARPS = NUM_GROUPS * GROUP_WARPS;  // warps 0..15
+constexpr int ESTAGES = NUM_GROUPS;          // expanded ring: stage g belongs to group g
 constexpr int EPI_WARP0 = 16;
 constexpr int TMA_WARP = 20;
 constexpr int MMA_WARP = 21;
@@ -88,20 +89,23 @@ struct Smem {
   static constexpr int kPkB = kBnCta * PackedTile<BW>::kRowBytes;
   static constexpr int kPkAStride = (kPkA + 127) / 128 * 128;
   static constexpr int kPkBStride = (kPkB + 127) / 128 * 128;
-  // Expanded-B stages: a CTA of a pair holds 16 KB per stage, a lone CTA 32 KB.
-  static constexpr int kES = PAIR ? MAX_ESTAGES : 3;
-  // Output staging for the bulk tensor stores: 128 rows x 128-byte swizzled
-  // blocks of 16 KB (64 bf16 or 32 fp32 columns each).
-  static constexpr int kStageBlocks = PAIR ? 4 : 2;
+  // bytes that do not depend on the ring depth or the output staging
+  static constexpr int kFixed = ESTAGES * kExpBBytes + 256 + 4 * 2 * BN * 4 + 512 + 16 + 1024;
+  static constexpr int kBudget = 227 * 1024;
+  // Packed ring: 8 stages (two per group) where they fit, else 4. Output staging:
+  // 128 rows x 128-byte swizzled blocks of 16 KB (64 bf16 or 32 fp32 columns).
+  static constexpr int kPS = kFixed + 8 * (kPkAStride + kPkBStride) + (PAIR ? 4 : 2) * 16384 <= kBudget ? 8 : 4;
+  static constexpr int kRest = kBudget - kFixed - kPS * (kPkAStride + kPkBStride);
+  static constexpr int kStageBlocks = (PAIR && kRest >= 4 * 16384) ? 4 : (kRest >= 2 * 16384 ? 2 : 1);
   static constexpr int kExpB = 0;
-  static constexpr int kStage = kExpB + kES * kExpBBytes;
+  static constexpr int kStage = kExpB + ESTAGES * kExpBBytes;
   static constexpr int kPackA = kStage + kStageBlocks * 16384;
-  static constexpr int kPackB = kPackA + PSTAGES * kPkAStride;
-  static constexpr int kLut = kPackB + PSTAGES * kPkBStride;
+  static constexpr int kPackB = kPackA + kPS * kPkAStride;
+  static constexpr int kLut = kPackB + kPS * kPkBStride;
   static constexpr int kEpi = kLut + 256;                 // 4 warps x (r'[256], bias[256]) floats
   static constexpr int kBars = kEpi + 4 * 2 * BN * 4;
   // barriers: pk_full[P], pk_empty[P], ex_full[E], ex_empty[E], acc_full, acc_empty
-  static constexpr int kNumBars = 2 * PSTAGES + 2 * kES + 2;
+  static constexpr int kNumBars = 2 * kPS + 2 * ESTAGES + 2;
   static constexpr int kMisc = kBars + kNumBars * 8;  // tmem base, abort flag
   static constexpr int kTotal = kMisc + 16;
   // Room to align the base, and never less than half an SM's shared memory:
@@ -109,6 +113,8 @@ struct Smem {
   // wait in tcgen05.alloc for the first one to finish.
   static constexpr int kMinAlloc = 120 * 1024;
   static constexpr int kAlloc = kTotal + 1024 > kMinAlloc ? kTotal + 1024 : kMinAlloc;
+  static_assert(kNumBars * 8 <= 512, "barrier area");
+  static_assert(kAlloc <= kBudget, "shared memory plan exceeds 227 KB");
 };
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
@@ -282,12 +288,6 @@ __device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
   return d;
 }
 
-__device__ __forceinline__ uint32_t lds_u32(uint32_t addr) {
-  uint32_t v;
-  asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(addr));
-  return v;
-}
-
 __device__ __forceinline__ uint32_t lds_u16(uint32_t addr) {
   uint16_t v;
   asm volatile("ld.shared.u16 %0, [%1];" : "=h"(v) : "r"(addr));
@@ -297,6 +297,30 @@ __device__ __forceinline__ uint32_t lds_u16(uint32_t addr) {
 __device__ __forceinline__ void sts_v4(uint32_t addr, uint4 v) {
   asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
                : "memory");
+}
+
+// One packed row of a k-step (BYTES = 16, 32 or 48; 16-byte aligned) into registers.
+template <int BYTES>
+__device__ __forceinline__ void lds_row(uint32_t addr, uint32_t* w) {
+#pragma unroll
+  for (int i = 0; i < BYTES / 16; ++i)
+    asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(w[4 * i]), "=r"(w[4 * i + 1]), "=r"(w[4 * i + 2]), "=r"(w[4 * i + 3])
+                 : "r"(addr + 16 * i));
+}
+
+// Codes 8i .. 8i+7 of a packed row held in registers (little-endian bit stream).
+template <int BITS>
+__device__ __forceinline__ uint64_t row_chunk(const uint32_t* w, int i) {
+  if constexpr (BITS == 4) {
+    return w[i];
+  } else if constexpr (BITS == 2) {
+    return (w[i >> 1] >> (16 * (i & 1))) & 0xFFFFu;
+  } else {  // 6 bits: 48 bits starting at byte 6 i
+    const int byte = 6 * i, wi = byte >> 2, sh = 8 * (byte & 3);
+    const uint64_t lo = w[wi], hi = (wi + 1 < 12) ? w[wi + 1] : 0u;
+    return (((hi << 32) | lo) >> sh) & 0xFFFFFFFFFFFFull;
+  }
 }
 
 // ---- code -> fp16 expansion ---------------------------------------------------
@@ -398,19 +422,6 @@ __device__ __forceinline__ uint4 expand8(uint64_t packed, const Lut8& t8, uint32
 }
 
 // Eight packed codes starting at shared address `addr` (8*BITS bits).
-template <int BITS>
-__device__ __forceinline__ uint64_t load_chunk(uint32_t addr) {
-  if constexpr (BITS == 4) {
-    return lds_u32(addr);
-  } else if constexpr (BITS == 2) {
-    return lds_u16(addr);
-  } else {
-    const uint32_t base = addr & ~3u;
-    const uint64_t lo = lds_u32(base);
-    const uint64_t hi = lds_u32(base + 4);
-    return ((hi << 32) | lo) >> (8 * (addr - base));
-  }
-}
 
 // Offset of (row, 16-byte chunk c) in a K-major 128-byte-swizzled tile of 64 fp16 per row.
 __device__ __forceinline__ uint32_t sw128_offset(int row, int c) {
@@ -455,7 +466,7 @@ __device__ __forceinline__ void bulk_wait_read() { asm volatile("cp.async.bulk.w
 __device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 
 // Stores 16 consecutive 32-bit TMEM columns of this thread's lane.
-__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&v)[16]) {
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t* v) {
   asm volatile(
       "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
       "%15, %16};" ::"r"(taddr),
@@ -498,17 +509,17 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   const int unit = PAIR ? (int)(blockIdx.x >> 1) : (int)blockIdx.x;
   const int nunits = PAIR ? (int)(gridDim.x >> 1) : (int)gridDim.x;
   auto bar = [&](int i) { return smem_u32(&bars[i]); };
-  constexpr int ESTAGES = S::kES;
+  constexpr int PSTAGES = S::kPS;
   const int PK_FULL = 0, PK_EMPTY = PSTAGES, EX_FULL = 2 * PSTAGES, EX_EMPTY = 2 * PSTAGES + ESTAGES,
             ACC_FULL = 2 * PSTAGES + 2 * ESTAGES, ACC_EMPTY = ACC_FULL + 1;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < PSTAGES; ++s) {
       mbar_init(bar(PK_FULL + s), 1);
-      mbar_init(bar(PK_EMPTY + s), NUM_CONV_WARPS);
+      mbar_init(bar(PK_EMPTY + s), GROUP_WARPS);           // the warps of one group
     }
     for (int s = 0; s < ESTAGES; ++s) {
-      mbar_init(bar(EX_FULL + s), NUM_CONV_WARPS * NCTA);  // converters of both CTAs
+      mbar_init(bar(EX_FULL + s), GROUP_WARPS * NCTA);     // one group in each CTA
       mbar_init(bar(EX_EMPTY + s), 1);
     }
     mbar_init(bar(ACC_FULL), 1);
@@ -540,6 +551,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 
   const int KB = args.K / BK;
   const int num_tiles = args.num_tiles;
+  // k-steps this CTA runs over all its tiles (the converters' flat sequence)
+  const uint32_t my_tiles = unit < num_tiles ? (uint32_t)((num_tiles - 1 - unit) / nunits + 1) : 0u;
+  const uint32_t total_steps = my_tiles * (uint32_t)KB;
 
   if (warp == TMA_WARP) {
     if (lane == 0) {
@@ -564,101 +578,62 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         }
       }
     }
-  } else if (warp < NUM_A_WARPS) {
-    // ---- A converters: row r = 32 (warp % 4) + lane (its TMEM lane), K half hf ----
-    // Each thread expands 4 chunks (32 codes) of its row and stores them as 16
-    // TMEM columns (two fp16 per column, lower K in the low half).
-    Lut8 ta;
-    const uint32_t qa0 = args.lut_a[0], qa1 = args.lut_a[1];
-    if constexpr (BA == 4) ta = make_lut8(args.lut_a);
-    const int q = warp & 3, hf = warp >> 2;
-    const int r = 32 * q + lane;
-    constexpr int RB_A = PackedTile<BA>::kRowBytes;
-    const uint32_t ld_a = (uint32_t)(r * RB_A + hf * 4 * BA);   // 4 chunks = 4 * BA bytes, 8-aligned
-    const uint32_t t_lane = tmem_base + ((uint32_t)(32 * q) << 16) + (uint32_t)(A_COL0 + 16 * hf);
-    uint32_t pc = 0;
-    bool ok = true;
-    for (int t = unit; t < num_tiles && ok; t += nunits) {
-      for (int kb = 0; kb < KB; ++kb, ++pc) {
-        const int ps = pc % PSTAGES, es = pc % ESTAGES;
-        const uint32_t pph = (pc / PSTAGES) & 1u, eph = (pc / ESTAGES) & 1u;
-        const bool got = wait_bounded(bar(PK_FULL + ps), pph, abort_flag, args.status) &&
-                         wait_bounded(bar(EX_EMPTY + es), eph ^ 1u, abort_flag, args.status);
-        __syncwarp();
-        if (__any_sync(0xFFFFFFFFu, !got)) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();  // the MMAs that read this TMEM stage are complete
-        const uint32_t pa = sbase + S::kPackA + ps * S::kPkAStride + ld_a;
-        uint64_t ra[4];
-        if constexpr (BA == 4) {
-          uint32_t w0, w1, w2, w3;
-          asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(w0), "=r"(w1), "=r"(w2), "=r"(w3) : "r"(pa));
-          ra[0] = w0; ra[1] = w1; ra[2] = w2; ra[3] = w3;
-        } else {
-#pragma unroll
-          for (int i = 0; i < 4; ++i) ra[i] = load_chunk<BA>(pa + i * BA);
-        }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(bar(PK_EMPTY + ps));  // packed stage read by this warp
-        uint32_t v[16];
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const uint4 e = expand8<BA>(ra[i], ta, qa0, qa1, sbase + S::kLut);
-          v[4 * i] = e.x; v[4 * i + 1] = e.y; v[4 * i + 2] = e.z; v[4 * i + 3] = e.w;
-        }
-        tmem_st16(t_lane + (uint32_t)(32 * es), v);
-        asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) {
-          if constexpr (PAIR) mbar_arrive_cluster(bar(EX_FULL + es), 0);  // the leader's barrier
-          else mbar_arrive(bar(EX_FULL + es));
-        }
-      }
-    }
   } else if (warp < NUM_CONV_WARPS) {
-    // ---- B converters: chunk (row, c) = (ct/8 + 32 i, ct % 8) of every stage ----
-    Lut8 tw;
+    // ---- converters: group g = warp / 4 expands k-steps g, g+4, g+8, ... ----
+    // Thread (quad q = warp % 4, lane) owns row r = 32 q + lane of both operands:
+    // the activation row goes to TMEM lane r (32 columns of fp16 pairs, lower K
+    // in the low half) and the weight row(s) to the swizzled shared stage. The
+    // four groups run out of phase, so one group's waits overlap another's
+    // arithmetic; each group expands before it waits for its ring slot.
+    const int g = warp / GROUP_WARPS, q = warp % GROUP_WARPS;
+    const int r = 32 * q + lane;
+    Lut8 ta, tw;
+    const uint32_t qa0 = args.lut_a[0], qa1 = args.lut_a[1];
     const uint32_t qw0 = args.lut_w[0], qw1 = args.lut_w[1];
+    if constexpr (BA == 4) ta = make_lut8(args.lut_a);
     if constexpr (BW == 4) tw = make_lut8(args.lut_w);
-    const int ct = threadIdx.x - NUM_A_WARPS * 32;  // 0..255
-    const int r0 = ct >> 3, c = ct & 7;
-    const uint32_t st_off = sw128_offset(r0, c);
-    constexpr int RB_B = PackedTile<BW>::kRowBytes;
-    const int ld_b = r0 * RB_B + c * BW;            // 8 codes = BW bytes
-    constexpr int ROWS_PER_PASS = NUM_B_WARPS * 32 / 8;  // 32
-    constexpr int ST_STRIDE = ROWS_PER_PASS / 8 * 1024;  // 4096 bytes
-    uint32_t pc = 0;
-    bool ok = true;
-    for (int t = unit; t < num_tiles && ok; t += nunits) {
-      for (int kb = 0; kb < KB; ++kb, ++pc) {
-        const int ps = pc % PSTAGES, es = pc % ESTAGES;
-        const uint32_t pph = (pc / PSTAGES) & 1u, eph = (pc / ESTAGES) & 1u;
-        const bool got = wait_bounded(bar(PK_FULL + ps), pph, abort_flag, args.status) &&
-                         wait_bounded(bar(EX_EMPTY + es), eph ^ 1u, abort_flag, args.status);
-        __syncwarp();
-        if (__any_sync(0xFFFFFFFFu, !got)) {
-          ok = false;
-          break;
-        }
-        const uint32_t pb = sbase + S::kPackB + ps * S::kPkBStride + ld_b;
-        const uint32_t eb = sbase + S::kExpB + es * S::kExpBBytes + st_off;
-        uint64_t rb[BN_CTA / ROWS_PER_PASS];
+    constexpr int RB_A = PackedTile<BA>::kRowBytes, RB_B = PackedTile<BW>::kRowBytes;
+    constexpr int NB_ROWS = BN_CTA / BM;  // weight rows per thread: 1 (pair) or 2
+    const uint32_t t_lane = tmem_base + ((uint32_t)(32 * q) << 16) + (uint32_t)(A_COL0 + 32 * g);
+    for (uint32_t pc = (uint32_t)g, j = 0; pc < total_steps; pc += NUM_GROUPS, ++j) {
+      const int ps = pc % PSTAGES;
+      const uint32_t pph = (pc / PSTAGES) & 1u;
+      bool got = wait_bounded(bar(PK_FULL + ps), pph, abort_flag, args.status);
+      __syncwarp();
+      if (__any_sync(0xFFFFFFFFu, !got)) break;
+      uint32_t wa[RB_A / 4], wb[NB_ROWS][RB_B / 4];
+      lds_row<RB_A>(sbase + S::kPackA + ps * S::kPkAStride + r * RB_A, wa);
 #pragma unroll
-        for (int i = 0; i < BN_CTA / ROWS_PER_PASS; ++i) rb[i] = load_chunk<BW>(pb + i * ROWS_PER_PASS * RB_B);
-        __syncwarp();
-        if (lane == 0) mbar_arrive(bar(PK_EMPTY + ps));  // packed stage read by this warp
+      for (int h = 0; h < NB_ROWS; ++h)
+        lds_row<RB_B>(sbase + S::kPackB + ps * S::kPkBStride + (r + BM * h) * RB_B, wb[h]);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(PK_EMPTY + ps));  // packed stage read by this warp
+      uint32_t v[32];
 #pragma unroll
-        for (int i = 0; i < BN_CTA / ROWS_PER_PASS; ++i)
-          sts_v4(eb + i * ST_STRIDE, expand8<BW>(rb[i], tw, qw0, qw1, sbase + S::kLut + 128));
-        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-        __syncwarp();
-        if (lane == 0) {
-          if constexpr (PAIR) mbar_arrive_cluster(bar(EX_FULL + es), 0);  // the leader's barrier
-          else mbar_arrive(bar(EX_FULL + es));
-        }
+      for (int i = 0; i < 8; ++i) {
+        const uint4 e = expand8<BA>(row_chunk<BA>(wa, i), ta, qa0, qa1, sbase + S::kLut);
+        v[4 * i] = e.x; v[4 * i + 1] = e.y; v[4 * i + 2] = e.z; v[4 * i + 3] = e.w;
+      }
+      got = wait_bounded(bar(EX_EMPTY + g), (j & 1u) ^ 1u, abort_flag, args.status);
+      __syncwarp();
+      if (__any_sync(0xFFFFFFFFu, !got)) break;
+      tc_fence_after();  // the MMAs that read this stage are complete
+      tmem_st16(t_lane, v);
+      tmem_st16(t_lane + 16u, v + 16);
+      const uint32_t eb = sbase + S::kExpB + g * S::kExpBBytes;
+#pragma unroll
+      for (int h = 0; h < NB_ROWS; ++h) {
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+          sts_v4(eb + sw128_offset(r + BM * h, i), expand8<BW>(row_chunk<BW>(wb[h], i), tw, qw0, qw1, sbase + S::kLut + 128));
+      }
+      asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) {
+        if constexpr (PAIR) mbar_arrive_cluster(bar(EX_FULL + g), 0);  // the leader's barrier
+        else mbar_arrive(bar(EX_FULL + g));
       }
     }
   } else if (warp == MMA_WARP) {
