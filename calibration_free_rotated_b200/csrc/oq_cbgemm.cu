@@ -428,6 +428,27 @@ __device__ __forceinline__ uint32_t sw128_offset(int row, int c) {
   return (uint32_t)((row >> 3) * 1024 + (row & 7) * 128 + ((c ^ (row & 7)) << 4));
 }
 
+// ---- packed f32x2 arithmetic (two columns per instruction) -------------------
+__device__ __forceinline__ unsigned long long f2_pack(float lo, float hi) {
+  unsigned long long r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ void f2_unpack(unsigned long long v, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ unsigned long long f2_mul(unsigned long long a, unsigned long long b) {
+  unsigned long long r;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+__device__ __forceinline__ unsigned long long f2_fma(unsigned long long a, unsigned long long b,
+                                                     unsigned long long c) {
+  unsigned long long r;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+  return r;
+}
+
 __device__ __forceinline__ float bf16_to_f32(uint16_t v) { return __uint_as_float((uint32_t)v << 16); }
 
 // Two floats -> bf16x2 (lo in the low half), round to nearest even.
@@ -728,20 +749,25 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             const int lc = c0 - p0;  // column within the pass
             const uint32_t blk = stage + (uint32_t)(lc / cpb) * 16384u + (uint32_t)rl * 128u;
             const int j0 = (lc % cpb) * (kind == 0 ? 2 : 4) / 16;  // first 16-byte chunk of the row
+            const unsigned long long as2 = f2_pack(a_scale, a_scale);
 #pragma unroll
-            for (int q = 0; q < 2; ++q) {  // 8 columns at a time
+            for (int q = 0; q < 2; ++q) {  // 8 columns at a time, as f32x2 pairs
+              const ulonglong2 r01 = *reinterpret_cast<const ulonglong2*>(col_r + c0 + 8 * q);
+              const ulonglong2 r23 = *reinterpret_cast<const ulonglong2*>(col_r + c0 + 8 * q + 4);
+              const ulonglong2 b01 = *reinterpret_cast<const ulonglong2*>(col_b + c0 + 8 * q);
+              const ulonglong2 b23 = *reinterpret_cast<const ulonglong2*>(col_b + c0 + 8 * q + 4);
+              const unsigned long long rr[4] = {r01.x, r01.y, r23.x, r23.y};
+              const unsigned long long bb[4] = {b01.x, b01.y, b23.x, b23.y};
               float y[8];
-              const float4 r0 = *reinterpret_cast<const float4*>(col_r + c0 + 8 * q);
-              const float4 r1 = *reinterpret_cast<const float4*>(col_r + c0 + 8 * q + 4);
-              const float4 b0 = *reinterpret_cast<const float4*>(col_b + c0 + 8 * q);
-              const float4 b1 = *reinterpret_cast<const float4*>(col_b + c0 + 8 * q + 4);
-              const float rr[8] = {r0.x, r0.y, r0.z, r0.w, r1.x, r1.y, r1.z, r1.w};
-              const float bb[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
 #pragma unroll
-              for (int j = 0; j < 8; ++j) {
-                float val = fmaf(__uint_as_float(v[8 * q + j]) * a_scale, rr[j], bb[j]);
-                if (args.epilogue == OQ_EPI_GELU) val = 0.5f * val * (1.0f + erff(val * 0.70710678118654752f));
-                y[j] = val;
+              for (int j = 0; j < 4; ++j) {
+                const unsigned long long acc2 =
+                    f2_pack(__uint_as_float(v[8 * q + 2 * j]), __uint_as_float(v[8 * q + 2 * j + 1]));
+                f2_unpack(f2_fma(f2_mul(acc2, as2), rr[j], bb[j]), y[2 * j], y[2 * j + 1]);
+              }
+              if (args.epilogue == OQ_EPI_GELU) {
+#pragma unroll
+                for (int j = 0; j < 8; ++j) y[j] = 0.5f * y[j] * (1.0f + erff(y[j] * 0.70710678118654752f));
               }
               if (kind == 0) {
                 sts_v4(blk + (uint32_t)(((j0 + q) ^ (rl & 7)) << 4),
