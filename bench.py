@@ -388,11 +388,26 @@ def run_profile_case(args):
         wn = torch.rand(N, device="cuda").to(torch.bfloat16)
         y = torch.empty(M, N, device="cuda", dtype=torch.bfloat16)
         run = lambda: oq.linear_codes(d, cba, cbw, a, an, w, wn, out_bf16=y, want_f32=False, want_bf16=True)
-    for _ in range(args.warmup + args.steps):
+    for _ in range(args.warmup):
         run()
     torch.cuda.synchronize()
+    times = []
+    for _ in range(args.steps):  # back to back: inputs smaller than L2 stay cached
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        run()
+        e1.record()
+        e1.synchronize()
+        times.append(e0.elapsed_time(e1))
     oq.device_status()
-    print(json.dumps({"profile": args.profile, "rows": M, "d": d, "n": N, "launches": args.warmup + args.steps}))
+    ms = statistics.median(times) if times else float("nan")
+    out = {"profile": args.profile, "rows": M, "d": d, "n": N, "launches": args.warmup + args.steps,
+           "median_ms": ms}
+    if args.profile == "rotq":
+        out["GB/s"] = algorithmic(M, d, N, args.bits_a, args.bits_w)[0] / ms / 1e6
+    else:
+        out["TFLOP/s"] = algorithmic(M, d, N, args.bits_a, args.bits_w)[1] / ms / 1e9
+    print(json.dumps(out))
     return 0
 
 

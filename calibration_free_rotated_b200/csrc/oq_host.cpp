@@ -209,56 +209,63 @@ uint16_t double_to_fp16_rne(double v) {
 // ---------------------------------------------------------------------------
 // Bucket table for the rotate+quantize kernel's centroid search.
 //
-// The kernel forms t (fp32) and y = fma(t, G, C) with C = 1.5*2^23 + off0, so
-// y's low mantissa bits hold q = round(t*G + off0) exactly (one rounding of the
-// exact t*G + C).  Bucket q covers z = t*G + off0 in [q - 1/2, q + 1/2).  G is
-// chosen so that consecutive fp32 boundaries are >= 1.25 buckets apart (at most
-// one boundary per bucket) and no boundary lies within 0.02 bucket of a bucket
-// edge (so a t that rounds to either neighbour at an edge gets the same answer).
-// Entry q: the boundary inside the bucket (or 3e38 if none) with its low b
+// The kernel maps a normalised coordinate t into the unit interval,
+// y = sat(t * alpha + 1/2) (fp32), and reads the bucket q = round(y * NB) from
+// the low mantissa bits of fma(y, NB, 1.5 * 2^23).  Bucket q covers
+// y * NB in [q - 1/2, q + 1/2).  alpha maps every boundary into (0, 1) with a
+// little room; NB (a power of two) is large enough that consecutive fp32
+// boundaries are >= 1.25 buckets apart (at most one boundary per bucket), and
+// alpha is nudged until no boundary lies within 0.02 bucket of a bucket edge
+// (a y that rounds to either neighbour at an edge then gets the same answer).
+// Entry q: the bucket's boundary in y (or 3e38 if none) with its low b
 // mantissa bits replaced by base_q = #{boundaries below the bucket}; the code
-// is (entry & (2^b - 1)) + (t > entry).  Replacing those bits moves a threshold
-// by fewer than 2^b fp32 ulps (< 4e-6 relative), far inside the 1e-5 boundary
-// band of the parity rule.
+// is base_q + (y > entry).  Replacing those bits moves a threshold by fewer
+// than 2^b fp32 ulps of y < 1 (below 4e-6 in y, a few 1e-7 in t), far inside
+// the 1e-5 boundary band of the parity rule.  The middle boundary of an even
+// codebook is t = 0, i.e. y = 1/2 exactly, whose low mantissa bits are zero:
+// its entry is >= 1/2, so t = 0 takes the lower centroid as the tie rule says.
 // ---------------------------------------------------------------------------
 void build_qtable(oq_codebook_t cb) {
   const int L = 1 << cb->bits;
-  std::vector<float> b32(L - 1);
-  for (int k = 0; k < L - 1; ++k) b32[k] = (float)cb->bounds[k];
-  double min_gap = 2.0;
-  for (int k = 0; k + 1 < L - 1; ++k) min_gap = std::fmin(min_gap, (double)b32[k + 1] - (double)b32[k]);
-  float G = (float)(1.25 / min_gap);
-  if (L == 2) G = 4.0f;
-  double off0 = 0.0;
+  std::vector<double> b(L - 1);
+  double bmax = 0.0, gap = 1e300;
+  for (int k = 0; k < L - 1; ++k) {
+    b[k] = (double)(float)cb->bounds[k];
+    bmax = std::fmax(bmax, std::fabs(b[k]));
+    if (k > 0) gap = std::fmin(gap, b[k] - b[k - 1]);
+  }
+  double T = bmax > 0.0 ? bmax * 1.02 + 1e-6 : 1.0;
+  int NB = 2;
+  while (NB < (1 << 16) && 1.25 * (2.0 * T / NB) > gap) NB *= 2;
+  float alpha = 0.0f;
+  std::vector<double> yb(L - 1);
   for (int attempt = 0; attempt < 100000; ++attempt) {
-    off0 = std::ceil((double)G * 1.001) + 2.0;
+    alpha = (float)(0.5 / T);
     bool ok = true;
-    for (int k = 0; k < L - 1 && ok; ++k) {
-      const double z = (double)b32[k] * (double)G + off0;
-      const double f = z - std::floor(z);
-      if (std::fabs(f - 0.5) < 0.02) ok = false;
+    for (int k = 0; k < L - 1; ++k) {
+      yb[k] = (double)(float)(b[k] * (double)alpha + 0.5);
+      const double z = yb[k] * NB;
+      if (std::fabs(z - std::floor(z) - 0.5) < 0.02) ok = false;
     }
     if (ok) break;
-    G = (float)((double)G * 1.0007);
+    T *= 1.0007;
   }
-  const int Q = 2 * (int)off0 + 2;
-  cb->qtable.assign(Q, 0u);
+  cb->qtable.assign(NB + 1, 0u);
   const uint32_t lowmask = (uint32_t)L - 1u;
-  for (int q = 0; q < Q; ++q) {
-    const double lo = q - 0.5, hi = q + 0.5;
+  for (int q = 0; q <= NB; ++q) {
+    const double lo = (q - 0.5) / NB, hi = (q + 0.5) / NB;
     uint32_t base = 0;
     float thr = 3.0e38f;
     for (int k = 0; k < L - 1; ++k) {
-      const double z = (double)b32[k] * (double)G + off0;
-      if (z < lo) ++base;
-      else if (z < hi) thr = b32[k];
+      if (yb[k] < lo) ++base;
+      else if (yb[k] < hi) thr = (float)yb[k];
     }
     uint32_t bits;
     std::memcpy(&bits, &thr, 4);
     cb->qtable[q] = (bits & ~lowmask) | base;
   }
-  cb->qt_scale = G;
-  cb->qt_offset = (float)(12582912.0 + off0);  // 1.5 * 2^23 + off0, exact in fp32
+  cb->qt_alpha = alpha;
+  cb->qt_nb = NB;
 }
 
 // ---------------------------------------------------------------------------

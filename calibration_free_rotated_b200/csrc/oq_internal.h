@@ -28,8 +28,9 @@ struct oq_codebook_s {
   std::vector<uint16_t> lut;      // fp16 bits of RNE(sqrt(d) c_k)
   int iterations = 0;
   double distortion = 0.0;
-  // Bucket table for the branchless centroid search (see oq_host.cpp).
-  float qt_scale = 0.0f, qt_offset = 0.0f;
+  // Bucket table for the branchless centroid search (see build_qtable).
+  float qt_alpha = 0.0f;  // y = t * qt_alpha + 1/2 maps the boundaries into (0, 1)
+  int qt_nb = 0;          // buckets; the table has qt_nb + 1 entries
   std::vector<uint32_t> qtable;
   std::mutex mu;
   uint32_t* dev_qtable[OQ_MAX_DEVICES] = {};

@@ -1,0 +1,512 @@
+// Rotate+quantize kernel template (kernel 1), shared by the translation units
+// that instantiate it (one per configuration, compiled in parallel) and the
+// launcher in oq_rotq.cu.  The design notes are at the top of oq_rotq.cu.
+#pragma once
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cmath>
+#include <cstring>
+
+#include "oq_internal.h"
+
+namespace oq {
+namespace rotq {
+
+constexpr unsigned long long kWaitLimitNs = 1000000000ull;
+
+struct Args {
+  const uint16_t* X;
+  uint8_t* codes;
+  float* norm_f32;
+  uint16_t* norm_bf16;
+  const uint32_t* perm2;  // pi as uint16 pairs: word k = pi(2k) | pi(2k+1) << 16
+  const uint32_t* signs;  // sign words [d/32]
+  const uint32_t* qtable;
+  int* status;
+  int M, d, P, groups, stages, qtable_len, seg_log;
+  uint32_t bar_off, part_off, qt_off, ring_off;  // byte offsets in dynamic shared memory
+  float alpha_h;                                 // alpha / sqrt(h)
+  float nb;                                      // buckets of the search table
+};
+
+// Kernel configurations: pair-buffer stride (IBS) and gather-address form.
+//   0: P*d <= 6144,  IBS = 24 KB, byte addresses
+//   1: d <= 12288,   IBS = 48 KB, byte addresses
+//   2: d <= 16384,   IBS = 64 KB, word addresses (16-bit byte addresses overflow)
+template <int CFG>
+struct Cfg {
+  static constexpr uint32_t IBS = CFG == 0 ? 0x6000u : (CFG == 1 ? 0xC000u : 0x10000u);
+  static constexpr uint32_t HALF = IBS / 2;  // ring: second row of each pair
+  static constexpr bool WORD_ADDR = CFG == 2;
+};
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ unsigned long long global_ns() {
+  unsigned long long t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Bounded wait: gives up after ~1 s, records OQ_ERR_TIMEOUT and returns false.
+static __device__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity, int* status) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const unsigned long long t0 = global_ns();
+  for (uint32_t i = 1;; ++i) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((i & 63u) == 0 && global_ns() - t0 > kWaitLimitNs) {
+      atomicExch(status, OQ_ERR_TIMEOUT);
+      return false;
+    }
+  }
+}
+
+// One stage = R = 2P rows; row 2p lands at slot + p*2d, row 2p+1 at slot + HALF + p*2d.
+// Warp 0 issues it: lane 0 posts the byte count, then the lanes share the copies.
+template <int CFG>
+__device__ __forceinline__ void issue_stage_load(const Args& a, uint32_t ring, uint32_t bars, int it, int lane) {
+  const int grp = blockIdx.x + it * gridDim.x;
+  if (grp >= a.groups) return;
+  const int slot = it % a.stages;
+  const int R = 2 * a.P;
+  const int row0 = grp * R;
+  const int nrows = min(R, a.M - row0);
+  const uint32_t rowb = (uint32_t)a.d * 2u;
+  const uint32_t bar = bars + 8u * slot;
+  const uint32_t dst0 = ring + (uint32_t)slot * Cfg<CFG>::IBS;
+  if (lane == 0)
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"((uint32_t)nrows * rowb)
+                 : "memory");
+  __syncwarp();
+  for (int r = lane; r < nrows; r += 32) {
+    const uint32_t dst = dst0 + (uint32_t)(r & 1) * Cfg<CFG>::HALF + (uint32_t)(r >> 1) * rowb;
+    const uint16_t* src = a.X + (size_t)(row0 + r) * a.d;
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+        "l"(src), "r"(rowb), "r"(bar)
+        : "memory");
+  }
+}
+
+// ---- packed f32x2 arithmetic ---------------------------------------------------
+__device__ __forceinline__ unsigned long long f2_pack(float lo, float hi) {
+  unsigned long long r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ unsigned long long u2_pack(uint32_t lo, uint32_t hi) {
+  unsigned long long r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "r"(lo), "r"(hi));
+  return r;
+}
+__device__ __forceinline__ void f2_unpack(unsigned long long v, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ void u2_unpack(unsigned long long v, uint32_t& lo, uint32_t& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=r"(lo), "=r"(hi) : "l"(v));
+}
+__device__ __forceinline__ unsigned long long f2_add(unsigned long long a, unsigned long long b) {
+  unsigned long long r;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+__device__ __forceinline__ unsigned long long f2_sub(unsigned long long a, unsigned long long b) {
+  unsigned long long r;
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+__device__ __forceinline__ unsigned long long f2_fma(unsigned long long a, unsigned long long b,
+                                                     unsigned long long c) {
+  unsigned long long r;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+  return r;
+}
+__device__ __forceinline__ float fma_sat(float a, float b, float c) {
+  float r;
+  asm("fma.rn.sat.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
+__device__ __forceinline__ uint32_t lds_u32(uint32_t addr) {
+  uint32_t v;
+  asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(addr));
+  return v;
+}
+__device__ __forceinline__ uint4 lds_u128(uint32_t addr) {
+  uint4 v;
+  asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr));
+  return v;
+}
+__device__ __forceinline__ void sts_u128(uint32_t addr, uint32_t x, uint32_t y, uint32_t z, uint32_t w) {
+  asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(x), "r"(y), "r"(z), "r"(w) : "memory");
+}
+
+// Stores 32 codes packed in BITS words (code i at bits [i*BITS, (i+1)*BITS)).
+template <int BITS>
+__device__ __forceinline__ void store_words(uint8_t* dst, const uint32_t (&w)[BITS]) {
+  if constexpr (BITS == 4) {
+    *reinterpret_cast<uint4*>(dst) = make_uint4(w[0], w[1], w[2], w[3]);
+  } else if constexpr (BITS == 2) {
+    *reinterpret_cast<uint2*>(dst) = make_uint2(w[0], w[1]);
+  } else if constexpr (BITS == 6) {
+    uint2* p = reinterpret_cast<uint2*>(dst);
+    p[0] = make_uint2(w[0], w[1]);
+    p[1] = make_uint2(w[2], w[3]);
+    p[2] = make_uint2(w[4], w[5]);
+  } else {
+    uint32_t* p = reinterpret_cast<uint32_t*>(dst);
+#pragma unroll
+    for (int k = 0; k < BITS; ++k) p[k] = w[k];
+  }
+}
+
+// Adds code i (low BITS bits of c, higher bits ignored) to the row's words.
+// Widths dividing 32: funnel the code in from the top of its word, so after
+// the word's last code every code sits at its own position.
+template <int BITS>
+__device__ __forceinline__ void put_code(uint32_t (&w)[BITS], int i, uint32_t c) {
+  if constexpr (32 % BITS == 0) {
+    constexpr int PER = 32 / BITS;
+    w[i / PER] = __funnelshift_r(w[i / PER], c, BITS);
+  } else {
+    c &= (1u << BITS) - 1u;
+    const int bit = i * BITS, wi = bit >> 5, sh = bit & 31;
+    w[wi] |= c << sh;
+    if (sh + BITS > 32) w[wi + 1] |= c >> (32 - sh);
+  }
+}
+
+// Gather step of one stage, for pair buffer BUF (0 or 1; a compile-time
+// offset of BUF * IBS on every shared-memory address).
+template <int CFG, int LOGHB>
+struct Gather {
+  // Gathers the 32 pair words of this thread from pair buffer BUF, applies the
+  // signs, splits them into f32x2 (row 2p, row 2p+1) and accumulates squares.
+  template <int BUF>
+  static __device__ __forceinline__ void run(unsigned long long (&v)[32], unsigned long long& ss2,
+                                             const uint32_t (&offw)[16], const uint32_t (&sb)[8], uint32_t s_base) {
+    unsigned long long sq[4] = {0ull, 0ull, 0ull, 0ull};
+#pragma unroll
+    for (int k = 0; k < 16; ++k) {
+      uint32_t a0, a1;
+      if constexpr (Cfg<CFG>::WORD_ADDR) {
+        a0 = s_base + ((offw[k] & 0xFFFFu) << 2);
+        a1 = s_base + ((offw[k] >> 16) << 2);
+      } else {
+        a0 = offw[k] & 0xFFFFu;
+        a1 = offw[k] >> 16;
+      }
+      const uint32_t w0 = lds_u32(a0 + BUF * Cfg<CFG>::IBS);
+      const uint32_t w1 = lds_u32(a1 + BUF * Cfg<CFG>::IBS);
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const int i = 2 * k + e;
+        const uint32_t w = e ? w1 : w0;
+        // sign byte of coordinate i moved to bit 31 (0 or 0x80000000)
+        const uint32_t sg = __byte_perm(sb[i >> 2], 0u, 0x0444u | ((uint32_t)(i & 3) << 12));
+        const uint32_t ra = (w << 16) + sg;          // row 2p   (add == xor on bit 31)
+        const uint32_t rb = (w & 0xFFFF0000u) ^ sg;  // row 2p+1
+        v[i] = u2_pack(ra, rb);
+        sq[i & 3] = f2_fma(v[i], v[i], sq[i & 3]);
+      }
+    }
+    ss2 = f2_add(f2_add(sq[0], sq[1]), f2_add(sq[2], sq[3]));
+  }
+};
+
+// Per-thread constants of the kernel (all registers).
+struct Thread {
+  int tid, lane, pr, g, spr, nparts;
+  bool active;
+  uint32_t s_base, s_bars, s_ring, qkey;
+  uint32_t src_pair;  // ring: row 2pr, columns 32g.., with the lane's chunk rotation
+  uint32_t ib_w0, ib_w1;
+  float2* partial;
+};
+
+// Interleave stage `it` (ring slot it % stages) into pair buffer it & 1.
+template <int CFG>
+__device__ __forceinline__ bool interleave(const Args& a, const Thread& t, int it) {
+  constexpr uint32_t IBS = Cfg<CFG>::IBS, HALF = Cfg<CFG>::HALF;
+  const int slot = it % a.stages;
+  const uint32_t parity = (uint32_t)(it / a.stages) & 1u;
+  if (!mbar_wait_bounded(t.s_bars + 8u * slot, parity, a.status)) return false;
+  const uint32_t src = t.s_ring + (uint32_t)slot * IBS + t.src_pair;
+  const uint32_t boff = (uint32_t)(it & 1) * IBS;
+#pragma unroll
+  for (int n = 0; n < 4; ++n) {
+    const uint32_t s_a = src ^ (16u * n);
+    const uint4 A = lds_u128(s_a);
+    const uint4 B = lds_u128(s_a + HALF);
+    sts_u128((t.ib_w0 ^ (32u * n)) + boff, __byte_perm(A.x, B.x, 0x5410), __byte_perm(A.x, B.x, 0x7632),
+             __byte_perm(A.y, B.y, 0x5410), __byte_perm(A.y, B.y, 0x7632));
+    sts_u128((t.ib_w1 ^ (32u * n)) + boff, __byte_perm(A.z, B.z, 0x5410), __byte_perm(A.z, B.z, 0x7632),
+             __byte_perm(A.w, B.w, 0x5410), __byte_perm(A.w, B.w, 0x7632));
+  }
+  return true;
+}
+
+// Gather + signs + FWHT of stage `it`, and the segment partials of its squared norms.
+template <int LOGHB, int CFG>
+__device__ __forceinline__ void transform(const Args& a, const Thread& t, int it, unsigned long long (&v)[32],
+                                          const uint32_t (&offw)[16], const uint32_t (&sb)[8]) {
+  unsigned long long ss2;
+  if (it & 1)
+    Gather<CFG, LOGHB>::template run<1>(v, ss2, offw, sb, t.s_base);
+  else
+    Gather<CFG, LOGHB>::template run<0>(v, ss2, offw, sb, t.s_base);
+  {
+    float lo, hi;
+    f2_unpack(ss2, lo, hi);
+    const int seg = 1 << a.seg_log;
+    for (int o = 1; o < seg; o <<= 1) {
+      lo += __shfl_xor_sync(0xFFFFFFFFu, lo, o);
+      hi += __shfl_xor_sync(0xFFFFFFFFu, hi, o);
+    }
+    if ((t.lane & (seg - 1)) == 0) t.partial[(it & 1) * t.nparts + (t.tid >> a.seg_log)] = make_float2(lo, hi);
+  }
+  // in-thread Walsh-Hadamard butterflies over bits 0..4 of the block index
+#pragma unroll
+  for (int s = 1; s < 32; s <<= 1) {
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+      if ((i & s) == 0) {
+        const unsigned long long x0 = v[i], x1 = v[i + s];
+        v[i] = f2_add(x0, x1);
+        v[i + s] = f2_sub(x0, x1);
+      }
+    }
+  }
+  // across the h/32 lanes of a block: bits 5.. of the block index
+#pragma unroll
+  for (int k = 0; k < LOGHB; ++k) {
+    const float sg = ((t.lane >> k) & 1) ? -1.0f : 1.0f;
+    const unsigned long long sg2 = f2_pack(sg, sg);
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+      float lo, hi;
+      f2_unpack(v[i], lo, hi);
+      const float olo = __shfl_xor_sync(0xFFFFFFFFu, lo, 1 << k);
+      const float ohi = __shfl_xor_sync(0xFFFFFFFFu, hi, 1 << k);
+      v[i] = f2_fma(v[i], sg2, f2_pack(olo, ohi));
+    }
+  }
+}
+
+// Normalise, search, pack and store stage `it`.
+template <int BITS>
+__device__ __forceinline__ void quantize(const Args& a, const Thread& t, int it, const unsigned long long (&v)[32]) {
+  const int R = 2 * a.P;
+  const int grp = blockIdx.x + it * gridDim.x;
+  const int row0 = grp * R;
+  const int nrows = min(R, a.M - row0);
+  const bool row_a = t.active && 2 * t.pr < nrows, row_b = t.active && 2 * t.pr + 1 < nrows;
+  if (!row_a) return;
+  float sum_a = 0.0f, sum_b = 0.0f;
+  {
+    const float2* src = t.partial + (it & 1) * t.nparts + ((t.pr * t.spr) >> a.seg_log);
+    const int cnt = t.spr >> a.seg_log;
+    for (int k = 0; k < cnt; ++k) {
+      const float2 p = src[k];
+      sum_a += p.x;
+      sum_b += p.y;
+    }
+  }
+  const float A_a = sum_a > 0.0f ? a.alpha_h * rsqrtf(sum_a) : 0.0f;
+  const float A_b = sum_b > 0.0f ? a.alpha_h * rsqrtf(sum_b) : 0.0f;
+  const unsigned long long NB2 = f2_pack(a.nb, a.nb);
+  const unsigned long long C2 = f2_pack(12582912.0f, 12582912.0f);  // 1.5 * 2^23
+
+  uint32_t wa[BITS], wb[BITS];
+#pragma unroll
+  for (int k = 0; k < BITS; ++k) wa[k] = wb[k] = 0u;
+#pragma unroll
+  for (int i = 0; i < 32; ++i) {
+    float xa, xb;
+    f2_unpack(v[i], xa, xb);
+    const float ya = fma_sat(xa, A_a, 0.5f), yb = fma_sat(xb, A_b, 0.5f);
+    const unsigned long long y1 = f2_pack(ya, yb);
+    uint32_t qa, qb;
+    u2_unpack(f2_fma(y1, NB2, C2), qa, qb);
+    const uint32_t ea = lds_u32((qa << 2) + t.qkey), eb = lds_u32((qb << 2) + t.qkey);
+    uint32_t da, db;
+    u2_unpack(f2_sub(u2_pack(ea, eb), y1), da, db);
+    put_code<BITS>(wa, i, ea + (da >> 31));
+    put_code<BITS>(wb, i, eb + (db >> 31));
+  }
+  const int row = row0 + 2 * t.pr;
+  const size_t rb = (size_t)(a.d / 8 * BITS);
+  uint8_t* dst = a.codes + (size_t)row * rb + (size_t)t.g * (4 * BITS);
+  store_words<BITS>(dst, wa);
+  if (row_b) store_words<BITS>(dst + rb, wb);
+  if (t.g == 0) {
+    const float s_a = sqrtf(sum_a), s_b = sqrtf(sum_b);
+    if (a.norm_f32) {
+      a.norm_f32[row] = s_a;
+      if (row_b) a.norm_f32[row + 1] = s_b;
+    }
+    if (a.norm_bf16) {
+      const __nv_bfloat16 ha = __float2bfloat16_rn(s_a), hb = __float2bfloat16_rn(s_b);
+      a.norm_bf16[row] = *reinterpret_cast<const uint16_t*>(&ha);
+      if (row_b) a.norm_bf16[row + 1] = *reinterpret_cast<const uint16_t*>(&hb);
+    }
+  }
+}
+
+template <int BITS, int LOGHB, int CFG>
+__global__ void __launch_bounds__(CFG == 2 ? 512 : 384, 1) rotq_kernel(const __grid_constant__ Args a) {
+  extern __shared__ __align__(1024) unsigned char smem[];
+  const int d = a.d, P = a.P;
+  Thread t;
+  t.tid = threadIdx.x;
+  t.lane = t.tid & 31;
+  const int warp = t.tid >> 5;
+  t.spr = d >> 5;  // 32-coordinate segments per row
+  t.active = t.tid < P * t.spr;
+  t.pr = t.active ? t.tid / t.spr : 0;  // row pair (inactive threads shadow pair 0, never store)
+  t.g = t.active ? t.tid - t.pr * t.spr : 0;
+  t.nparts = (int)(blockDim.x >> a.seg_log);
+  t.s_base = smem_u32(smem);
+  t.s_bars = t.s_base + a.bar_off;
+  t.s_ring = t.s_base + a.ring_off;
+  t.partial = reinterpret_cast<float2*>(smem + a.part_off);
+  uint32_t* qtab = reinterpret_cast<uint32_t*>(smem + a.qt_off);
+  t.qkey = smem_u32(qtab) - 0x2D000000u;  // = qtab - 4 * bits(1.5 * 2^23)
+
+  // The address arithmetic below relies on a 128-byte aligned shared window
+  // base and (byte-address forms) on every pair-buffer address fitting 16 bits.
+  if ((t.s_base & 127u) != 0u || (!Cfg<CFG>::WORD_ADDR && t.s_base + 4u * (uint32_t)(P * d) > 0xFFFFu)) {
+    if (t.tid == 0) atomicExch(a.status, OQ_ERR_UNSUPPORTED);
+    return;
+  }
+
+  if (t.tid == 0) {
+    for (int s = 0; s < a.stages; ++s)
+      asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(t.s_bars + 8u * s) : "memory");
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  for (int k = t.tid; k < a.qtable_len; k += blockDim.x) qtab[k] = __ldg(a.qtable + k);
+
+  // gather addresses: pair word of column c of pair pr sits at word
+  // pr*d + swz(c) of a pair buffer, swz swapping the 16-byte halves of odd
+  // 32-column segments (conflict-free interleave stores)
+  uint32_t offw[16];
+  {
+    const uint32_t rowbase = (uint32_t)t.pr * (uint32_t)d;
+#pragma unroll
+    for (int k = 0; k < 16; ++k) {
+      const uint32_t pw = __ldg(a.perm2 + 16 * t.g + k);
+      uint32_t c0 = pw & 0xFFFFu, c1 = pw >> 16;
+      c0 ^= ((c0 >> 5) & 1u) << 2;
+      c1 ^= ((c1 >> 5) & 1u) << 2;
+      uint32_t o0 = rowbase + c0, o1 = rowbase + c1;  // word indices
+      if constexpr (!Cfg<CFG>::WORD_ADDR) {
+        o0 = t.s_base + 4u * o0;
+        o1 = t.s_base + 4u * o1;
+      }
+      offw[k] = (o0 & 0xFFFFu) | (o1 << 16);
+    }
+  }
+  // sign bytes: byte m of sb[q] is 0x80 when coordinate 32g + 4q + m is negated
+  uint32_t sb[8];
+  {
+    const uint32_t sw = __ldg(a.signs + t.g);
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      uint32_t x = 0;
+#pragma unroll
+      for (int m = 0; m < 4; ++m) x |= ((sw >> (4 * q + m)) & 1u) << (8 * m + 7);
+      sb[q] = x;
+    }
+  }
+  // interleave addresses: 16-byte chunk c = n ^ rot of the thread's 32 columns
+  // (lane-rotated, conflict-free ring reads); odd segments swap halves
+  {
+    const uint32_t rot16 = (uint32_t)((t.g >> 1) & 3) << 4;
+    t.src_pair = ((uint32_t)t.pr * (uint32_t)d * 2u + (uint32_t)t.g * 64u) ^ rot16;
+    const uint32_t ib_seg = t.s_base + 4u * ((uint32_t)t.pr * (uint32_t)d + 32u * (uint32_t)t.g);
+    const uint32_t h0 = (uint32_t)(t.g & 1) << 4;
+    t.ib_w0 = (ib_seg + h0) ^ (rot16 << 1);
+    t.ib_w1 = (ib_seg + (16u - h0)) ^ (rot16 << 1);
+  }
+  __syncthreads();
+
+  if (warp == 0) {
+    for (int s = 0; s < a.stages; ++s) issue_stage_load<CFG>(a, t.s_ring, t.s_bars, s, t.lane);
+  }
+
+  const int n_it = a.groups > (int)blockIdx.x ? (a.groups - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
+  if (n_it == 0) return;
+  unsigned long long v[32];
+
+  // prologue: stage 0
+  bool ok = interleave<CFG>(a, t, 0);
+  if (__syncthreads_or(!ok)) return;
+  if (warp == 0) {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    issue_stage_load<CFG>(a, t.s_ring, t.s_bars, a.stages, t.lane);
+  }
+  transform<LOGHB, CFG>(a, t, 0, v, offw, sb);
+  for (int it = 0; it < n_it; ++it) {
+    const bool more = it + 1 < n_it;
+    ok = more ? interleave<CFG>(a, t, it + 1) : true;
+    if (__syncthreads_or(!ok)) return;  // partials of `it`, pair buffer of it+1, ring slot released
+    if (more && warp == 0) {
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      issue_stage_load<CFG>(a, t.s_ring, t.s_bars, it + 1 + a.stages, t.lane);
+    }
+    quantize<BITS>(a, t, it, v);
+    if (more) transform<LOGHB, CFG>(a, t, it + 1, v, offw, sb);
+  }
+}
+
+using KernelFn = void (*)(Args);
+
+// Kernels of configuration CFG for bits 1..6 and log2(h/32) 0..5 (nullptr otherwise).
+KernelFn pick_cfg0(int bits, int loghb);
+KernelFn pick_cfg1(int bits, int loghb);
+KernelFn pick_cfg2(int bits, int loghb);
+
+#define OQ_ROTQ_DEFINE_PICK(CFG)                       \
+  template <int BITS>                                  \
+  static KernelFn pick_loghb_##CFG(int loghb) {        \
+    switch (loghb) {                                   \
+      case 0: return rotq_kernel<BITS, 0, CFG>;        \
+      case 1: return rotq_kernel<BITS, 1, CFG>;        \
+      case 2: return rotq_kernel<BITS, 2, CFG>;        \
+      case 3: return rotq_kernel<BITS, 3, CFG>;        \
+      case 4: return rotq_kernel<BITS, 4, CFG>;        \
+      case 5: return rotq_kernel<BITS, 5, CFG>;        \
+    }                                                  \
+    return nullptr;                                    \
+  }                                                    \
+  KernelFn pick_cfg##CFG(int bits, int loghb) {        \
+    switch (bits) {                                    \
+      case 1: return pick_loghb_##CFG<1>(loghb);       \
+      case 2: return pick_loghb_##CFG<2>(loghb);       \
+      case 3: return pick_loghb_##CFG<3>(loghb);       \
+      case 4: return pick_loghb_##CFG<4>(loghb);       \
+      case 5: return pick_loghb_##CFG<5>(loghb);       \
+      case 6: return pick_loghb_##CFG<6>(loghb);       \
+    }                                                  \
+    return nullptr;                                    \
+  }
+
+}  // namespace rotq
+}  // namespace oq
