@@ -50,15 +50,16 @@ def load_peaks():
     return FALLBACK_PEAKS, "fallback"
 
 
-def profiled_traffic(kernel_file, summary_name):
+def profiled_traffic(kernel_files, summary_name):
     """DRAM bytes per launch from the committed ncu summary, if it was taken on
-    the current source of that kernel (matching sha256), else None."""
+    the current source of that kernel (sha256 of its source files, concatenated
+    in the order given, matching the summary's source_sha256), else None."""
     import hashlib
     path = os.path.join(ROOT, "profiles", summary_name)
-    src = os.path.join(ROOT, "calibration_free_rotated_b200", "csrc", kernel_file)
-    if not (os.path.exists(path) and os.path.exists(src)):
+    srcs = [os.path.join(ROOT, "calibration_free_rotated_b200", "csrc", f) for f in kernel_files]
+    if not (os.path.exists(path) and all(os.path.exists(s) for s in srcs)):
         return None
-    sha = hashlib.sha256(open(src, "rb").read()).hexdigest()
+    sha = hashlib.sha256(b"".join(open(s, "rb").read() for s in srcs)).hexdigest()
     vals = {}
     for line in open(path):
         if ":" in line:
@@ -328,8 +329,8 @@ def run_ours(args, world, rank, local):
     peaks, peak_kind = load_peaks()
     gemm_tflops = flops / k2_avg / 1e12
     aq_gbs = aq_bytes / k1_avg / 1e9
-    gemm_traffic = profiled_traffic("oq_cbgemm.cu", "cbgemm_flux_qkv_w4a4.md")
-    aq_traffic = profiled_traffic("oq_rotq.cu", "rotq_flux_qkv_act_w4.md")
+    gemm_traffic = profiled_traffic(["oq_cbgemm.cu"], "cbgemm_flux_qkv_w4a4.md")
+    aq_traffic = profiled_traffic(["oq_rotq.cuh", "oq_rotq.cu"], "rotq_flux_qkv_act_w4.md")
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": 1e3 * total_s / args.steps, "higher_is_better": True,

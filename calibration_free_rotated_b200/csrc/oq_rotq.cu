@@ -124,7 +124,6 @@ int launch_rotq(oq_rpbh_t r, oq_codebook_t cb, const void* X, int M, uint8_t* co
   a.d = d;
   a.P = p.P;
   a.groups = p.groups;
-  a.stages = p.stages;
   a.qtable_len = qlen;
   a.seg_log = p.seg_log;
   a.bar_off = p.bar_off;

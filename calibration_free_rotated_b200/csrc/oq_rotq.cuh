@@ -25,7 +25,7 @@ struct Args {
   const uint32_t* signs;  // sign words [d/32]
   const uint32_t* qtable;
   int* status;
-  int M, d, P, groups, stages, qtable_len, seg_log;
+  int M, d, P, groups, qtable_len, seg_log;
   uint32_t bar_off, part_off, qt_off, ring_off;  // byte offsets in dynamic shared memory
   float alpha_h;                                 // alpha / sqrt(h)
   float nb;                                      // buckets of the search table
@@ -40,6 +40,7 @@ struct Cfg {
   static constexpr uint32_t IBS = CFG == 0 ? 0x6000u : (CFG == 1 ? 0xC000u : 0x10000u);
   static constexpr uint32_t HALF = IBS / 2;  // ring: second row of each pair
   static constexpr bool WORD_ADDR = CFG == 2;
+  static constexpr int STAGES = CFG == 2 ? 1 : 2;  // ring slots (compile-time: slot and phase are shifts)
 };
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
@@ -83,7 +84,7 @@ template <int CFG>
 __device__ __forceinline__ void issue_stage_load(const Args& a, uint32_t ring, uint32_t bars, int it, int lane) {
   const int grp = blockIdx.x + it * gridDim.x;
   if (grp >= a.groups) return;
-  const int slot = it % a.stages;
+  const int slot = it % Cfg<CFG>::STAGES;
   const int R = 2 * a.P;
   const int row0 = grp * R;
   const int nrows = min(R, a.M - row0);
@@ -240,12 +241,12 @@ struct Thread {
   float2* partial;
 };
 
-// Interleave stage `it` (ring slot it % stages) into pair buffer it & 1.
+// Interleave stage `it` (ring slot it % STAGES) into pair buffer it & 1.
 template <int CFG>
 __device__ __forceinline__ bool interleave(const Args& a, const Thread& t, int it) {
   constexpr uint32_t IBS = Cfg<CFG>::IBS, HALF = Cfg<CFG>::HALF;
-  const int slot = it % a.stages;
-  const uint32_t parity = (uint32_t)(it / a.stages) & 1u;
+  const int slot = it % Cfg<CFG>::STAGES;
+  const uint32_t parity = (uint32_t)(it / Cfg<CFG>::STAGES) & 1u;
   if (!mbar_wait_bounded(t.s_bars + 8u * slot, parity, a.status)) return false;
   const uint32_t src = t.s_ring + (uint32_t)slot * IBS + t.src_pair;
   const uint32_t boff = (uint32_t)(it & 1) * IBS;
@@ -272,14 +273,18 @@ __device__ __forceinline__ void transform(const Args& a, const Thread& t, int it
   else
     Gather<CFG, LOGHB>::template run<0>(v, ss2, offw, sb, t.s_base);
   {
+#pragma unroll
+    for (int k = 0; k < 5; ++k) {
+      if (k < a.seg_log) {
+        float lo, hi;
+        f2_unpack(ss2, lo, hi);
+        ss2 = f2_add(ss2, f2_pack(__shfl_xor_sync(0xFFFFFFFFu, lo, 1 << k), __shfl_xor_sync(0xFFFFFFFFu, hi, 1 << k)));
+      }
+    }
     float lo, hi;
     f2_unpack(ss2, lo, hi);
-    const int seg = 1 << a.seg_log;
-    for (int o = 1; o < seg; o <<= 1) {
-      lo += __shfl_xor_sync(0xFFFFFFFFu, lo, o);
-      hi += __shfl_xor_sync(0xFFFFFFFFu, hi, o);
-    }
-    if ((t.lane & (seg - 1)) == 0) t.partial[(it & 1) * t.nparts + (t.tid >> a.seg_log)] = make_float2(lo, hi);
+    if ((t.lane & ((1 << a.seg_log) - 1)) == 0)
+      t.partial[(it & 1) * t.nparts + (t.tid >> a.seg_log)] = make_float2(lo, hi);
   }
   // in-thread Walsh-Hadamard butterflies over bits 0..4 of the block index
 #pragma unroll
@@ -397,7 +402,7 @@ __global__ void __launch_bounds__(CFG == 2 ? 512 : 384, 1) rotq_kernel(const __g
   }
 
   if (t.tid == 0) {
-    for (int s = 0; s < a.stages; ++s)
+    for (int s = 0; s < Cfg<CFG>::STAGES; ++s)
       asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(t.s_bars + 8u * s) : "memory");
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
@@ -448,7 +453,7 @@ __global__ void __launch_bounds__(CFG == 2 ? 512 : 384, 1) rotq_kernel(const __g
   __syncthreads();
 
   if (warp == 0) {
-    for (int s = 0; s < a.stages; ++s) issue_stage_load<CFG>(a, t.s_ring, t.s_bars, s, t.lane);
+    for (int s = 0; s < Cfg<CFG>::STAGES; ++s) issue_stage_load<CFG>(a, t.s_ring, t.s_bars, s, t.lane);
   }
 
   const int n_it = a.groups > (int)blockIdx.x ? (a.groups - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
@@ -460,7 +465,7 @@ __global__ void __launch_bounds__(CFG == 2 ? 512 : 384, 1) rotq_kernel(const __g
   if (__syncthreads_or(!ok)) return;
   if (warp == 0) {
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-    issue_stage_load<CFG>(a, t.s_ring, t.s_bars, a.stages, t.lane);
+    issue_stage_load<CFG>(a, t.s_ring, t.s_bars, Cfg<CFG>::STAGES, t.lane);
   }
   transform<LOGHB, CFG>(a, t, 0, v, offw, sb);
   for (int it = 0; it < n_it; ++it) {
@@ -469,7 +474,7 @@ __global__ void __launch_bounds__(CFG == 2 ? 512 : 384, 1) rotq_kernel(const __g
     if (__syncthreads_or(!ok)) return;  // partials of `it`, pair buffer of it+1, ring slot released
     if (more && warp == 0) {
       asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-      issue_stage_load<CFG>(a, t.s_ring, t.s_bars, it + 1 + a.stages, t.lane);
+      issue_stage_load<CFG>(a, t.s_ring, t.s_bars, it + 1 + Cfg<CFG>::STAGES, t.lane);
     }
     quantize<BITS>(a, t, it, v);
     if (more) transform<LOGHB, CFG>(a, t, it + 1, v, offw, sb);
