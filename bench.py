@@ -412,6 +412,47 @@ def run_profile_case(args):
     return 0
 
 
+def run_ablation(args):
+    """Rotation ablation ([OQ] "Rotation Ablation (Table 3)", latency column):
+    times oq_quantize_act (4-bit) under RPBH, Block-RHT (no permutation) and Full
+    RHT (d's largest power-of-two block) on N(0,1) bf16 rows.  L2 is flushed
+    (a 256 MB write) before every timed launch; CUDA events bracket the launch
+    alone.  Prints one JSON line per (shape, rotation); not the contract line."""
+    import torch
+    from calibration_free_rotated_b200 import build
+    build.build()
+    from calibration_free_rotated_b200 import orbitquant as oq
+    peaks, src = load_peaks()
+    torch.manual_seed(0)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+    d = args.d
+    for M in (args.rows, 32768):
+        X = torch.randn(M, d, device="cuda").to(torch.bfloat16)
+        codes = torch.empty(M, d // 2, dtype=torch.uint8, device="cuda")
+        norms = torch.empty(M, dtype=torch.float32, device="cuda")
+        cb = oq.Codebook(d, 4)
+        for kind, block in (("rpbh", args.block), ("block_rht", args.block), ("full_rht", 0)):
+            r = oq.Rpbh(0, d, block, kind=kind)
+            for _ in range(args.warmup):
+                oq.quantize_act(r, cb, X, codes, norms)
+            times = []
+            for _ in range(args.steps):
+                flush.zero_()
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record()
+                oq.quantize_act(r, cb, X, codes, norms)
+                e1.record()
+                e1.synchronize()
+                times.append(e0.elapsed_time(e1))
+            oq.device_status()
+            ms = statistics.median(times)
+            gbs = algorithmic(M, d, 1, 4, 4)[0] / ms / 1e6
+            print(json.dumps({"ablation": "rotation", "kind": kind, "block": r.block, "rows": M, "d": d, "bits": 4,
+                              "median_us": 1e3 * ms, "GB/s": gbs, "frac_hbm": gbs / peaks["hbm_gbs"],
+                              "peak_source": src}), flush=True)
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -420,6 +461,7 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--profile", choices=["rotq", "gemm"], help="launch one kernel only (for ncu captures)")
+    ap.add_argument("--ablation", choices=["rotation"], help="time the rotation variants of the ablation table")
     ap.add_argument("--rows", type=int, default=4608)
     ap.add_argument("--d", type=int, default=3072)
     ap.add_argument("--n", type=int, default=9216)
@@ -429,6 +471,8 @@ def main():
     args = ap.parse_args()
     if args.profile:
         return run_profile_case(args)
+    if args.ablation:
+        return run_ablation(args)
     if args.warmup < 3:
         args.warmup = 3
     world, rank, local = dist_setup()

@@ -399,11 +399,15 @@ int oq_get_device_status(void* stream) {
   return OQ_OK;
 }
 
-int oq_make_rpbh(uint64_t seed, int d, int block, oq_rpbh_t* out) {
+int oq_make_rotation(uint64_t seed, int d, int block, int kind, oq_rpbh_t* out) {
   clear_error();
   if (!out) return fail(OQ_ERR_ARG, "out is NULL");
   *out = nullptr;
   if (d < 1) return fail(OQ_ERR_ARG, "d must be >= 1 (got %d)", d);
+  if (kind != OQ_ROT_RPBH && kind != OQ_ROT_BLOCK_RHT && kind != OQ_ROT_FULL_RHT)
+    return fail(OQ_ERR_ARG, "unknown rotation kind %d", kind);
+  if (kind == OQ_ROT_FULL_RHT && block != 0 && block != (d & -d))
+    return fail(OQ_ERR_ARG, "a full RHT of d=%d has block %d (got %d)", d, d & -d, block);
   int h = block == 0 ? (d & -d) : block;
   if (h < 1 || (h & (h - 1)) != 0 || d % h != 0)
     return fail(OQ_ERR_ARG, "block %d must be a power of two dividing d=%d", block, d);
@@ -412,6 +416,7 @@ int oq_make_rpbh(uint64_t seed, int d, int block, oq_rpbh_t* out) {
   r->seed = seed;
   r->d = d;
   r->h = h;
+  r->kind = kind;
   r->perm.resize(d);
   for (int j = 0; j < d; ++j) r->perm[j] = j;
   uint64_t st = seed;
@@ -421,6 +426,9 @@ int oq_make_rpbh(uint64_t seed, int d, int block, oq_rpbh_t* out) {
     r->perm[i] = r->perm[j];
     r->perm[j] = tmp;
   }
+  // Block-RHT and Full RHT: the same draws (so the same signs), identity permutation
+  if (kind != OQ_ROT_RPBH)
+    for (int j = 0; j < d; ++j) r->perm[j] = j;
   r->sign_bits.assign((d + 31) / 32, 0u);
   for (int j = 0; j < d; ++j)
     if (splitmix64_next(st) >> 63) r->sign_bits[j >> 5] |= 1u << (j & 31);
@@ -438,6 +446,17 @@ int oq_make_rpbh(uint64_t seed, int d, int block, oq_rpbh_t* out) {
     cudaGetLastError();  // no device here: clear the sticky "no device" error
   }
   *out = r;
+  return OQ_OK;
+}
+
+int oq_make_rpbh(uint64_t seed, int d, int block, oq_rpbh_t* out) {
+  return oq_make_rotation(seed, d, block, OQ_ROT_RPBH, out);
+}
+
+int oq_rotation_kind(oq_rpbh_t r, int* kind) {
+  clear_error();
+  if (!r || !kind) return fail(OQ_ERR_ARG, "NULL argument");
+  *kind = r->kind;
   return OQ_OK;
 }
 

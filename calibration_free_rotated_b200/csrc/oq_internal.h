@@ -14,6 +14,7 @@
 struct oq_rpbh_s {
   uint64_t seed = 0;
   int d = 0, h = 0;
+  int kind = OQ_ROT_RPBH;  // OQ_ROT_*; only OQ_ROT_RPBH permutes
   std::vector<int32_t> perm;        // pi, (P x)_j = x_{pi(j)}
   std::vector<uint32_t> sign_bits;  // bit j%32 of word j/32 set <=> sign_j = -1
   std::mutex mu;

@@ -95,9 +95,13 @@ int launch_rotq(oq_rpbh_t r, oq_codebook_t cb, const void* X, int M, uint8_t* co
   const int qlen = (int)cb->qtable.size();
   if (qlen > 4097) return fail(OQ_ERR_UNSUPPORTED, "codebook d=%d bits=%d needs a %d-entry search table", cb->d, bits, qlen);
   const RotqPlan p = plan_rotq(d, h, M, qlen);
-  rotq::KernelFn kern = p.cfg == 0   ? rotq::pick_cfg0(bits, p.loghb)
-                        : p.cfg == 1 ? rotq::pick_cfg1(bits, p.loghb)
-                                     : rotq::pick_cfg2(bits, p.loghb);
+  rotq::KernelFn kern;
+  if (r->kind == OQ_ROT_RPBH)
+    kern = p.cfg == 0 ? rotq::pick_cfg0(bits, p.loghb)
+                      : (p.cfg == 1 ? rotq::pick_cfg1(bits, p.loghb) : rotq::pick_cfg2(bits, p.loghb));
+  else
+    kern = p.cfg == 0 ? rotq::pick_cfg0_np(bits, p.loghb)
+                      : (p.cfg == 1 ? rotq::pick_cfg1_np(bits, p.loghb) : rotq::pick_cfg2_np(bits, p.loghb));
   if (!kern) return fail(OQ_ERR_UNSUPPORTED, "no rotate+quantize kernel for bits=%d h=%d d=%d", bits, h, d);
 
   const uint16_t* perm;

@@ -231,12 +231,45 @@ struct Gather {
   }
 };
 
+// Gather step without a permutation (Block-RHT, Full RHT): thread (p, g)
+// reads its own 32 columns of both rows of pair p straight from ring slot SLOT
+// (no pair buffer, no interleave pass) and applies the signs while widening.
+template <int CFG>
+struct Direct {
+  template <int SLOT>
+  static __device__ __forceinline__ void run(unsigned long long (&v)[32], unsigned long long& ss2, uint32_t src,
+                                             const uint32_t (&sb)[8]) {
+    constexpr uint32_t OFF = SLOT * Cfg<CFG>::IBS, HALF = Cfg<CFG>::HALF;
+    unsigned long long sq[4] = {0ull, 0ull, 0ull, 0ull};
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      const uint4 A = lds_u128(src + OFF + 16u * c);
+      const uint4 B = lds_u128(src + OFF + HALF + 16u * c);
+      const uint32_t wa[4] = {A.x, A.y, A.z, A.w}, wb[4] = {B.x, B.y, B.z, B.w};
+#pragma unroll
+      for (int m = 0; m < 4; ++m) {
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          const int i = 8 * c + 2 * m + e;
+          const uint32_t sg = __byte_perm(sb[i >> 2], 0u, 0x0444u | ((uint32_t)(i & 3) << 12));
+          const uint32_t ra = e ? ((wa[m] & 0xFFFF0000u) ^ sg) : ((wa[m] << 16) + sg);
+          const uint32_t rb = e ? ((wb[m] & 0xFFFF0000u) ^ sg) : ((wb[m] << 16) + sg);
+          v[i] = u2_pack(ra, rb);
+          sq[i & 3] = f2_fma(v[i], v[i], sq[i & 3]);
+        }
+      }
+    }
+    ss2 = f2_add(f2_add(sq[0], sq[1]), f2_add(sq[2], sq[3]));
+  }
+};
+
 // Per-thread constants of the kernel (all registers).
 struct Thread {
   int tid, lane, pr, g, spr, nparts;
   bool active;
   uint32_t s_base, s_bars, s_ring, qkey;
   uint32_t src_pair;  // ring: row 2pr, columns 32g.., with the lane's chunk rotation
+  uint32_t src_direct;  // ring slot 0: row 2pr, columns 32g.. (no rotation)
   uint32_t ib_w0, ib_w1;
   float2* partial;
 };
@@ -264,14 +297,22 @@ __device__ __forceinline__ bool interleave(const Args& a, const Thread& t, int i
 }
 
 // Gather + signs + FWHT of stage `it`, and the segment partials of its squared norms.
-template <int LOGHB, int CFG>
+template <int LOGHB, int CFG, bool PERM>
 __device__ __forceinline__ void transform(const Args& a, const Thread& t, int it, unsigned long long (&v)[32],
                                           const uint32_t (&offw)[16], const uint32_t (&sb)[8]) {
   unsigned long long ss2;
-  if (it & 1)
-    Gather<CFG, LOGHB>::template run<1>(v, ss2, offw, sb, t.s_base);
-  else
-    Gather<CFG, LOGHB>::template run<0>(v, ss2, offw, sb, t.s_base);
+  if constexpr (PERM) {
+    if (it & 1)
+      Gather<CFG, LOGHB>::template run<1>(v, ss2, offw, sb, t.s_base);
+    else
+      Gather<CFG, LOGHB>::template run<0>(v, ss2, offw, sb, t.s_base);
+  } else {
+    static_assert(Cfg<CFG>::STAGES <= 2, "slot offsets are unrolled for two slots");
+    if (it % Cfg<CFG>::STAGES == 1)
+      Direct<CFG>::template run<1>(v, ss2, t.src_direct, sb);
+    else
+      Direct<CFG>::template run<0>(v, ss2, t.src_direct, sb);
+  }
   {
 #pragma unroll
     for (int k = 0; k < 5; ++k) {
@@ -374,7 +415,7 @@ __device__ __forceinline__ void quantize(const Args& a, const Thread& t, int it,
   }
 }
 
-template <int BITS, int LOGHB, int CFG>
+template <int BITS, int LOGHB, int CFG, bool PERM>
 __global__ void __launch_bounds__(CFG == 2 ? 512 : 384, 1) rotq_kernel(const __grid_constant__ Args a) {
   extern __shared__ __align__(1024) unsigned char smem[];
   const int d = a.d, P = a.P;
@@ -412,7 +453,7 @@ __global__ void __launch_bounds__(CFG == 2 ? 512 : 384, 1) rotq_kernel(const __g
   // pr*d + swz(c) of a pair buffer, swz swapping the 16-byte halves of odd
   // 32-column segments (conflict-free interleave stores)
   uint32_t offw[16];
-  {
+  if constexpr (PERM) {
     const uint32_t rowbase = (uint32_t)t.pr * (uint32_t)d;
 #pragma unroll
     for (int k = 0; k < 16; ++k) {
@@ -449,6 +490,7 @@ __global__ void __launch_bounds__(CFG == 2 ? 512 : 384, 1) rotq_kernel(const __g
     const uint32_t h0 = (uint32_t)(t.g & 1) << 4;
     t.ib_w0 = (ib_seg + h0) ^ (rot16 << 1);
     t.ib_w1 = (ib_seg + (16u - h0)) ^ (rot16 << 1);
+    t.src_direct = t.s_ring + (uint32_t)t.pr * (uint32_t)d * 2u + (uint32_t)t.g * 64u;
   }
   __syncthreads();
 
@@ -460,57 +502,82 @@ __global__ void __launch_bounds__(CFG == 2 ? 512 : 384, 1) rotq_kernel(const __g
   if (n_it == 0) return;
   unsigned long long v[32];
 
-  // prologue: stage 0
-  bool ok = interleave<CFG>(a, t, 0);
-  if (__syncthreads_or(!ok)) return;
-  if (warp == 0) {
-    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-    issue_stage_load<CFG>(a, t.s_ring, t.s_bars, Cfg<CFG>::STAGES, t.lane);
-  }
-  transform<LOGHB, CFG>(a, t, 0, v, offw, sb);
-  for (int it = 0; it < n_it; ++it) {
-    const bool more = it + 1 < n_it;
-    ok = more ? interleave<CFG>(a, t, it + 1) : true;
-    if (__syncthreads_or(!ok)) return;  // partials of `it`, pair buffer of it+1, ring slot released
-    if (more && warp == 0) {
+  if constexpr (PERM) {
+    // prologue: stage 0
+    bool ok = interleave<CFG>(a, t, 0);
+    if (__syncthreads_or(!ok)) return;
+    if (warp == 0) {
       asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-      issue_stage_load<CFG>(a, t.s_ring, t.s_bars, it + 1 + Cfg<CFG>::STAGES, t.lane);
+      issue_stage_load<CFG>(a, t.s_ring, t.s_bars, Cfg<CFG>::STAGES, t.lane);
     }
-    quantize<BITS>(a, t, it, v);
-    if (more) transform<LOGHB, CFG>(a, t, it + 1, v, offw, sb);
+    transform<LOGHB, CFG, PERM>(a, t, 0, v, offw, sb);
+    for (int it = 0; it < n_it; ++it) {
+      const bool more = it + 1 < n_it;
+      ok = more ? interleave<CFG>(a, t, it + 1) : true;
+      if (__syncthreads_or(!ok)) return;  // partials of `it`, pair buffer of it+1, ring slot released
+      if (more && warp == 0) {
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        issue_stage_load<CFG>(a, t.s_ring, t.s_bars, it + 1 + Cfg<CFG>::STAGES, t.lane);
+      }
+      quantize<BITS>(a, t, it, v);
+      if (more) transform<LOGHB, CFG, PERM>(a, t, it + 1, v, offw, sb);
+    }
+  } else {
+    // no permutation: each stage is read straight from its ring slot, which is
+    // released at the barrier that follows its transform
+    bool ok = mbar_wait_bounded(t.s_bars, 0u, a.status);
+    if (ok) transform<LOGHB, CFG, PERM>(a, t, 0, v, offw, sb);
+    for (int it = 0; it < n_it; ++it) {
+      if (__syncthreads_or(!ok)) return;  // partials of `it`; ring slot of `it` released
+      if (warp == 0) {
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        issue_stage_load<CFG>(a, t.s_ring, t.s_bars, it + Cfg<CFG>::STAGES, t.lane);
+      }
+      quantize<BITS>(a, t, it, v);
+      if (it + 1 < n_it) {
+        const int nx = it + 1;
+        ok = mbar_wait_bounded(t.s_bars + 8u * (nx % Cfg<CFG>::STAGES), (uint32_t)(nx / Cfg<CFG>::STAGES) & 1u,
+                               a.status);
+        if (ok) transform<LOGHB, CFG, PERM>(a, t, nx, v, offw, sb);
+      }
+    }
   }
 }
 
 using KernelFn = void (*)(Args);
 
-// Kernels of configuration CFG for bits 1..6 and log2(h/32) 0..5 (nullptr otherwise).
+// Kernels of configuration CFG for bits 1..6 and log2(h/32) 0..5 (nullptr otherwise),
+// with (RPBH) or without (Block-RHT, Full RHT) the permutation.
 KernelFn pick_cfg0(int bits, int loghb);
 KernelFn pick_cfg1(int bits, int loghb);
 KernelFn pick_cfg2(int bits, int loghb);
+KernelFn pick_cfg0_np(int bits, int loghb);
+KernelFn pick_cfg1_np(int bits, int loghb);
+KernelFn pick_cfg2_np(int bits, int loghb);
 
-#define OQ_ROTQ_DEFINE_PICK(CFG)                       \
-  template <int BITS>                                  \
-  static KernelFn pick_loghb_##CFG(int loghb) {        \
-    switch (loghb) {                                   \
-      case 0: return rotq_kernel<BITS, 0, CFG>;        \
-      case 1: return rotq_kernel<BITS, 1, CFG>;        \
-      case 2: return rotq_kernel<BITS, 2, CFG>;        \
-      case 3: return rotq_kernel<BITS, 3, CFG>;        \
-      case 4: return rotq_kernel<BITS, 4, CFG>;        \
-      case 5: return rotq_kernel<BITS, 5, CFG>;        \
-    }                                                  \
-    return nullptr;                                    \
-  }                                                    \
-  KernelFn pick_cfg##CFG(int bits, int loghb) {        \
-    switch (bits) {                                    \
-      case 1: return pick_loghb_##CFG<1>(loghb);       \
-      case 2: return pick_loghb_##CFG<2>(loghb);       \
-      case 3: return pick_loghb_##CFG<3>(loghb);       \
-      case 4: return pick_loghb_##CFG<4>(loghb);       \
-      case 5: return pick_loghb_##CFG<5>(loghb);       \
-      case 6: return pick_loghb_##CFG<6>(loghb);       \
-    }                                                  \
-    return nullptr;                                    \
+#define OQ_ROTQ_DEFINE_PICK(NAME, CFG, PERM)                \
+  template <int BITS>                                       \
+  static KernelFn NAME##_loghb(int loghb) {                 \
+    switch (loghb) {                                        \
+      case 0: return rotq_kernel<BITS, 0, CFG, PERM>;       \
+      case 1: return rotq_kernel<BITS, 1, CFG, PERM>;       \
+      case 2: return rotq_kernel<BITS, 2, CFG, PERM>;       \
+      case 3: return rotq_kernel<BITS, 3, CFG, PERM>;       \
+      case 4: return rotq_kernel<BITS, 4, CFG, PERM>;       \
+      case 5: return rotq_kernel<BITS, 5, CFG, PERM>;       \
+    }                                                       \
+    return nullptr;                                         \
+  }                                                         \
+  KernelFn NAME(int bits, int loghb) {                      \
+    switch (bits) {                                         \
+      case 1: return NAME##_loghb<1>(loghb);                \
+      case 2: return NAME##_loghb<2>(loghb);                \
+      case 3: return NAME##_loghb<3>(loghb);                \
+      case 4: return NAME##_loghb<4>(loghb);                \
+      case 5: return NAME##_loghb<5>(loghb);                \
+      case 6: return NAME##_loghb<6>(loghb);                \
+    }                                                       \
+    return nullptr;                                         \
   }
 
 }  // namespace rotq

@@ -1,9 +1,9 @@
 // Instantiations of the rotate+quantize kernel for configuration 2
-// (12288 < d <= 16384: 64 KB pair buffers, word gather addresses).
+// (12288 < d <= 16384: 64 KB pair buffers, word gather addresses), RPBH (with the permutation).
 #include "oq_rotq.cuh"
 
 namespace oq {
 namespace rotq {
-OQ_ROTQ_DEFINE_PICK(2)
+OQ_ROTQ_DEFINE_PICK(pick_cfg2, 2, true)
 }  // namespace rotq
 }  // namespace oq

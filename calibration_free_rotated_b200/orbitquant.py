@@ -16,6 +16,7 @@ LIB_PATH = os.path.join(_HERE, "liborbitquant.so")
 
 OQ_OK, OQ_ERR_ARG, OQ_ERR_UNSUPPORTED, OQ_ERR_ALIGN, OQ_ERR_CUDA, OQ_ERR_TIMEOUT, OQ_ERR_NOMEM = range(7)
 EPILOGUES = {"none": 0, "gelu": 1}
+ROTATIONS = {"rpbh": 0, "block_rht": 1, "full_rht": 2}  # OQ_ROT_*
 
 if not os.path.exists(LIB_PATH):
     raise ImportError(
@@ -30,6 +31,8 @@ _SIGS = {
     "oq_last_error": (ctypes.c_char_p, []),
     "oq_get_device_status": (_c_int, [_c_void_p]),
     "oq_make_rpbh": (_c_int, [ctypes.c_uint64, _c_int, _c_int, ctypes.POINTER(_c_void_p)]),
+    "oq_make_rotation": (_c_int, [ctypes.c_uint64, _c_int, _c_int, _c_int, ctypes.POINTER(_c_void_p)]),
+    "oq_rotation_kind": (_c_int, [_c_void_p, ctypes.POINTER(_c_int)]),
     "oq_rpbh_info": (_c_int, [_c_void_p, ctypes.POINTER(_c_int), ctypes.POINTER(_c_int)]),
     "oq_rpbh_export": (_c_int, [_c_void_p, _c_void_p, _c_void_p]),
     "oq_free_rpbh": (None, [_c_void_p]),
@@ -82,15 +85,18 @@ def _stream(stream):
 
 
 class Rpbh:
-    """Handle of the RPBH rotation for one (seed, d, block)."""
+    """Handle of the RPBH rotation for one (seed, d, block); `kind` selects a
+    variant of the rotation ablation ("rpbh", "block_rht", "full_rht")."""
 
-    def __init__(self, seed: int, d: int, block: int = 0):
+    def __init__(self, seed: int, d: int, block: int = 0, kind: str = "rpbh"):
         h = ctypes.c_void_p()
-        _check(_lib.oq_make_rpbh(seed, d, block, ctypes.byref(h)))
+        _check(_lib.oq_make_rotation(seed, d, block, ROTATIONS[kind], ctypes.byref(h)))
         self._h = h
-        dd, bb = ctypes.c_int(), ctypes.c_int()
+        dd, bb, kk = ctypes.c_int(), ctypes.c_int(), ctypes.c_int()
         _check(_lib.oq_rpbh_info(h, ctypes.byref(dd), ctypes.byref(bb)))
+        _check(_lib.oq_rotation_kind(h, ctypes.byref(kk)))
         self.seed, self.d, self.block = seed, dd.value, bb.value
+        self.kind = {v: k for k, v in ROTATIONS.items()}[kk.value]
 
     @property
     def handle(self):

@@ -93,6 +93,26 @@ OQ_API int oq_get_device_status(void* stream);
  * ------------------------------------------------------------------------- */
 OQ_API int oq_make_rpbh(uint64_t seed, int d, int block, oq_rpbh_t* out);
 
+/* ---------------------------------------------------------------------------
+ * Rotation variants of the rotation ablation ([OQ] Experiments, "Rotation
+ * Ablation (Table 3)"), as rotation handles that every entry point accepts:
+ *   OQ_ROT_RPBH       blkdiag(H_h D_1..) P_pi, exactly oq_make_rpbh.
+ *   OQ_ROT_BLOCK_RHT  "Block-RHT (no perm)": blkdiag(H_h D_1..), P = I.  The
+ *                     signs are those RPBH draws for the same seed (the
+ *                     generator still runs through the Fisher-Yates draws), so
+ *                     the two differ only by the permutation.
+ *   OQ_ROT_FULL_RHT   "Full RHT": one Hadamard block spanning the largest power
+ *                     of two dividing d (all of d when d is a power of two),
+ *                     P = I, the same signs.  `block` must be 0 or that size.
+ * (The table's dense Haar rotation is a comparison system and is not built.)
+ * Errors: as oq_make_rpbh; OQ_ERR_ARG for an unknown kind or a FULL_RHT block
+ * other than 0 or d's largest power-of-two divisor.
+ * ------------------------------------------------------------------------- */
+enum { OQ_ROT_RPBH = 0, OQ_ROT_BLOCK_RHT = 1, OQ_ROT_FULL_RHT = 2 };
+OQ_API int oq_make_rotation(uint64_t seed, int d, int block, int kind, oq_rpbh_t* out);
+/* Kind (OQ_ROT_*) of a rotation handle. */
+OQ_API int oq_rotation_kind(oq_rpbh_t r, int* kind);
+
 /* d and h of a handle.  Either output may be NULL. */
 OQ_API int oq_rpbh_info(oq_rpbh_t r, int* d, int* block);
 

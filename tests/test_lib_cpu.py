@@ -108,3 +108,28 @@ def test_workspace_bytes(oq):
     assert oq.workspace_bytes(4608, 3072, 4) == 4608 * 3072 // 2 + 4 * 4608
     assert oq.workspace_bytes(3, 64, 6) == 256 + 12
     assert oq.workspace_bytes(0, 64, 4) == 0
+
+
+@pytest.mark.parametrize("seed,d,block", [(0, 3072, 128), (5, 256, 64), (9, 1536, 0)])
+def test_rotation_variants_share_the_rpbh_signs(oq, seed, d, block):
+    # [OQ] "Rotation Ablation (Table 3)": Block-RHT is RPBH without P (same
+    # draws, so the same signs); Full RHT spans d's largest power-of-two block.
+    _, rpbh_signs = oq.Rpbh(seed, d, block).export()
+    for kind in ("block_rht", "full_rht"):
+        r = oq.Rpbh(seed, d, 0 if kind == "full_rht" else block, kind=kind)
+        perm, signs = r.export()
+        assert r.kind == kind
+        assert np.array_equal(perm, np.arange(d, dtype=np.int32))
+        assert np.array_equal(signs, rpbh_signs)
+        if kind == "full_rht":
+            assert r.block == (d & -d) == orpbh.default_block(d)
+        else:
+            assert r.block == (block or orpbh.default_block(d))
+
+
+def test_rotation_variant_errors(oq):
+    with pytest.raises(oq.OQError):
+        oq.Rpbh(0, 3072, 128, kind="full_rht")  # a full RHT of 3072 has block 1024
+    h = ctypes.c_void_p()
+    assert oq.lib().oq_make_rotation(0, 256, 64, 7, ctypes.byref(h)) == oq.OQ_ERR_ARG
+    assert oq.Rpbh(0, 3072, 1024, kind="full_rht").block == 1024

@@ -37,10 +37,10 @@ def oq():
 _handles = {}
 
 
-def _lib_handles(oq, seed, d, h, bits):
-    key = (seed, d, h, bits)
+def _lib_handles(oq, seed, d, h, bits, kind="rpbh"):
+    key = (seed, d, h, bits, kind)
     if key not in _handles:
-        _handles[key] = (oq.Rpbh(seed, d, h), oq.Codebook(d, bits))
+        _handles[key] = (oq.Rpbh(seed, d, h, kind=kind), oq.Codebook(d, bits))
     return _handles[key]
 
 
@@ -48,9 +48,9 @@ def _to_dev(bits_u16):
     return torch.from_numpy(np.ascontiguousarray(bits_u16).view(np.int16)).cuda().view(torch.bfloat16)
 
 
-def _check_rows(oq, codebooks, X_bits, d, h, bits, seed=0, weight=False, rows=None, report=None):
+def _check_rows(oq, codebooks, X_bits, d, h, bits, seed=0, weight=False, rows=None, report=None, kind="rpbh"):
     """Runs the kernel on all of X_bits; checks rows `rows` (default all) against the oracle."""
-    r, cb = _lib_handles(oq, seed, d, h, bits)
+    r, cb = _lib_handles(oq, seed, d, h, bits, kind)
     X = _to_dev(X_bits)
     if weight:
         codes, norms = oq.quantize_weight(r, cb, X)
@@ -65,6 +65,8 @@ def _check_rows(oq, codebooks, X_bits, d, h, bits, seed=0, weight=False, rows=No
     else:
         norms_np = norms.cpu().numpy()[rows]
     perm, signs = orpbh.draw_permutation_and_signs(seed, d)
+    if kind != "rpbh":  # Block-RHT / Full RHT: the same signs, no permutation
+        perm = np.arange(d)
     ref = codebooks(d, bits)
     xs = inputs.bf16_bits_to_f64(X_bits[rows])
     if weight:
@@ -179,3 +181,27 @@ def test_sweep_largest_full_size_sampled(oq, codebooks):
     X = inputs.sweep_activations(M, d)
     rows = np.concatenate([np.linspace(0, M - 1, 24).astype(int), np.arange(M - 8, M)])
     _check_rows(oq, codebooks, X, d, 256, 2, rows=rows)
+
+
+@pytest.mark.parametrize("d,h,kind,bits", [(3072, 128, "block_rht", 4), (3072, 1024, "full_rht", 4),
+                                           (1024, 1024, "full_rht", 2), (256, 64, "block_rht", 6),
+                                           (1536, 128, "block_rht", 3), (8960, 128, "block_rht", 4),
+                                           (12288, 128, "block_rht", 2), (16384, 1024, "block_rht", 4)])
+def test_rotation_variants(oq, codebooks, d, h, kind, bits):
+    # [OQ] "Rotation Ablation (Table 3)": Block-RHT (no permutation) and Full RHT
+    # against the oracle with the identity permutation and the RPBH signs;
+    # ragged tails, sparse rows and a zero row included
+    M = 300 if d >= 8192 else 1000
+    X = inputs.sweep_activations(M, d)
+    rep = []
+    _check_rows(oq, codebooks, X, d, h, bits, kind=kind, report=rep)
+    assert rep[0][0] <= rep[0][1]
+    if d == 3072:
+        W = inputs.weights(2, inputs.T_W, 200, d)
+        _check_rows(oq, codebooks, W, d, h, bits, weight=True, kind=kind)
+
+
+def test_widest_rows_rpbh(oq, codebooks):
+    # d = 16384, the widest row the kernels take (one row pair per stage)
+    X = inputs.sweep_activations(130, 16384)
+    _check_rows(oq, codebooks, X, 16384, 256, 4)
