@@ -14,6 +14,7 @@ of the same workload; it is the deliberately slow program the ratio divides by.
 
 import argparse
 import json
+import math
 import os
 import statistics
 import sys
@@ -453,6 +454,163 @@ def run_ablation(args):
     return 0
 
 
+def _flush_and_time(fn, flush, steps, warmup):
+    """Median CUDA-event time (ms) of fn() with a 256 MB L2 flush before each call."""
+    import torch
+    for _ in range(warmup):
+        fn()
+    times = []
+    for _ in range(steps):
+        flush.zero_()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        fn()
+        e1.record()
+        e1.synchronize()
+        times.append(e0.elapsed_time(e1))
+    return statistics.median(times)
+
+
+def run_workload(args):
+    """Per-kernel times of the two-layer workloads (one JSON line each; not the
+    contract line).  flux_mlp: X[4608 x 3072] -> fc1 [12288 x 3072] + GELU ->
+    fc2 [3072 x 12288], W2A4, block 128.  wan_ffn: X[32760 x 1536] Student-t(3)
+    -> fc1 [8960 x 1536] + GELU -> fc2 [1536 x 8960], W4A6, block 128.  Every
+    launch is timed alone after a 256 MB L2 flush."""
+    import torch
+    from calibration_free_rotated_b200 import build
+    build.build()
+    from calibration_free_rotated_b200 import inputs
+    from calibration_free_rotated_b200 import orbitquant as oq
+    peaks, src = load_peaks()
+    wl, M, d1, d2, bw, ba = {"flux_mlp": (3, 4608, 3072, 12288, 2, 4),
+                             "wan_ffn": (4, 32760, 1536, 8960, 4, 6)}[args.workload]
+    h = 128
+    dev = torch.device("cuda")
+    bf = lambda bits: torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).to(dev).view(torch.bfloat16)
+    X = bf(inputs.activations(wl, M, d1))
+    r1, r2 = oq.Rpbh(0, d1, h), oq.Rpbh(0, d2, h)
+    ca1, cw1, ca2, cw2 = oq.Codebook(d1, ba), oq.Codebook(d1, bw), oq.Codebook(d2, ba), oq.Codebook(d2, bw)
+    w1c, w1n = oq.quantize_weight(r1, cw1, bf(inputs.weights(wl, inputs.T_W, d2, d1)))
+    w2c, w2n = oq.quantize_weight(r2, cw2, bf(inputs.weights(wl, inputs.T_W2, d1, d2)))
+    a1c, a1n = oq.quantize_act(r1, ca1, X)
+    Y1 = torch.empty((M, d2), dtype=torch.bfloat16, device=dev)
+    a2c = torch.empty((M, d2 * ba // 8), dtype=torch.uint8, device=dev)
+    a2n = torch.empty((M,), dtype=torch.float32, device=dev)
+    Y2 = torch.empty((M, d1), dtype=torch.bfloat16, device=dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    steps = [
+        ("act_quant_1", lambda: oq.quantize_act(r1, ca1, X, a1c, a1n), "hbm", algorithmic(M, d1, d2, ba, bw)[0]),
+        ("fc1_gelu", lambda: oq.linear_codes(d1, ca1, cw1, a1c, a1n, w1c, w1n, epilogue="gelu", out_bf16=Y1,
+                                             want_f32=False, want_bf16=True), "tensor", 2.0 * M * d1 * d2),
+        ("act_quant_2", lambda: oq.quantize_act(r2, ca2, Y1, a2c, a2n), "hbm", algorithmic(M, d2, d1, ba, bw)[0]),
+        ("fc2", lambda: oq.linear_codes(d2, ca2, cw2, a2c, a2n, w2c, w2n, out_bf16=Y2, want_f32=False,
+                                        want_bf16=True), "tensor", 2.0 * M * d1 * d2),
+    ]
+    out = {"workload": args.workload, "M": M, "d_in": d1, "d_hidden": d2, "bits_w": bw, "bits_a": ba, "block": h,
+           "kernels": {}, "peak_source": src}
+    total = 0.0
+    for name, fn, bound, work in steps:
+        ms = _flush_and_time(fn, flush, args.steps, args.warmup)
+        total += ms
+        if bound == "hbm":
+            ach = work / ms / 1e6
+            out["kernels"][name] = {"ms": ms, "GB/s": ach, "frac": ach / peaks["hbm_gbs"]}
+        else:
+            ach = work / ms / 1e9
+            out["kernels"][name] = {"ms": ms, "TFLOP/s": ach, "frac": ach / peaks["bf16_tflops"]}
+    oq.device_status()
+    out["step_ms"] = total
+    out["TFLOP/s"] = 4.0 * M * d1 * d2 / total / 1e9
+    print(json.dumps(out), flush=True)
+    return 0
+
+
+def _sylvester(h, device):
+    import torch
+    H = torch.ones((1, 1), dtype=torch.float64, device=device)
+    while H.shape[0] < h:
+        H = torch.cat([torch.cat([H, H], 1), torch.cat([H, -H], 1)], 0)
+    return H
+
+
+def run_sweep(args):
+    """The standalone rotate+quantize sweep: M in {1k, 16k, 64k} x d in {1536,
+    3072, 12288} x block {64, 128, 256} x bits {2, 4, 6} on N(0,1) rows whose
+    last M/8 are one-hot / k-sparse (one zero row).  Per run: the kernel's time
+    (L2 flushed, CUDA events), GB/s against the measured HBM copy rate, and the
+    empirical per-row squared error ||t - c[code]||^2 of the unit rotated rows
+    (dense rows and sparse rows apart, up to 4096 of each) next to the Lloyd-Max
+    distortion d * D(d, b) of the codebook.  The error is measured with a
+    separate torch rotation (fp64) of the exported permutation and signs; the
+    codes are the kernel's.  One JSON line per run."""
+    import torch
+    from calibration_free_rotated_b200 import build
+    build.build()
+    from calibration_free_rotated_b200 import inputs
+    from calibration_free_rotated_b200 import orbitquant as oq
+    peaks, src = load_peaks()
+    dev = torch.device("cuda")
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    Ms = [int(x) for x in args.sweep_rows.split(",")]
+    for d in (1536, 3072, 12288):
+        for M in Ms:
+            X = torch.empty((M, d), dtype=torch.bfloat16, device=dev)
+            for r0 in range(0, M, 8192):  # generated in row blocks to bound host memory
+                r1 = min(M, r0 + 8192)
+                Xb = inputs.sweep_activations(M, d, rows=(r0, r1))
+                X[r0:r1] = torch.from_numpy(np.ascontiguousarray(Xb).view(np.int16)).to(dev).view(torch.bfloat16)
+            n_adv = M // 8
+            rows_dense = torch.arange(0, min(4096, M - n_adv), device=dev)
+            rows_adv = torch.arange(M - n_adv, min(M - 1, M - n_adv + 4096), device=dev)  # not the zero row
+            for h in (64, 128, 256):
+                r = oq.Rpbh(0, d, h)
+                perm, sbits = r.export()
+                sign = torch.tensor([-1.0 if (sbits[j >> 5] >> (j & 31)) & 1 else 1.0 for j in range(d)],
+                                    dtype=torch.float64, device=dev)
+                perm_t = torch.from_numpy(perm.astype(np.int64)).to(dev)
+                H = _sylvester(h, dev) / math.sqrt(h)
+
+                def unit_rotated(rows):
+                    x = X[rows].double()[:, perm_t] * sign
+                    u = (x.view(len(rows), d // h, h) @ H.T).view(len(rows), d)
+                    return u / u.norm(dim=1, keepdim=True).clamp_min(1e-300)
+
+                T = {"dense": unit_rotated(rows_dense), "adversarial": unit_rotated(rows_adv)}
+                for bits in (2, 4, 6):
+                    cb = oq.Codebook(d, bits)
+                    ex = cb.export()
+                    c, D = ex["centroids"], ex["distortion"]
+                    codes = torch.empty((M, d * bits // 8), dtype=torch.uint8, device=dev)
+                    norms = torch.empty((M,), dtype=torch.float32, device=dev)
+                    ms = _flush_and_time(lambda: oq.quantize_act(r, cb, X, codes, norms), flush, args.steps,
+                                         args.warmup)
+                    gbs = algorithmic(M, d, 1, bits, bits)[0] / ms / 1e6
+                    cent = torch.from_numpy(np.asarray(c, dtype=np.float64)).to(dev)
+                    line = {"sweep": "rotate_quantize", "M": M, "d": d, "block": h, "bits": bits, "median_us": 1e3 * ms,
+                            "GB/s": gbs, "frac_hbm": gbs / peaks["hbm_gbs"], "peak_source": src,
+                            "mse_theory": d * D}
+                    for key, rows in (("dense", rows_dense), ("adversarial", rows_adv)):
+                        k = _unpack_codes_torch(codes[rows], bits, d)
+                        err = ((T[key] - cent[k]) ** 2).sum(dim=1)
+                        line["mse_" + key] = float(err.mean())
+                    print(json.dumps(line), flush=True)
+            del X
+    oq.device_status()
+    return 0
+
+
+def _unpack_codes_torch(packed, bits, d):
+    """Little-endian bit stream [rows, d*bits/8] -> int64 codes [rows, d]."""
+    import torch
+    b = packed.to(torch.int64)
+    bitpos = torch.arange(d, device=packed.device) * bits
+    byte, sh = bitpos // 8, bitpos % 8
+    lo = b[:, byte]
+    hi = b[:, torch.clamp(byte + 1, max=packed.shape[1] - 1)]
+    return ((lo | (hi << 8)) >> sh) & ((1 << bits) - 1)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -462,6 +620,9 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--profile", choices=["rotq", "gemm"], help="launch one kernel only (for ncu captures)")
     ap.add_argument("--ablation", choices=["rotation"], help="time the rotation variants of the ablation table")
+    ap.add_argument("--workload", choices=["flux_mlp", "wan_ffn"], help="per-kernel times of a two-layer workload")
+    ap.add_argument("--sweep", action="store_true", help="the rotate+quantize sweep with empirical MSE")
+    ap.add_argument("--sweep-rows", default="1024,16384,65536")
     ap.add_argument("--rows", type=int, default=4608)
     ap.add_argument("--d", type=int, default=3072)
     ap.add_argument("--n", type=int, default=9216)
@@ -473,6 +634,10 @@ def main():
         return run_profile_case(args)
     if args.ablation:
         return run_ablation(args)
+    if args.workload:
+        return run_workload(args)
+    if args.sweep:
+        return run_sweep(args)
     if args.warmup < 3:
         args.warmup = 3
     world, rank, local = dist_setup()
