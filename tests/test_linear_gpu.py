@@ -241,3 +241,27 @@ def test_empty_shapes(oq):
                              torch.ones(32, dtype=torch.bfloat16, device="cuda"))
     assert y32.shape == (0, 32)
     oq.device_status()
+
+
+def test_gelu_epilogue_matches_exact_erf(oq):
+    # The GELU epilogue against the exact erf form, 0.5 y (1 + erf(y / sqrt 2)),
+    # evaluated in fp64 on the host on the kernel's own pre-activation output
+    # (the same launch without the epilogue): isolates the GELU arithmetic.
+    # Random codes and norms scaled so that y spans roughly [-12, 12].
+    torch.manual_seed(3)
+    M, N, d = 200, 272, 256
+    ca, cw = _lib_cb(oq, d, 4), _lib_cb(oq, d, 4)
+    a = torch.randint(0, 256, (M, d // 2), dtype=torch.uint8, device="cuda")
+    w = torch.randint(0, 256, (N, d // 2), dtype=torch.uint8, device="cuda")
+    an = torch.rand(M, device="cuda") * 6.0
+    wn = (torch.rand(N, device="cuda") * 6.0).to(torch.bfloat16)
+    bias = (torch.randn(N, device="cuda") * 2.0).to(torch.bfloat16)
+    pre, _ = oq.linear_codes(d, ca, cw, a, an, w, wn, bias=bias, epilogue="none")
+    got, _ = oq.linear_codes(d, ca, cw, a, an, w, wn, bias=bias, epilogue="gelu")
+    torch.cuda.synchronize()
+    oq.device_status()
+    y = pre.double().cpu().numpy()
+    assert y.min() < -6.0 and y.max() > 6.0
+    ref = np.vectorize(lambda v: 0.5 * v * (1.0 + math.erf(v / math.sqrt(2.0))))(y)
+    err = np.abs(got.double().cpu().numpy() - ref)
+    assert err.max() <= 2e-6 * max(1.0, float(np.abs(y).max()))
