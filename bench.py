@@ -297,31 +297,55 @@ def run_ours(args, world, rank, local):
     aq_bytes, flops = algorithmic(M, K, N, 4, 4)
     value = whole_job_value(flops * args.steps, world, total_s) / 1e12
 
-    # end to end through the public oq_linear call with host buffers
-    Xh = torch.empty((M, K), dtype=torch.bfloat16, pin_memory=True)
-    Xh.copy_(X0.cpu())
-    Yh = torch.empty((M, N), dtype=torch.bfloat16, pin_memory=True)
-    ws = torch.empty((oq.workspace_bytes(M, K, 4),), dtype=torch.uint8, device=dev)
-    Xd = torch.empty_like(X0)
-    Yd = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+    # end to end through the public oq_linear call with host buffers: every step
+    # uploads its X from pinned host memory and reads its Y back.  Steps are
+    # pipelined the way a caller would: upload of step i+1 and download of step
+    # i-1 run on their own copy streams while step i computes (two device
+    # buffer sets; events order each step's copy -> compute -> copy).
+    n_e2e = 2
+    Xh = [torch.empty((M, K), dtype=torch.bfloat16, pin_memory=True) for _ in range(n_e2e)]
+    Yh = [torch.empty((M, N), dtype=torch.bfloat16, pin_memory=True) for _ in range(n_e2e)]
+    for xh in Xh:
+        xh.copy_(X0.cpu())
+    ws = [torch.empty((oq.workspace_bytes(M, K, 4),), dtype=torch.uint8, device=dev) for _ in range(n_e2e)]
+    Xd = [torch.empty_like(X0) for _ in range(n_e2e)]
+    Yd = [torch.empty((M, N), dtype=torch.bfloat16, device=dev) for _ in range(n_e2e)]
+    s_in, s_out = torch.cuda.Stream(), torch.cuda.Stream()
+    ev_in = [torch.cuda.Event() for _ in range(n_e2e)]
+    ev_done = [torch.cuda.Event() for _ in range(n_e2e)]
+    ev_out = [torch.cuda.Event() for _ in range(n_e2e)]
+    for e in ev_out:
+        e.record(s_out)
 
-    def e2e_step():
-        Xd.copy_(Xh, non_blocking=True)
-        oq.linear(r, cb, cb, Xd, wc0, wn, bias=bias, out_bf16=Yd, want_f32=False, want_bf16=True, workspace=ws,
-                  stream=stream)
-        Yh.copy_(Yd, non_blocking=True)
+    def e2e_step(i):
+        b = i % n_e2e
+        s_in.wait_event(ev_done[b])  # device X buffer b is free once step i-2 has computed
+        with torch.cuda.stream(s_in):
+            Xd[b].copy_(Xh[b], non_blocking=True)
+        ev_in[b].record(s_in)
+        stream.wait_event(ev_in[b])
+        stream.wait_event(ev_out[b])  # Y buffer b has been read back (step i-2)
+        oq.linear(r, cb, cb, Xd[b], wc0, wn, bias=bias, out_bf16=Yd[b], want_f32=False, want_bf16=True,
+                  workspace=ws[b], stream=stream)
+        ev_done[b].record(stream)
+        s_out.wait_event(ev_done[b])
+        with torch.cuda.stream(s_out):
+            Yh[b].copy_(Yd[b], non_blocking=True)
+        ev_out[b].record(s_out)
 
-    for _ in range(max(1, args.warmup)):
-        e2e_step()
+    for e in ev_done:
+        e.record(stream)
+    for i in range(max(1, args.warmup)):
+        e2e_step(i)
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
-    e0.record(stream)
-    for _ in range(args.steps):
-        e2e_step()
-    e1.record(stream)
+    e0.record(s_in)  # the first upload starts the timed region
+    for i in range(args.steps):
+        e2e_step(i)
+    e1.record(s_out)  # the last download ends it
     torch.cuda.synchronize()
     e2e_s = reduce_max([e0.elapsed_time(e1) / 1e3], world)[0]
     oq.device_status()
