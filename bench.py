@@ -106,13 +106,17 @@ class ClockSampler:
                         self.reasons.add(name)
             except Exception:
                 pass
-            if self._stop.wait(0.005):
+            self._started.set()
+            if self._stop.wait(0.001):
                 break
 
     def __enter__(self):
         if self._nv is not None:
+            self._started = threading.Event()
             self._t = threading.Thread(target=self._poll, daemon=True)
             self._t.start()
+            self._started.wait(1.0)  # polling before the timed work is enqueued
+            self.samples.clear()
         return self
 
     def __exit__(self, *exc):

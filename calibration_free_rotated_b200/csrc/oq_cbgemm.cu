@@ -396,18 +396,22 @@ __device__ __forceinline__ uint4 expand8(uint64_t packed, const Lut8& t8, uint32
   if constexpr (BITS == 4) {
     r = expand8_nib((uint32_t)packed, t8);
   } else if constexpr (BITS == 2) {
-    // Selector nibbles (2c0, 2c0+1, 2c1, 2c1+1) pick two fp16 from the 4-entry table
-    // {q1:q0}.  With z = c0 + 4 c1: sel = 0x1010 + 0x22 z + 0x2178 c1 (no carries
-    // into bit 16; the byte permute reads only the low 16 bits of its selector).
-    const uint32_t w = (uint32_t)packed;
-    uint32_t o[4];
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const uint32_t z = (i == 0 ? w : shr_imad<4>(i == 1 ? w : (i == 2 ? shr_imad<4>(w) : shr_imad<8>(w)))) & 0xFu;
-      const uint32_t c1 = shr_imad<2>(z);
-      o[i] = prmt(q0, q1, c1 * 0x2178u + (z * 0x22u + 0x1010u));
-    }
-    r = make_uint4(o[0], o[1], o[2], o[3]);
+    // q0 / q1 are the low / high byte planes of the 4-entry table.  The eight
+    // 2-bit codes are spread to one code per nibble (three shift-mask steps,
+    // shifts on the IMAD pipe); each nibble then selects its entry's bytes
+    // from the planes, and the bytes interleave into fp16 pairs.
+    uint32_t n = (uint32_t)packed & 0xFFFFu;
+    n = (n | mul_lo(n, 1u << 8)) & 0x00FF00FFu;
+    n = (n | mul_lo(n, 1u << 4)) & 0x0F0F0F0Fu;
+    n = (n | mul_lo(n, 1u << 2)) & 0x33333333u;  // nibble i = code i
+    const uint32_t n_hi = shr_imad<16>(n);
+    uint32_t lo = prmt(q0, q0, n), hi = prmt(q1, q1, n);
+    r.x = prmt(lo, hi, 0x5140u);
+    r.y = prmt(lo, hi, 0x7362u);
+    lo = prmt(q0, q0, n_hi);
+    hi = prmt(q1, q1, n_hi);
+    r.z = prmt(lo, hi, 0x5140u);
+    r.w = prmt(lo, hi, 0x7362u);
   } else {  // 6 bits: shared 64-entry table
     uint32_t o[4];
 #pragma unroll
@@ -657,8 +661,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     const int g = warp / GROUP_WARPS, q = warp % GROUP_WARPS;
     const int r = 32 * q + lane;
     Lut8 ta, tw;
-    const uint32_t qa0 = args.lut_a[0], qa1 = args.lut_a[1];
-    const uint32_t qw0 = args.lut_w[0], qw1 = args.lut_w[1];
+    // 2-bit tables as byte planes (low bytes of the 4 entries, high bytes)
+    const uint32_t qa0 = prmt(args.lut_a[0], args.lut_a[1], 0x6420), qa1 = prmt(args.lut_a[0], args.lut_a[1], 0x7531);
+    const uint32_t qw0 = prmt(args.lut_w[0], args.lut_w[1], 0x6420), qw1 = prmt(args.lut_w[0], args.lut_w[1], 0x7531);
     if constexpr (BA == 4) ta = make_lut8(args.lut_a);
     if constexpr (BW == 4) tw = make_lut8(args.lut_w);
     constexpr int RB_A = PackedTile<BA>::kRowBytes, RB_B = PackedTile<BW>::kRowBytes;
