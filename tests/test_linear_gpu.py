@@ -265,3 +265,33 @@ def test_gelu_epilogue_matches_exact_erf(oq):
     ref = np.vectorize(lambda v: 0.5 * v * (1.0 + math.erf(v / math.sqrt(2.0))))(y)
     err = np.abs(got.double().cpu().numpy() - ref)
     assert err.max() <= 2e-6 * max(1.0, float(np.abs(y).max()))
+
+
+@pytest.mark.parametrize("kind,h", [("block_rht", 64), ("full_rht", 0)])
+def test_full_layer_with_rotation_variants(oq, codebooks, kind, h):
+    # The rotation cancels in the product for every orthogonal rotation ([OQ]
+    # "Online Activation Quantization", last paragraph): oq_linear with the
+    # Block-RHT / Full RHT handles against the oracle on the same rotation
+    # (identity permutation, RPBH signs).
+    d, M, N = 256, 96, 160
+    r = oq.Rpbh(0, d, h, kind=kind)
+    hh = r.block
+    X = inputs.activations(1, M, d)
+    W = inputs.weights(1, inputs.T_W, N, d)
+    cb = _lib_cb(oq, d, 4)
+    wc, wn = oq.quantize_weight(r, cb, _dev_bf16(W))
+    y, _ = oq.linear(r, cb, cb, _dev_bf16(X), wc, wn)
+    torch.cuda.synchronize()
+    oq.device_status()
+    _, signs = orpbh.draw_permutation_and_signs(0, d)
+    perm = np.arange(d)
+    c = codebooks(d, 4)["centroids"]
+    ca, s, T = oqz.quantize_rows(inputs.bf16_bits_to_f64(X), perm, signs, hh, c)
+    cw, r16, _, Tw = oqz.quantize_weight_rows(inputs.bf16_bits_to_f64(W), perm, signs, hh, c)
+    # rows/columns whose codes all agree with the oracle (in-band flips aside)
+    got_a = oqz.unpack_codes(oq.quantize_act(r, cb, _dev_bf16(X))[0].cpu().numpy(), 4, d)
+    got_w = oqz.unpack_codes(wc.cpu().numpy(), 4, d)
+    rows, cols = (got_a == ca).all(axis=1), (got_w == cw).all(axis=1)
+    assert rows.sum() > M // 2 and cols.sum() > N // 2
+    ref = olin.linear_from_codes(ca, s, cw, r16, c, c, d)
+    assert _rel_fro(y.double().cpu().numpy()[np.ix_(rows, cols)], ref[np.ix_(rows, cols)]) <= TOL

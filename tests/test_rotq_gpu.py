@@ -205,3 +205,26 @@ def test_widest_rows_rpbh(oq, codebooks):
     # d = 16384, the widest row the kernels take (one row pair per stage)
     X = inputs.sweep_activations(130, 16384)
     _check_rows(oq, codebooks, X, 16384, 256, 4)
+
+
+@pytest.mark.parametrize("d,h,bits", [(3072, 128, 4), (1536, 64, 2), (12288, 256, 6), (3072, 128, 6)])
+def test_empirical_distortion_matches_lloyd_max(oq, codebooks, d, h, bits):
+    # [OQ] "Theoretical Basis": after RPBH each coordinate of a unit row follows
+    # f_d, so the per-row squared error of the kernel's codes on N(0,1) rows is
+    # d * D(d, b), the Lloyd-Max distortion (a property that holds at any M).
+    # The rotated rows come from the oracle; the codes from the kernel.
+    M = 2048
+    X = inputs.sweep_activations(M, d, seed_offset=1)[: M - M // 8]  # the N(0,1) rows only
+    r, cb = _lib_handles(oq, 0, d, h, bits)
+    codes, _ = oq.quantize_act(r, cb, _to_dev(X))
+    torch.cuda.synchronize()
+    got = oqz.unpack_codes(codes.cpu().numpy(), bits, d)
+    perm, signs = orpbh.draw_permutation_and_signs(0, d)
+    U = orpbh.rotate(inputs.bf16_bits_to_f64(X), perm, signs, h)
+    T = U / np.linalg.norm(U, axis=1, keepdims=True)
+    book = codebooks(d, bits)
+    err = np.sum((T - book["centroids"][got]) ** 2, axis=1).mean()
+    theory = d * book["distortion"]
+    # N(0,1) rows: the error of a row is a mean over d coordinates; 1792 rows
+    # bring the sampling spread well below 1%
+    assert abs(err / theory - 1.0) < 0.01, (err, theory)
