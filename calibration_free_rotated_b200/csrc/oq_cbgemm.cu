@@ -18,7 +18,7 @@
 //                128-byte-swizzled UMMA layout in shared memory.
 //                (Both use register byte-permute tables for 2 and 4 bits and a
 //                128-byte shared table for 6 bits.)
-//   warp 21      one thread of the leader CTA issues tcgen05.mma (kind::f16,
+//   warp 21      one elected lane of the leader CTA's warp issues tcgen05.mma (kind::f16,
 //                A from TMEM, B from shared memory, M = 256 across the pair,
 //                N = 256, K = 16, fp32 accumulate in TMEM); tcgen05.commit
 //                (multicast to both CTAs) frees ring stages and publishes the
@@ -277,6 +277,17 @@ __device__ __forceinline__ void umma_commit(uint32_t bar) {
   } else {
     asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar) : "memory");
   }
+}
+
+// True in exactly one lane of the (fully converged) warp.
+__device__ __forceinline__ bool elect_one() {
+  uint32_t p;
+  asm volatile(
+      "{\n\t.reg .pred e;\n\t.reg .b32 r;\n\t"
+      "elect.sync r|e, 0xffffffff;\n\t"
+      "selp.u32 %0, 1, 0, e;\n\t}"
+      : "=r"(p));
+  return p != 0;
 }
 
 __device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
@@ -711,36 +722,45 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       }
     }
   } else if (warp == MMA_WARP) {
-    if (lane == 0 && rank == 0) {
+    // The whole warp runs the loop, converged, so the stage addresses and
+    // descriptors stay warp-uniform; one elected lane issues the MMAs and
+    // commits.  (Issuing from a lone active lane cost about 1.4x more cycles
+    // per k-step.)  The B descriptor of stage es, k-slice k is the stage-0
+    // descriptor plus the byte offset / 16.
+    if (rank == 0) {
       uint32_t ec = 0, lt = 0;
       bool ok = true;
+      const uint64_t bdesc0 = umma_desc_sw128(sbase + S::kExpB);
+      const uint32_t a_tmem0 = tmem_base + (uint32_t)A_COL0;
       for (int t = unit; t < num_tiles && ok; t += nunits, ++lt) {
         const uint32_t aph = lt & 1u;
-        const bool got = PAIR ? wait_bounded_cluster(bar(ACC_EMPTY), aph ^ 1u, abort_flag, args.status)
-                              : wait_bounded(bar(ACC_EMPTY), aph ^ 1u, abort_flag, args.status);
-        if (!got) break;
+        bool got = PAIR ? wait_bounded_cluster(bar(ACC_EMPTY), aph ^ 1u, abort_flag, args.status)
+                        : wait_bounded(bar(ACC_EMPTY), aph ^ 1u, abort_flag, args.status);
+        if (!__all_sync(0xFFFFFFFFu, got)) break;
         tc_fence_after();
         for (int kb = 0; kb < KB; ++kb, ++ec) {
-          const int es = ec % ESTAGES;
+          const uint32_t es = ec % ESTAGES;
           const uint32_t eph = (ec / ESTAGES) & 1u;
           const bool full = PAIR ? wait_bounded_cluster(bar(EX_FULL + es), eph, abort_flag, args.status)
                                  : wait_bounded(bar(EX_FULL + es), eph, abort_flag, args.status);
-          if (!full) {
+          if (!__all_sync(0xFFFFFFFFu, full)) {
             ok = false;
             break;
           }
           tc_fence_after();
-          const uint32_t a_tmem = tmem_base + (uint32_t)(A_COL0 + 32 * es);
-          const uint32_t b_addr = sbase + S::kExpB + es * S::kExpBBytes;
+          const uint32_t a_tmem = a_tmem0 + 32u * es;
+          const uint64_t bdesc = bdesc0 + (uint64_t)((es * (uint32_t)S::kExpBBytes) >> 4);
+          if (elect_one()) {
 #pragma unroll
-          for (int k = 0; k < BK / 16; ++k) {
-            umma_f16_ts<PAIR>(tmem_base, a_tmem + 8u * k, umma_desc_sw128(b_addr + 32 * k),
-                              (kb > 0 || k > 0) ? 1u : 0u);
+            for (int k = 0; k < BK / 16; ++k)
+              umma_f16_ts<PAIR>(tmem_base, a_tmem + 8u * k, bdesc + 2u * k, (kb > 0 || k > 0) ? 1u : 0u);
+            umma_commit<PAIR>(bar(EX_EMPTY + es));
           }
-          umma_commit<PAIR>(bar(EX_EMPTY + es));
+          __syncwarp();
         }
         if (!ok) break;
-        umma_commit<PAIR>(bar(ACC_FULL));
+        if (elect_one()) umma_commit<PAIR>(bar(ACC_FULL));
+        __syncwarp();
       }
     }
   } else if (warp >= EPI_WARP0 && warp < EPI_WARP0 + 4) {
