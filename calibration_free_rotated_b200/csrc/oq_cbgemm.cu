@@ -56,6 +56,8 @@ constexpr int MMA_WARP = 21;
 constexpr int NUM_THREADS = 22 * 32;
 constexpr int TMEM_COLS = 512;
 constexpr int A_COL0 = BN;                   // A stage s: TMEM columns A_COL0 + 32 s .. + 31
+constexpr int SPARE_COL = A_COL0 + 32 * ESTAGES;  // the last 128 columns: epilogue spill area
+static_assert(SPARE_COL + BN / 2 == TMEM_COLS, "TMEM plan");
 constexpr unsigned long long kWaitLimitNs = 1000000000ull;
 
 struct GemmArgs {
@@ -305,6 +307,12 @@ __device__ __forceinline__ uint32_t lds_u16(uint32_t addr) {
   return v;
 }
 
+__device__ __forceinline__ uint4 lds_v4(uint32_t addr) {
+  uint4 v;
+  asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr));
+  return v;
+}
+
 __device__ __forceinline__ void sts_v4(uint32_t addr, uint4 v) {
   asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
                : "memory");
@@ -519,6 +527,29 @@ __device__ __forceinline__ uint32_t bf16x2_rn(float lo, float hi) {
   uint32_t r;
   asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
   return r;
+}
+
+// Epilogue arithmetic of 8 consecutive columns c .. c+7 of one row:
+// y = acc * (s_m / d) * r'_n + bias_n, optional GELU, rounded to bf16.
+__device__ __forceinline__ uint4 epi8_bf16(const uint32_t* v, const float* col_r, const float* col_b, int c,
+                                           unsigned long long as2, bool gelu) {
+  const ulonglong2 r01 = *reinterpret_cast<const ulonglong2*>(col_r + c);
+  const ulonglong2 r23 = *reinterpret_cast<const ulonglong2*>(col_r + c + 4);
+  const ulonglong2 b01 = *reinterpret_cast<const ulonglong2*>(col_b + c);
+  const ulonglong2 b23 = *reinterpret_cast<const ulonglong2*>(col_b + c + 4);
+  const unsigned long long rr[4] = {r01.x, r01.y, r23.x, r23.y};
+  const unsigned long long bb[4] = {b01.x, b01.y, b23.x, b23.y};
+  uint32_t o[4];
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    unsigned long long y2 = f2_fma(f2_mul(f2_pack(__uint_as_float(v[2 * j]), __uint_as_float(v[2 * j + 1])), as2),
+                                   rr[j], bb[j]);
+    if (gelu) y2 = gelu2(y2);
+    float y0, y1;
+    f2_unpack(y2, y0, y1);
+    o[j] = bf16x2_rn(y0, y1);
+  }
+  return make_uint4(o[0], o[1], o[2], o[3]);
 }
 
 // Named barrier 1 over the four epilogue warps.
@@ -770,6 +801,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     // next tile's MMAs overlap the conversion and the stores. The four warps
     // take every decision together (named barrier 1), so none can wait on a
     // barrier that another has left.
+    //
+    // bf16-only output with the four-block staging (the usual case): the
+    // accumulator is first evacuated without arithmetic -- columns 128..255 to
+    // the spare TMEM columns, columns 0..127 as raw fp32 into the staging
+    // buffer (exactly its 64 KB) -- and released; the arithmetic then runs
+    // from those copies while the next tile's MMAs proceed.  The first half is
+    // converted in place (each thread rewrites only its own row, and a raw
+    // chunk is always read before a bf16 chunk lands on it).
     const int quad = warp & 3;  // TMEM lanes 32*quad .. 32*quad+31
     const int rl = quad * 32 + lane;  // row within the CTA's 128
     const bool leader = (warp == EPI_WARP0 && lane == 0);
@@ -794,6 +833,103 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       const bool got = wait_bounded(bar(ACC_FULL), lt & 1u, abort_flag, args.status);
       if (epi_any(!got)) break;
       tc_fence_after();
+      if (S::kStageBlocks == 4 && args.y16 != nullptr && args.y32 == nullptr) {
+        constexpr int H = BN / 2;
+        const uint32_t spare = taddr + (uint32_t)SPARE_COL;
+        const uint32_t rsw = (uint32_t)(rl & 7);  // the row's 128-byte swizzle
+        if (leader) bulk_wait_read();  // the previous tile's stores have read the staging buffer
+        epi_bar();
+#pragma unroll 1
+        for (int c = 0; c < H; c += 32) {  // columns H.. -> spare TMEM columns
+          uint32_t v[32];
+          __syncwarp();
+          tmem_ld16(taddr + (uint32_t)(H + c), v);
+          tmem_ld16(taddr + (uint32_t)(H + c + 16), v + 16);
+          asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+          tmem_st16(spare + (uint32_t)c, v);
+          tmem_st16(spare + (uint32_t)(c + 16), v + 16);
+        }
+#pragma unroll 1
+        for (int c = 0; c < H; c += 32) {  // columns 0.. -> staging block c / 32, raw fp32
+          uint32_t v[32];
+          __syncwarp();
+          tmem_ld16(taddr + (uint32_t)c, v);
+          tmem_ld16(taddr + (uint32_t)(c + 16), v + 16);
+          asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+          const uint32_t rowb = stage + (uint32_t)(c / 32) * 16384u + (uint32_t)rl * 128u;
+#pragma unroll
+          for (int j = 0; j < 8; ++j)
+            sts_v4(rowb + (((uint32_t)j ^ rsw) << 4), make_uint4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]));
+        }
+        asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) {
+          if constexpr (PAIR) mbar_arrive_cluster(bar(ACC_EMPTY), 0);  // the leader's barrier
+          else mbar_arrive(bar(ACC_EMPTY));
+        }
+        const unsigned long long as2 = f2_pack(a_scale, a_scale);
+        const bool gelu = args.epilogue == OQ_EPI_GELU;
+        // columns 0..127: raw fp32 (blocks 0..3) -> bf16 (blocks 0, 1)
+#pragma unroll 1
+        for (int c0 = 0; c0 < H; c0 += 16) {
+          const uint32_t src = stage + (uint32_t)(c0 / 32) * 16384u + (uint32_t)rl * 128u;
+          const uint32_t jr = (uint32_t)(c0 % 32) / 4;
+          uint32_t v[16];
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const uint4 w = lds_v4(src + (((jr + i) ^ rsw) << 4));
+            v[4 * i] = w.x; v[4 * i + 1] = w.y; v[4 * i + 2] = w.z; v[4 * i + 3] = w.w;
+          }
+          const uint32_t dst = stage + (uint32_t)(c0 / 64) * 16384u + (uint32_t)rl * 128u;
+          const uint32_t jb = (uint32_t)(c0 % 64) / 8;
+          sts_v4(dst + ((jb ^ rsw) << 4), epi8_bf16(v, col_r, col_b, c0, as2, gelu));
+          sts_v4(dst + (((jb + 1) ^ rsw) << 4), epi8_bf16(v + 8, col_r, col_b, c0 + 8, as2, gelu));
+        }
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        epi_bar();
+        if (leader) {
+          for (int b = 0; b < 2; ++b)
+            if (n0 + 64 * b < args.N && m0 < args.M) tma_store_2d(&map_y16, stage + (uint32_t)b * 16384u, n0 + 64 * b, m0);
+          bulk_commit();
+        }
+        // columns 128..255: spare TMEM -> bf16 (blocks 2, 3); the next load is in flight during the arithmetic
+        {
+          uint32_t va[16], vb[16];
+          __syncwarp();
+          tmem_ld16(spare, va);
+          asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll 1
+          for (int c0 = 0; c0 < H; c0 += 32) {
+            __syncwarp();
+            tmem_ld16(spare + (uint32_t)(c0 + 16), vb);
+            {
+              const uint32_t dst = stage + (uint32_t)(2 + c0 / 64) * 16384u + (uint32_t)rl * 128u;
+              const uint32_t jb = (uint32_t)(c0 % 64) / 8;
+              sts_v4(dst + ((jb ^ rsw) << 4), epi8_bf16(va, col_r, col_b, H + c0, as2, gelu));
+              sts_v4(dst + (((jb + 1) ^ rsw) << 4), epi8_bf16(va + 8, col_r, col_b, H + c0 + 8, as2, gelu));
+            }
+            asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+            __syncwarp();
+            if (c0 + 32 < H) tmem_ld16(spare + (uint32_t)(c0 + 32), va);
+            {
+              const uint32_t dst = stage + (uint32_t)(2 + (c0 + 16) / 64) * 16384u + (uint32_t)rl * 128u;
+              const uint32_t jb = (uint32_t)((c0 + 16) % 64) / 8;
+              sts_v4(dst + ((jb ^ rsw) << 4), epi8_bf16(vb, col_r, col_b, H + c0 + 16, as2, gelu));
+              sts_v4(dst + (((jb + 1) ^ rsw) << 4), epi8_bf16(vb + 8, col_r, col_b, H + c0 + 24, as2, gelu));
+            }
+            asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+          }
+        }
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        epi_bar();
+        if (leader) {
+          for (int b = 2; b < 4; ++b)
+            if (n0 + 64 * b < args.N && m0 < args.M) tma_store_2d(&map_y16, stage + (uint32_t)b * 16384u, n0 + 64 * b, m0);
+          bulk_commit();
+        }
+        continue;
+      }
 #pragma unroll 1
       for (int kind = 0; kind < 2; ++kind) {  // 0: bf16 output, 1: fp32 output
         const bool want = kind == 0 ? args.y16 != nullptr : args.y32 != nullptr;

@@ -295,3 +295,33 @@ def test_full_layer_with_rotation_variants(oq, codebooks, kind, h):
     assert rows.sum() > M // 2 and cols.sum() > N // 2
     ref = olin.linear_from_codes(ca, s, cw, r16, c, c, d)
     assert _rel_fro(y.double().cpu().numpy()[np.ix_(rows, cols)], ref[np.ix_(rows, cols)]) <= TOL
+
+
+@pytest.mark.parametrize("ba,bw,epilogue,M,N", [(4, 4, "none", 2048, 2560), (4, 2, "gelu", 1000, 2320),
+                                                 (6, 4, "gelu", 777, 1216), (2, 2, "none", 300, 272)])
+def test_bf16_only_output(oq, codebooks, ba, bw, epilogue, M, N):
+    # bf16-only output (the layer's usual call) takes the epilogue that first
+    # evacuates the accumulator (spare TMEM columns + raw staging) and converts
+    # afterwards; its result must be the fp32 path's output rounded to bf16,
+    # bit for bit, over several tiles per CTA pair and ragged M / N tails.
+    d, h = 512, 128
+    rng = np.random.default_rng(ba * 100 + bw * 10 + M % 7)
+    X = inputs.to_bf16_bits(rng.standard_normal((M, d)))
+    W = inputs.to_bf16_bits(rng.standard_normal((N, d)) * 0.02)
+    bias = inputs.to_bf16_bits(rng.standard_normal(N) * 0.1)
+    ca, s = _oracle_act(codebooks, X, d, h, ba)
+    cw, r16 = _oracle_weight(codebooks, W, d, h, bw)
+    cb_a, cb_w = _lib_cb(oq, d, ba), _lib_cb(oq, d, bw)
+    args = (d, cb_a, cb_w, _dev_u8(oqz.pack_codes(ca, ba)), torch.from_numpy(s.astype(np.float32)).cuda(),
+            _dev_u8(oqz.pack_codes(cw, bw)), _dev_bf16(oqz.bf16_bits(r16)))
+    y32, _ = oq.linear_codes(*args, bias=_dev_bf16(bias), epilogue=epilogue)
+    _, y16 = oq.linear_codes(*args, bias=_dev_bf16(bias), epilogue=epilogue, want_f32=False, want_bf16=True)
+    torch.cuda.synchronize()
+    oq.device_status()
+    assert torch.equal(y16, y32.to(torch.bfloat16))
+    rows = np.linspace(0, M - 1, 24).astype(int)
+    ref = olin.linear_from_codes(ca[rows], s[rows], cw, r16, codebooks(d, ba)["centroids"],
+                                 codebooks(d, bw)["centroids"], d, bias=inputs.bf16_bits_to_f64(bias),
+                                 gelu=(epilogue == "gelu"))
+    # bf16 output: the rounding adds up to 2^-9 relative per element
+    assert _rel_fro(y16.double().cpu().numpy()[rows], ref) <= TOL + 2.0 ** -9
