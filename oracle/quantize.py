@@ -27,7 +27,7 @@ Readings of what the pages leave open:
 
 import numpy as np
 
-from .rpbh import rotate
+from .rpbh import rotate, rotate_composed
 
 EPS = 1e-12
 
@@ -51,11 +51,19 @@ def quantize_rows(X, perm, signs, h, centroids, eps: float = EPS):
     ``t`` is the normalised rotated row (x~'), returned so that tests can find
     entries that lie near a decision boundary.
     """
-    U = rotate(X, perm, signs, h)
+    return _quantize_rotated(rotate(X, perm, signs, h), centroids, eps)
+
+
+def _quantize_rotated(U, centroids, eps):
     s = np.sqrt(np.sum(U * U, axis=-1))
     T = U / (s[..., None] + eps)
     codes = nearest_centroid(T, centroids)
     return codes, s, T
+
+
+def quantize_rows_composed(X, rounds, h, centroids, eps: float = EPS):
+    """quantize_rows with the composed rotation Pi_k ... Pi_1 (rpbh.rotate_composed)."""
+    return _quantize_rotated(rotate_composed(X, rounds, h), centroids, eps)
 
 
 def bf16_round(v) -> np.ndarray:
@@ -81,11 +89,19 @@ def bf16_bits(v) -> np.ndarray:
 
 def quantize_weight_rows(W, perm, signs, h, centroids, eps: float = EPS):
     """Weight rows -> (codes, r_bf16 as float64, r fp64 unrounded, t)."""
-    U = rotate(W, perm, signs, h)
+    return _quantize_weight_rotated(rotate(W, perm, signs, h), centroids, eps)
+
+
+def _quantize_weight_rotated(U, centroids, eps):
     r = np.sqrt(np.sum(U * U, axis=-1))
     T = U / (r[..., None] + eps)
     codes = nearest_centroid(T, centroids)
     return codes, bf16_round(r), r, T
+
+
+def quantize_weight_rows_composed(W, rounds, h, centroids, eps: float = EPS):
+    """quantize_weight_rows with the composed rotation (rpbh.rotate_composed)."""
+    return _quantize_weight_rotated(rotate_composed(W, rounds, h), centroids, eps)
 
 
 def pack_codes(codes: np.ndarray, bits: int) -> np.ndarray:

@@ -21,6 +21,16 @@ Readings of what the page leaves open:
   j = next() mod (i+1), swap pi[i], pi[j]), then d sign draws
   sign_j = -1 if the top bit of next() is set else +1.
 
+Composed rounds ([RHT] Methodology; "Key contributions" 1 and 3): the
+composition R_k of k randomized Hadamard transforms, each a Hadamard matrix
+times its own Rademacher diagonal.  Two rounds make every single coordinate
+close to Gaussian for any input, three also decorrelate the coordinates.
+Reading for a block rotation: each round is a full RPBH round with its own
+permutation and signs, Pi^(k) = Pi_k ... Pi_1 (the permutation is what lets a
+later round mix coordinates that an earlier round kept inside one block).
+Round 1 is the plain RPBH draw of the seed; round r + 1 continues the same
+SplitMix64 stream after round r's draws (Fisher-Yates pass, then d signs).
+
 Everything here is dense and slow on purpose: no butterflies, no fusion.
 """
 
@@ -36,18 +46,30 @@ def default_block(d: int) -> int:
     return d & (-d)
 
 
-def draw_permutation_and_signs(seed: int, d: int):
-    """Fisher-Yates permutation then d Rademacher signs from one SplitMix64 stream.
-
-    Returns (perm int64[d], signs float64[d] in {-1, +1}).
-    """
-    g = SplitMix64(seed)
+def _draw_round(g: SplitMix64, d: int):
     perm = list(range(d))
     for i in range(d - 1, 0, -1):
         j = g.next() % (i + 1)
         perm[i], perm[j] = perm[j], perm[i]
     signs = [(-1.0 if (g.next() >> 63) else 1.0) for _ in range(d)]
     return np.array(perm, dtype=np.int64), np.array(signs, dtype=np.float64)
+
+
+def draw_permutation_and_signs(seed: int, d: int):
+    """Fisher-Yates permutation then d Rademacher signs from one SplitMix64 stream.
+
+    Returns (perm int64[d], signs float64[d] in {-1, +1}).
+    """
+    return _draw_round(SplitMix64(seed), d)
+
+
+def draw_rounds(seed: int, d: int, rounds: int):
+    """[(perm, signs)] of rounds 1..k of the composed rotation, all from one
+    SplitMix64(seed) stream in order (round 1 = draw_permutation_and_signs)."""
+    if rounds < 1:
+        raise ValueError("rounds must be >= 1")
+    g = SplitMix64(seed)
+    return [_draw_round(g, d) for _ in range(rounds)]
 
 
 def hadamard(h: int) -> np.ndarray:
@@ -100,3 +122,20 @@ def rotate(X: np.ndarray, perm: np.ndarray, signs: np.ndarray, h: int) -> np.nda
         sl = slice(i * h, (i + 1) * h)
         out[..., sl] = Z[..., sl] @ H.T   # H_h z_i for each row
     return out
+
+
+def composed_matrix(rounds, h: int) -> np.ndarray:
+    """Dense Pi^(k) = Pi_k ... Pi_1 for rounds [(perm_1, signs_1), ...] (small d only)."""
+    d = len(rounds[0][0])
+    M = np.eye(d)
+    for perm, signs in rounds:
+        M = rpbh_matrix(perm, signs, h) @ M
+    return M
+
+
+def rotate_composed(X: np.ndarray, rounds, h: int) -> np.ndarray:
+    """x' = Pi_k ( ... (Pi_1 x)) for every row of X: round 1 first."""
+    U = np.asarray(X, dtype=np.float64)
+    for perm, signs in rounds:
+        U = rotate(U, perm, signs, h)
+    return U

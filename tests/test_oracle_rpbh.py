@@ -154,3 +154,79 @@ def test_full_block_identity_permutation_is_textbook_wht():
         e = np.zeros(d)
         e[k] = 1.0
         assert np.allclose(rpbh.rotate(e[None], perm, signs, d)[0], S[:, k] / 8.0, atol=1e-15)
+
+
+# ---- composed rounds ([RHT] Methodology, Key contributions 1 and 3) ----------
+
+def test_composed_round_one_is_the_rpbh_draw_and_later_rounds_differ():
+    d = 512
+    rounds = rpbh.draw_rounds(7, d, 3)
+    p, s = rpbh.draw_permutation_and_signs(7, d)
+    assert np.array_equal(rounds[0][0], p) and np.array_equal(rounds[0][1], s)
+    for perm, signs in rounds[1:]:
+        assert sorted(perm.tolist()) == list(range(d))
+        assert set(np.unique(signs).tolist()) <= {-1.0, 1.0}
+    assert not np.array_equal(rounds[1][0], rounds[0][0])
+    assert not np.array_equal(rounds[2][0], rounds[1][0])
+    # the stream continues: round 2 of a 2-round draw is round 2 of a 3-round draw
+    two = rpbh.draw_rounds(7, d, 2)
+    assert np.array_equal(two[1][0], rounds[1][0]) and np.array_equal(two[1][1], rounds[1][1])
+
+
+@pytest.mark.parametrize("d,h,k", [(64, 8, 2), (128, 32, 3), (256, 64, 2)])
+def test_composed_rotation_is_orthogonal_and_matches_the_dense_product(d, h, k):
+    rounds = rpbh.draw_rounds(3, d, k)
+    M = rpbh.composed_matrix(rounds, h)
+    assert np.allclose(M @ M.T, np.eye(d), atol=1e-12)
+    x = np.random.default_rng(1).standard_normal((5, d))
+    assert np.allclose(rpbh.rotate_composed(x, rounds, h), x @ M.T, atol=1e-12)
+    assert np.allclose(np.linalg.norm(rpbh.rotate_composed(x, rounds, h), axis=1), np.linalg.norm(x, axis=1))
+
+
+def test_two_rounds_of_a_one_hot_row_lie_on_the_1_over_h_lattice():
+    # Closed form: round 1 turns e_i into h entries of +-1/sqrt(h) (one block);
+    # round 2 scatters them, and block b, receiving n_b of them, becomes
+    # H_h times n_b entries of +-1/sqrt(h): every entry is k/h with |k| <= n_b
+    # and k = n_b (mod 2), and the n_b add up to h.
+    d, h = 1024, 32
+    rounds = rpbh.draw_rounds(11, d, 2)
+    x = np.zeros(d)
+    x[123] = 1.0
+    u1 = rpbh.rotate(x, *rounds[0], h)
+    assert np.count_nonzero(np.abs(u1) > 1e-12) == h
+    assert np.allclose(np.abs(u1[np.abs(u1) > 1e-12]), 1.0 / np.sqrt(h))
+    moved = u1[rounds[1][0]]                     # round 2's gather
+    n_b = (np.abs(moved) > 1e-12).reshape(d // h, h).sum(axis=1)
+    assert n_b.sum() == h
+    u2 = rpbh.rotate_composed(x, rounds, h)
+    k = np.rint(u2 * h).reshape(d // h, h)
+    assert np.allclose(u2.reshape(d // h, h) * h, k, atol=1e-9)
+    assert np.all(np.abs(k) <= n_b[:, None])
+    assert np.all((k - n_b[:, None]) % 2 == 0)
+
+
+def test_two_and_three_rounds_bring_sparse_rows_to_the_lloyd_max_distortion(codebooks):
+    # [RHT] Key contribution 1: after two rounds every coordinate of any input
+    # is close to Gaussian, so the Lloyd-Max codebook's distortion d * D(d, b)
+    # holds for one-hot and k-sparse rows too; a single block round leaves a
+    # one-hot row inside one block and its error many times larger.
+    from oracle import quantize as oqz
+    d, h, b = 3072, 128, 4
+    book = codebooks(d, b)
+    c, theory = book["centroids"], d * book["distortion"]
+    rng = np.random.default_rng(5)
+    M = 48
+    onehot = np.zeros((M, d))
+    onehot[np.arange(M), rng.integers(0, d, M)] = rng.choice([-1.0, 1.0], M)
+    sparse = np.zeros((M, d))
+    for i in range(M):
+        sparse[i, rng.choice(d, 8, replace=False)] = rng.standard_normal(8)
+
+    def ratio(X, k):
+        codes, _, T = oqz.quantize_rows_composed(X, rpbh.draw_rounds(0, d, k), h, c)
+        return np.sum((T - c[codes]) ** 2, axis=1).mean() / theory
+
+    assert ratio(onehot, 1) > 10.0 and ratio(sparse, 1) > 2.5
+    for k in (2, 3):
+        assert 0.6 < ratio(onehot, k) < 1.3
+        assert 0.8 < ratio(sparse, k) < 1.25
