@@ -360,6 +360,47 @@ int codebook_device_qtable(oq_codebook_t cb, const uint32_t** qtable) {
   return OQ_OK;
 }
 
+// Shared-memory slot of coordinate c in the composed kernel's array of f32
+// pairs: thread c / 32 owns a run of 32 slots whose 2-slot chunks are rotated
+// by the thread index (chunk (c / 2) % 16 at position chunk ^ (thread % 16)).
+static uint16_t composed_slot(uint32_t c) {
+  const uint32_t g = c >> 5, ch = (c >> 1) & 15u;
+  return (uint16_t)((g << 5) | ((ch ^ (g & 15u)) << 1) | (c & 1u));
+}
+
+int rpbh_composed_tables(oq_rpbh_t r, const uint16_t** slots, const uint32_t** signs) {
+  int dev;
+  if (int rc = current_device(&dev)) return rc;
+  std::lock_guard<std::mutex> lk(r->mu);
+  if (!r->dev_slots[dev]) {
+    const int d = r->d, words = (d + 31) / 32;
+    std::vector<uint16_t> sl((size_t)r->rounds * d);
+    std::vector<uint32_t> sg((size_t)r->rounds * words);
+    for (int k = 0; k < r->rounds; ++k) {
+      const int32_t* perm = k == 0 ? r->perm.data() : r->perm_more.data() + (size_t)(k - 1) * d;
+      const uint32_t* bits = k == 0 ? r->sign_bits.data() : r->sign_bits_more.data() + (size_t)(k - 1) * words;
+      for (int j = 0; j < d; ++j) sl[(size_t)k * d + j] = composed_slot((uint32_t)perm[j]);
+      std::memcpy(sg.data() + (size_t)k * words, bits, sizeof(uint32_t) * words);
+    }
+    uint16_t* dsl = nullptr;
+    uint32_t* dsg = nullptr;
+    cudaError_t e = cudaMalloc(&dsl, sizeof(uint16_t) * sl.size());
+    if (e == cudaSuccess) e = cudaMalloc(&dsg, sizeof(uint32_t) * sg.size());
+    if (e == cudaSuccess) e = cudaMemcpy(dsl, sl.data(), sizeof(uint16_t) * sl.size(), cudaMemcpyHostToDevice);
+    if (e == cudaSuccess) e = cudaMemcpy(dsg, sg.data(), sizeof(uint32_t) * sg.size(), cudaMemcpyHostToDevice);
+    if (e != cudaSuccess) {
+      cudaFree(dsl);
+      cudaFree(dsg);
+      return fail(OQ_ERR_CUDA, "uploading composed rotation tables: %s", cudaGetErrorString(e));
+    }
+    r->dev_slots[dev] = dsl;
+    r->dev_csigns[dev] = dsg;
+  }
+  *slots = r->dev_slots[dev];
+  *signs = r->dev_csigns[dev];
+  return OQ_OK;
+}
+
 int rpbh_device_tables(oq_rpbh_t r, const uint16_t** perm, const uint32_t** signs) {
   int dev;
   if (int rc = current_device(&dev)) return rc;
@@ -369,6 +410,79 @@ int rpbh_device_tables(oq_rpbh_t r, const uint16_t** perm, const uint32_t** sign
   }
   *perm = r->dev_perm[dev];
   *signs = r->dev_signs[dev];
+  return OQ_OK;
+}
+
+// One round of draws from the SplitMix64 stream `st`: the Fisher-Yates
+// permutation of 0..d-1 (for i = d-1 .. 1: j = next() mod (i+1), swap), then
+// d Rademacher signs (sign_j = -1 when the top bit of next() is set).
+static void draw_round(uint64_t& st, int d, int32_t* perm, uint32_t* sign_bits) {
+  for (int j = 0; j < d; ++j) perm[j] = j;
+  for (int i = d - 1; i >= 1; --i) {
+    const uint64_t j = splitmix64_next(st) % (uint64_t)(i + 1);
+    const int32_t tmp = perm[i];
+    perm[i] = perm[j];
+    perm[j] = tmp;
+  }
+  for (int w = 0; w < (d + 31) / 32; ++w) sign_bits[w] = 0u;
+  for (int j = 0; j < d; ++j)
+    if (splitmix64_next(st) >> 63) sign_bits[j >> 5] |= 1u << (j & 31);
+}
+
+// Rotation handle of `rounds` rounds drawn in order from SplitMix64(seed).
+static int make_rotation(uint64_t seed, int d, int block, int kind, int rounds, oq_rpbh_t* out) {
+  if (!out) return fail(OQ_ERR_ARG, "out is NULL");
+  *out = nullptr;
+  if (d < 1) return fail(OQ_ERR_ARG, "d must be >= 1 (got %d)", d);
+  if (kind != OQ_ROT_RPBH && kind != OQ_ROT_BLOCK_RHT && kind != OQ_ROT_FULL_RHT)
+    return fail(OQ_ERR_ARG, "unknown rotation kind %d", kind);
+  if (kind == OQ_ROT_FULL_RHT && block != 0 && block != (d & -d))
+    return fail(OQ_ERR_ARG, "a full RHT of d=%d has block %d (got %d)", d, d & -d, block);
+  int h = block == 0 ? (d & -d) : block;
+  if (h < 1 || (h & (h - 1)) != 0 || d % h != 0)
+    return fail(OQ_ERR_ARG, "block %d must be a power of two dividing d=%d", block, d);
+  if (rounds > 1 && d > 65536) return fail(OQ_ERR_ARG, "composed rotations need d <= 65536 (got %d)", d);
+  oq_rpbh_t r = new (std::nothrow) oq_rpbh_s;
+  if (!r) return fail(OQ_ERR_NOMEM, "allocating the RPBH handle");
+  r->seed = seed;
+  r->d = d;
+  r->h = h;
+  r->kind = kind;
+  r->rounds = rounds;
+  const size_t words = (size_t)(d + 31) / 32;
+  r->perm.resize(d);
+  r->sign_bits.resize(words);
+  r->perm_more.resize((size_t)(rounds - 1) * d);
+  r->sign_bits_more.resize((size_t)(rounds - 1) * words);
+  uint64_t st = seed;
+  draw_round(st, d, r->perm.data(), r->sign_bits.data());
+  // Block-RHT and Full RHT: the same draws (so the same signs), identity permutation
+  if (kind != OQ_ROT_RPBH)
+    for (int j = 0; j < d; ++j) r->perm[j] = j;
+  for (int k = 1; k < rounds; ++k)  // later rounds continue the same stream
+    draw_round(st, d, r->perm_more.data() + (size_t)(k - 1) * d, r->sign_bits_more.data() + (size_t)(k - 1) * words);
+  // Upload to the current device now when one is present; otherwise lazily.
+  int ndev = 0;
+  if (cudaGetDeviceCount(&ndev) == cudaSuccess && ndev > 0 && d <= 65536) {
+    int dev;
+    if (cudaGetDevice(&dev) == cudaSuccess && dev < OQ_MAX_DEVICES) {
+      if (int rc = upload_rpbh(r, dev)) {
+        delete r;
+        return rc;
+      }
+      if (rounds > 1) {
+        const uint16_t* sl;
+        const uint32_t* sg;
+        if (int rc = rpbh_composed_tables(r, &sl, &sg)) {
+          oq_free_rpbh(r);
+          return rc;
+        }
+      }
+    }
+  } else {
+    cudaGetLastError();  // no device here: clear the sticky "no device" error
+  }
+  *out = r;
   return OQ_OK;
 }
 
@@ -401,56 +515,39 @@ int oq_get_device_status(void* stream) {
 
 int oq_make_rotation(uint64_t seed, int d, int block, int kind, oq_rpbh_t* out) {
   clear_error();
-  if (!out) return fail(OQ_ERR_ARG, "out is NULL");
-  *out = nullptr;
-  if (d < 1) return fail(OQ_ERR_ARG, "d must be >= 1 (got %d)", d);
-  if (kind != OQ_ROT_RPBH && kind != OQ_ROT_BLOCK_RHT && kind != OQ_ROT_FULL_RHT)
-    return fail(OQ_ERR_ARG, "unknown rotation kind %d", kind);
-  if (kind == OQ_ROT_FULL_RHT && block != 0 && block != (d & -d))
-    return fail(OQ_ERR_ARG, "a full RHT of d=%d has block %d (got %d)", d, d & -d, block);
-  int h = block == 0 ? (d & -d) : block;
-  if (h < 1 || (h & (h - 1)) != 0 || d % h != 0)
-    return fail(OQ_ERR_ARG, "block %d must be a power of two dividing d=%d", block, d);
-  oq_rpbh_t r = new (std::nothrow) oq_rpbh_s;
-  if (!r) return fail(OQ_ERR_NOMEM, "allocating the RPBH handle");
-  r->seed = seed;
-  r->d = d;
-  r->h = h;
-  r->kind = kind;
-  r->perm.resize(d);
-  for (int j = 0; j < d; ++j) r->perm[j] = j;
-  uint64_t st = seed;
-  for (int i = d - 1; i >= 1; --i) {  // Fisher-Yates
-    uint64_t j = splitmix64_next(st) % (uint64_t)(i + 1);
-    int32_t tmp = r->perm[i];
-    r->perm[i] = r->perm[j];
-    r->perm[j] = tmp;
-  }
-  // Block-RHT and Full RHT: the same draws (so the same signs), identity permutation
-  if (kind != OQ_ROT_RPBH)
-    for (int j = 0; j < d; ++j) r->perm[j] = j;
-  r->sign_bits.assign((d + 31) / 32, 0u);
-  for (int j = 0; j < d; ++j)
-    if (splitmix64_next(st) >> 63) r->sign_bits[j >> 5] |= 1u << (j & 31);
-  // Upload to the current device now when one is present; otherwise lazily.
-  int ndev = 0;
-  if (cudaGetDeviceCount(&ndev) == cudaSuccess && ndev > 0 && d <= 65536) {
-    int dev;
-    if (cudaGetDevice(&dev) == cudaSuccess && dev < OQ_MAX_DEVICES) {
-      if (int rc = upload_rpbh(r, dev)) {
-        delete r;
-        return rc;
-      }
-    }
-  } else {
-    cudaGetLastError();  // no device here: clear the sticky "no device" error
-  }
-  *out = r;
-  return OQ_OK;
+  return make_rotation(seed, d, block, kind, 1, out);
 }
 
 int oq_make_rpbh(uint64_t seed, int d, int block, oq_rpbh_t* out) {
   return oq_make_rotation(seed, d, block, OQ_ROT_RPBH, out);
+}
+
+int oq_make_composed_rpbh(uint64_t seed, int d, int block, int rounds, oq_rpbh_t* out) {
+  clear_error();
+  if (rounds < 1 || rounds > 3) {
+    if (out) *out = nullptr;
+    return fail(OQ_ERR_ARG, "rounds must be 1, 2 or 3 (got %d)", rounds);
+  }
+  return make_rotation(seed, d, block, OQ_ROT_RPBH, rounds, out);
+}
+
+int oq_rotation_rounds(oq_rpbh_t r, int* rounds) {
+  clear_error();
+  if (!r || !rounds) return fail(OQ_ERR_ARG, "NULL argument");
+  *rounds = r->rounds;
+  return OQ_OK;
+}
+
+int oq_rpbh_export_round(oq_rpbh_t r, int round, int32_t* perm, uint32_t* sign_bits) {
+  clear_error();
+  if (!r) return fail(OQ_ERR_ARG, "NULL rpbh handle");
+  if (round < 1 || round > r->rounds) return fail(OQ_ERR_ARG, "round %d of a %d-round rotation", round, r->rounds);
+  const size_t words = r->sign_bits.size();
+  const int32_t* p = round == 1 ? r->perm.data() : r->perm_more.data() + (size_t)(round - 2) * r->d;
+  const uint32_t* b = round == 1 ? r->sign_bits.data() : r->sign_bits_more.data() + (size_t)(round - 2) * words;
+  if (perm) std::memcpy(perm, p, sizeof(int32_t) * r->d);
+  if (sign_bits) std::memcpy(sign_bits, b, sizeof(uint32_t) * words);
+  return OQ_OK;
 }
 
 int oq_rotation_kind(oq_rpbh_t r, int* kind) {
@@ -481,10 +578,12 @@ void oq_free_rpbh(oq_rpbh_t r) {
   int prev = -1;
   bool have_prev = cudaGetDevice(&prev) == cudaSuccess;
   for (int dev = 0; dev < OQ_MAX_DEVICES; ++dev) {
-    if (!r->dev_perm[dev] && !r->dev_signs[dev]) continue;
+    if (!r->dev_perm[dev] && !r->dev_signs[dev] && !r->dev_slots[dev] && !r->dev_csigns[dev]) continue;
     if (cudaSetDevice(dev) == cudaSuccess) {
       cudaFree(r->dev_perm[dev]);
       cudaFree(r->dev_signs[dev]);
+      cudaFree(r->dev_slots[dev]);
+      cudaFree(r->dev_csigns[dev]);
     }
   }
   if (have_prev) cudaSetDevice(prev);

@@ -17,9 +17,15 @@ struct oq_rpbh_s {
   int kind = OQ_ROT_RPBH;  // OQ_ROT_*; only OQ_ROT_RPBH permutes
   std::vector<int32_t> perm;        // pi, (P x)_j = x_{pi(j)}
   std::vector<uint32_t> sign_bits;  // bit j%32 of word j/32 set <=> sign_j = -1
+  // Composed rotation Pi_rounds ... Pi_1: rounds 2.. (round 1 is perm / sign_bits)
+  int rounds = 1;
+  std::vector<int32_t> perm_more;       // [rounds - 1][d]
+  std::vector<uint32_t> sign_bits_more;  // [rounds - 1][ceil(d/32)]
   std::mutex mu;
   uint16_t* dev_perm[OQ_MAX_DEVICES] = {};   // pi as uint16 [d]
   uint32_t* dev_signs[OQ_MAX_DEVICES] = {};  // sign words [d/32]
+  uint16_t* dev_slots[OQ_MAX_DEVICES] = {};  // composed kernel: [rounds][d] shared-memory slots
+  uint32_t* dev_csigns[OQ_MAX_DEVICES] = {};  // composed kernel: [rounds][d/32] sign words
 };
 
 struct oq_codebook_s {
@@ -52,6 +58,7 @@ uint16_t double_to_fp16_rne(double v);
 // Device-side state (oq_host.cpp).
 int current_device(int* dev);
 int rpbh_device_tables(oq_rpbh_t r, const uint16_t** perm, const uint32_t** signs);
+int rpbh_composed_tables(oq_rpbh_t r, const uint16_t** slots, const uint32_t** signs);
 int codebook_device_qtable(oq_codebook_t cb, const uint32_t** qtable);
 void build_qtable(oq_codebook_t cb);
 int device_status_word(int** status);
@@ -62,6 +69,8 @@ bool aligned16(const void* p);
 // Kernel launchers.
 int launch_rotq(oq_rpbh_t r, oq_codebook_t cb, const void* X, int M, uint8_t* codes, float* norm_f32,
                 uint16_t* norm_bf16, void* stream);
+int launch_rotq_composed(oq_rpbh_t r, oq_codebook_t cb, const void* X, int M, uint8_t* codes, float* norm_f32,
+                         uint16_t* norm_bf16, void* stream);
 int launch_cbgemm(int d, oq_codebook_t cb_a, oq_codebook_t cb_w, const uint8_t* a_codes, const float* a_norm, int M,
                   const uint8_t* w_codes, const uint16_t* w_norm, int N, const uint16_t* bias, int epilogue,
                   float* Y_f32, uint16_t* Y_bf16, void* stream);

@@ -58,7 +58,7 @@ extern "C" int oq_linear_noalloc(oq_rpbh_t r, oq_codebook_t cb_a, oq_codebook_t 
   // handle was created with this device current) and the status word (made
   // by the first kernel launch of any other entry point, or by
   // oq_get_device_status).
-  if (!r->dev_perm[dev])
+  if (!r->dev_perm[dev] || (r->rounds > 1 && !r->dev_slots[dev]))
     return oq::fail(OQ_ERR_ARG, "the RPBH handle has no tables on device %d: create it with that device current",
                     dev);
   if (!cb_a->dev_qtable[dev])

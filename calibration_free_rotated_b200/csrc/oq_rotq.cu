@@ -91,6 +91,7 @@ RotqPlan plan_rotq(int d, int h, int M, int qtable_len) {
 
 int launch_rotq(oq_rpbh_t r, oq_codebook_t cb, const void* X, int M, uint8_t* codes, float* norm_f32,
                 uint16_t* norm_bf16, void* stream) {
+  if (r->rounds > 1) return launch_rotq_composed(r, cb, X, M, codes, norm_f32, norm_bf16, stream);
   const int d = r->d, h = r->h, bits = cb->bits;
   const int qlen = (int)cb->qtable.size();
   if (qlen > 4097) return fail(OQ_ERR_UNSUPPORTED, "codebook d=%d bits=%d needs a %d-entry search table", cb->d, bits, qlen);

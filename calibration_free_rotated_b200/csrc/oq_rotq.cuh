@@ -263,6 +263,69 @@ struct Direct {
   }
 };
 
+// Unnormalised Walsh-Hadamard transform (Sylvester order) of the blocks of h =
+// 32 << LOGHB coordinates that span lanes 2^LOGHB-aligned: coordinate 32 l + i
+// of the block sits in v[i] of lane l (f32x2: both rows of a pair).  Five
+// in-thread stages over bits 0..4 of the block index, then LOGHB xor-shuffle
+// stages over bits 5.. (the lane bits).
+template <int LOGHB>
+__device__ __forceinline__ void fwht_pairs(unsigned long long (&v)[32], int lane) {
+#pragma unroll
+  for (int s = 1; s < 32; s <<= 1) {
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+      if ((i & s) == 0) {
+        const unsigned long long x0 = v[i], x1 = v[i + s];
+        v[i] = f2_add(x0, x1);
+        v[i + s] = f2_sub(x0, x1);
+      }
+    }
+  }
+#pragma unroll
+  for (int k = 0; k < LOGHB; ++k) {
+    const float sg = ((lane >> k) & 1) ? -1.0f : 1.0f;
+    const unsigned long long sg2 = f2_pack(sg, sg);
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+      float lo, hi;
+      f2_unpack(v[i], lo, hi);
+      const float olo = __shfl_xor_sync(0xFFFFFFFFu, lo, 1 << k);
+      const float ohi = __shfl_xor_sync(0xFFFFFFFFu, hi, 1 << k);
+      v[i] = f2_fma(v[i], sg2, f2_pack(olo, ohi));
+    }
+  }
+}
+
+// Centroid search and packing of the 32 coordinates of both rows held in v:
+// y = sat(x * A + 1/2) (A folds the row scale and 1/sqrt(h) into the table's
+// alpha), bucket q = round(y * nb) read from the low mantissa bits of
+// fma(y, nb, 1.5 * 2^23), table entry q = the bucket's boundary with the codes
+// below it in its low bits, code = entry + (y > boundary) from the sign of
+// (boundary - y); qkey is the table's shared address minus the bucket key of
+// q = 0.  wa / wb receive the packed codes of rows a / b.
+template <int BITS>
+__device__ __forceinline__ void search_pack(const unsigned long long (&v)[32], float A_a, float A_b, float nb,
+                                            uint32_t qkey, uint32_t (&wa)[BITS], uint32_t (&wb)[BITS]) {
+  const unsigned long long NB2 = f2_pack(nb, nb);
+  const unsigned long long C2 = f2_pack(12582912.0f, 12582912.0f);  // 1.5 * 2^23
+#pragma unroll
+  for (int k = 0; k < BITS; ++k) wa[k] = wb[k] = 0u;
+#pragma unroll
+  for (int i = 0; i < 32; ++i) {
+    float xa, xb;
+    f2_unpack(v[i], xa, xb);
+    const float ya = fma_sat(xa, A_a, 0.5f), yb = fma_sat(xb, A_b, 0.5f);
+    const unsigned long long y1 = f2_pack(ya, yb);
+    uint32_t qa, qb;
+    u2_unpack(f2_fma(y1, NB2, C2), qa, qb);
+    const uint32_t ea = lds_u32((qa << 2) + qkey), eb = lds_u32((qb << 2) + qkey);
+    uint32_t da, db;
+    u2_unpack(f2_sub(u2_pack(ea, eb), y1), da, db);
+    put_code<BITS>(wa, i, ea + (da >> 31));
+    put_code<BITS>(wb, i, eb + (db >> 31));
+  }
+}
+
 // Per-thread constants of the kernel (all registers).
 struct Thread {
   int tid, lane, pr, g, spr, nparts;
@@ -327,32 +390,7 @@ __device__ __forceinline__ void transform(const Args& a, const Thread& t, int it
     if ((t.lane & ((1 << a.seg_log) - 1)) == 0)
       t.partial[(it & 1) * t.nparts + (t.tid >> a.seg_log)] = make_float2(lo, hi);
   }
-  // in-thread Walsh-Hadamard butterflies over bits 0..4 of the block index
-#pragma unroll
-  for (int s = 1; s < 32; s <<= 1) {
-#pragma unroll
-    for (int i = 0; i < 32; ++i) {
-      if ((i & s) == 0) {
-        const unsigned long long x0 = v[i], x1 = v[i + s];
-        v[i] = f2_add(x0, x1);
-        v[i + s] = f2_sub(x0, x1);
-      }
-    }
-  }
-  // across the h/32 lanes of a block: bits 5.. of the block index
-#pragma unroll
-  for (int k = 0; k < LOGHB; ++k) {
-    const float sg = ((t.lane >> k) & 1) ? -1.0f : 1.0f;
-    const unsigned long long sg2 = f2_pack(sg, sg);
-#pragma unroll
-    for (int i = 0; i < 32; ++i) {
-      float lo, hi;
-      f2_unpack(v[i], lo, hi);
-      const float olo = __shfl_xor_sync(0xFFFFFFFFu, lo, 1 << k);
-      const float ohi = __shfl_xor_sync(0xFFFFFFFFu, hi, 1 << k);
-      v[i] = f2_fma(v[i], sg2, f2_pack(olo, ohi));
-    }
-  }
+  fwht_pairs<LOGHB>(v, t.lane);
 }
 
 // Normalise, search, pack and store stage `it`.
@@ -376,26 +414,8 @@ __device__ __forceinline__ void quantize(const Args& a, const Thread& t, int it,
   }
   const float A_a = sum_a > 0.0f ? a.alpha_h * rsqrtf(sum_a) : 0.0f;
   const float A_b = sum_b > 0.0f ? a.alpha_h * rsqrtf(sum_b) : 0.0f;
-  const unsigned long long NB2 = f2_pack(a.nb, a.nb);
-  const unsigned long long C2 = f2_pack(12582912.0f, 12582912.0f);  // 1.5 * 2^23
-
   uint32_t wa[BITS], wb[BITS];
-#pragma unroll
-  for (int k = 0; k < BITS; ++k) wa[k] = wb[k] = 0u;
-#pragma unroll
-  for (int i = 0; i < 32; ++i) {
-    float xa, xb;
-    f2_unpack(v[i], xa, xb);
-    const float ya = fma_sat(xa, A_a, 0.5f), yb = fma_sat(xb, A_b, 0.5f);
-    const unsigned long long y1 = f2_pack(ya, yb);
-    uint32_t qa, qb;
-    u2_unpack(f2_fma(y1, NB2, C2), qa, qb);
-    const uint32_t ea = lds_u32((qa << 2) + t.qkey), eb = lds_u32((qb << 2) + t.qkey);
-    uint32_t da, db;
-    u2_unpack(f2_sub(u2_pack(ea, eb), y1), da, db);
-    put_code<BITS>(wa, i, ea + (da >> 31));
-    put_code<BITS>(wb, i, eb + (db >> 31));
-  }
+  search_pack<BITS>(v, A_a, A_b, a.nb, t.qkey, wa, wb);
   const int row = row0 + 2 * t.pr;
   const size_t rb = (size_t)(a.d / 8 * BITS);
   uint8_t* dst = a.codes + (size_t)row * rb + (size_t)t.g * (4 * BITS);

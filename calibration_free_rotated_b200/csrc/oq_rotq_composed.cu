@@ -1,0 +1,272 @@
+// Composed RPBH rounds + norm + quantize + pack (rotation handles with k > 1
+// rounds).
+//
+// "Quantizing With Randomized Hadamard Transforms: Efficient Heuristic Now
+// Proven", Methodology and Key contributions 1 and 3: composing k randomized
+// Hadamard transforms makes every coordinate of any input close to Gaussian
+// (k = 2) and decorrelates the coordinates (k = 3).  With OrbitQuant's block
+// rotation each round is a full RPBH round, Pi_r = blkdiag(H_h D_r) P_r, and
+// the rows are rotated by Pi_k ... Pi_1 before the norm and the Lloyd-Max
+// search ("OrbitQuant", Methodology, "Online Activation Quantization").
+//
+// One CTA works on one row pair at a time (persistent over pairs); thread g
+// owns coordinates 32 g .. 32 g + 31 of both rows, the layout the butterflies
+// and the search of the one-round kernel use:
+//   * the pair is loaded from global memory (128-bit loads), widened to f32
+//     pairs and written to a shared array F of d 8-byte slots (row a, row b);
+//     a thread's 32 slots form a 256-byte run whose 16-byte chunks are rotated
+//     by the thread index, so the 128-bit writes are free of bank conflicts;
+//   * each round gathers its input from F through a table of precomputed slot
+//     indices (the permutation composed with the chunk rotation), flips the
+//     signs of its Rademacher word, runs the unnormalised block transform in
+//     registers and, unless it is the last round, writes the result back to F
+//     between two CTA barriers;
+//   * the sum of squares comes from round 1's gathered input (the rotation is
+//     orthogonal); the k factors sqrt(h) of the unnormalised transforms are
+//     folded into the search multiplier.
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cmath>
+#include <cstring>
+
+#include "oq_rotq.cuh"
+
+namespace oq {
+namespace rotq {
+
+struct ComposedArgs {
+  const uint16_t* X;
+  uint8_t* codes;
+  float* norm_f32;
+  uint16_t* norm_bf16;
+  const uint16_t* slots;  // [rounds][d]: F slot that round r's coordinate j reads
+  const uint32_t* signs;  // [rounds][d / 32]: sign words
+  const uint32_t* qtable;
+  int M, d, rounds, pairs, qtable_len;
+  uint32_t qt_off, part_off;  // byte offsets in dynamic shared memory
+  float alpha;                // search multiplier / h^(rounds / 2)
+  float nb;
+};
+
+__device__ __forceinline__ unsigned long long lds_u64(uint32_t addr) {
+  unsigned long long v;
+  asm volatile("ld.shared.u64 %0, [%1];" : "=l"(v) : "r"(addr));
+  return v;
+}
+
+// Writes the 32 f32 pairs of this thread to its 256-byte run of F (chunk c of
+// the run at position c ^ (g & 15)).
+__device__ __forceinline__ void store_run(uint32_t run, uint32_t rot, const unsigned long long (&v)[32]) {
+#pragma unroll
+  for (int c = 0; c < 16; ++c) {
+    uint32_t a0, b0, a1, b1;
+    u2_unpack(v[2 * c], a0, b0);
+    u2_unpack(v[2 * c + 1], a1, b1);
+    sts_u128(run + ((((uint32_t)c) ^ rot) << 4), a0, b0, a1, b1);
+  }
+}
+
+template <int BITS, int LOGHB>
+__global__ void __launch_bounds__(512, 1) rotq_composed_kernel(const __grid_constant__ ComposedArgs a) {
+  extern __shared__ __align__(1024) unsigned char smem[];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int T = a.d / 32;  // threads that own coordinates
+  const bool active = tid < T;
+  const uint32_t fbase = smem_u32(smem);
+  uint32_t* qtab = reinterpret_cast<uint32_t*>(smem + a.qt_off);
+  float2* part = reinterpret_cast<float2*>(smem + a.part_off);
+  for (int i = tid; i < a.qtable_len; i += blockDim.x) qtab[i] = a.qtable[i];
+  const uint32_t qkey = smem_u32(qtab) - 0x2D000000u;  // = qtab - 4 * bits(1.5 * 2^23)
+  const uint32_t run = fbase + 256u * (uint32_t)tid, rot = (uint32_t)tid & 15u;
+  const int nwarps = blockDim.x >> 5;
+  const size_t rowb = (size_t)a.d * 2;  // bytes of a bf16 row
+
+  for (int pr = blockIdx.x; pr < a.pairs; pr += gridDim.x) {
+    const int row = 2 * pr;
+    const bool has_b = row + 1 < a.M;
+    __syncthreads();  // the previous pair's readers of F and of the partials are done
+    if (active) {
+      const uint4* ra = reinterpret_cast<const uint4*>(reinterpret_cast<const unsigned char*>(a.X) + row * rowb) +
+                        4 * tid;
+      const uint4* rb = ra + rowb / 16;
+      unsigned long long v[32];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const uint4 A = ra[q];
+        const uint4 B = has_b ? rb[q] : make_uint4(0u, 0u, 0u, 0u);
+        const uint32_t wa[4] = {A.x, A.y, A.z, A.w}, wb[4] = {B.x, B.y, B.z, B.w};
+#pragma unroll
+        for (int m = 0; m < 4; ++m) {
+          v[8 * q + 2 * m] = u2_pack(wa[m] << 16, wb[m] << 16);
+          v[8 * q + 2 * m + 1] = u2_pack(wa[m] & 0xFFFF0000u, wb[m] & 0xFFFF0000u);
+        }
+      }
+      store_run(run, rot, v);
+    }
+    __syncthreads();
+
+    unsigned long long v[32];
+    unsigned long long sq[4] = {0ull, 0ull, 0ull, 0ull};
+    for (int r = 0; r < a.rounds; ++r) {
+      if (active) {
+        const uint4* sl = reinterpret_cast<const uint4*>(a.slots + (size_t)r * a.d) + 4 * tid;
+        const uint32_t sw = a.signs[(size_t)r * T + tid];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const uint4 S = sl[q];
+          const uint32_t s4[4] = {S.x, S.y, S.z, S.w};
+#pragma unroll
+          for (int m = 0; m < 8; ++m) {
+            const int i = 8 * q + m;
+            const uint32_t slot = (s4[m >> 1] >> (16 * (m & 1))) & 0xFFFFu;
+            uint32_t lo, hi;
+            u2_unpack(lds_u64(fbase + 8u * slot), lo, hi);
+            const uint32_t flip = (sw << (31 - i)) & 0x80000000u;  // sign of coordinate i
+            v[i] = u2_pack(lo ^ flip, hi ^ flip);
+          }
+        }
+      } else {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) v[i] = 0ull;
+      }
+      if (r == 0) {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) sq[i & 3] = f2_fma(v[i], v[i], sq[i & 3]);
+      }
+      fwht_pairs<LOGHB>(v, lane);
+      if (r + 1 < a.rounds) {
+        __syncthreads();  // every thread has gathered this round's input
+        if (active) store_run(run, rot, v);
+        __syncthreads();
+      }
+    }
+
+    // norms: per-warp shuffle sums, then the warps' partials in a fixed order
+    unsigned long long ss2 = f2_add(f2_add(sq[0], sq[1]), f2_add(sq[2], sq[3]));
+#pragma unroll
+    for (int k = 1; k < 32; k <<= 1) {
+      float lo, hi;
+      f2_unpack(ss2, lo, hi);
+      ss2 = f2_add(ss2, f2_pack(__shfl_xor_sync(0xFFFFFFFFu, lo, k), __shfl_xor_sync(0xFFFFFFFFu, hi, k)));
+    }
+    if (lane == 0) {
+      float lo, hi;
+      f2_unpack(ss2, lo, hi);
+      part[warp] = make_float2(lo, hi);
+    }
+    __syncthreads();
+    float sum_a = 0.0f, sum_b = 0.0f;
+    for (int w = 0; w < nwarps; ++w) {
+      const float2 p = part[w];
+      sum_a += p.x;
+      sum_b += p.y;
+    }
+    if (active) {
+      const float A_a = sum_a > 0.0f ? a.alpha * rsqrtf(sum_a) : 0.0f;
+      const float A_b = sum_b > 0.0f ? a.alpha * rsqrtf(sum_b) : 0.0f;
+      uint32_t wa[BITS], wb[BITS];
+      search_pack<BITS>(v, A_a, A_b, a.nb, qkey, wa, wb);
+      const size_t cb = (size_t)(a.d / 8 * BITS);
+      uint8_t* dst = a.codes + (size_t)row * cb + (size_t)tid * (4 * BITS);
+      store_words<BITS>(dst, wa);
+      if (has_b) store_words<BITS>(dst + cb, wb);
+      if (tid == 0) {
+        const float s_a = sqrtf(sum_a), s_b = sqrtf(sum_b);
+        if (a.norm_f32) {
+          a.norm_f32[row] = s_a;
+          if (has_b) a.norm_f32[row + 1] = s_b;
+        }
+        if (a.norm_bf16) {
+          const __nv_bfloat16 ha = __float2bfloat16_rn(s_a), hb = __float2bfloat16_rn(s_b);
+          a.norm_bf16[row] = *reinterpret_cast<const uint16_t*>(&ha);
+          if (has_b) a.norm_bf16[row + 1] = *reinterpret_cast<const uint16_t*>(&hb);
+        }
+      }
+    }
+  }
+}
+
+using ComposedFn = void (*)(ComposedArgs);
+
+template <int BITS>
+ComposedFn pick_composed_bits(int loghb) {
+  switch (loghb) {
+    case 0: return rotq_composed_kernel<BITS, 0>;
+    case 1: return rotq_composed_kernel<BITS, 1>;
+    case 2: return rotq_composed_kernel<BITS, 2>;
+    case 3: return rotq_composed_kernel<BITS, 3>;
+    case 4: return rotq_composed_kernel<BITS, 4>;
+    case 5: return rotq_composed_kernel<BITS, 5>;
+    default: return nullptr;
+  }
+}
+
+ComposedFn pick_composed(int bits, int loghb) {
+  switch (bits) {
+    case 1: return pick_composed_bits<1>(loghb);
+    case 2: return pick_composed_bits<2>(loghb);
+    case 3: return pick_composed_bits<3>(loghb);
+    case 4: return pick_composed_bits<4>(loghb);
+    case 5: return pick_composed_bits<5>(loghb);
+    case 6: return pick_composed_bits<6>(loghb);
+    default: return nullptr;
+  }
+}
+
+}  // namespace rotq
+
+int launch_rotq_composed(oq_rpbh_t r, oq_codebook_t cb, const void* X, int M, uint8_t* codes, float* norm_f32,
+                         uint16_t* norm_bf16, void* stream) {
+  const int d = r->d, h = r->h, bits = cb->bits;
+  int loghb = 0;
+  while ((32 << loghb) < h) ++loghb;
+  if (h < 32 || d % 32 != 0 || d > 16384)
+    return fail(OQ_ERR_UNSUPPORTED, "composed rotation kernel: d=%d h=%d (needs h >= 32, d <= 16384)", d, h);
+  const int qlen = (int)cb->qtable.size();
+  if (qlen > 4097) return fail(OQ_ERR_UNSUPPORTED, "codebook d=%d bits=%d needs a %d-entry search table", cb->d, bits, qlen);
+  rotq::ComposedFn kern = rotq::pick_composed(bits, loghb);
+  if (!kern) return fail(OQ_ERR_UNSUPPORTED, "no composed rotate+quantize kernel for bits=%d h=%d", bits, h);
+  const uint16_t* slots;
+  const uint32_t* signs;
+  if (int rc = rpbh_composed_tables(r, &slots, &signs)) return rc;
+  const uint32_t* qtable;
+  if (int rc = codebook_device_qtable(cb, &qtable)) return rc;
+  int nsm;
+  if (int rc = sm_count(&nsm)) return rc;
+
+  const int threads = (d / 32 + 31) / 32 * 32;
+  rotq::ComposedArgs a;
+  memset(&a, 0, sizeof(a));
+  a.X = static_cast<const uint16_t*>(X);
+  a.codes = codes;
+  a.norm_f32 = norm_f32;
+  a.norm_bf16 = norm_bf16;
+  a.slots = slots;
+  a.signs = signs;
+  a.qtable = qtable;
+  a.M = M;
+  a.d = d;
+  a.rounds = r->rounds;
+  a.pairs = (M + 1) / 2;
+  a.qtable_len = qlen;
+  a.qt_off = (uint32_t)threads * 256u;  // F: one 256-byte run per thread (inactive runs unused)
+  a.part_off = (a.qt_off + 4u * (uint32_t)qlen + 15u) & ~15u;
+  a.alpha = (float)((double)cb->qt_alpha / std::pow((double)h, 0.5 * r->rounds));
+  a.nb = (float)cb->qt_nb;
+  const size_t smem = a.part_off + (size_t)(threads / 32) * 8;
+
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return fail(OQ_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(e));
+  int per_sm = 0;
+  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, threads, smem);
+  if (e != cudaSuccess) return fail(OQ_ERR_CUDA, "occupancy query: %s", cudaGetErrorString(e));
+  if (per_sm < 1) return fail(OQ_ERR_UNSUPPORTED, "composed rotate+quantize kernel does not fit (d=%d)", d);
+  const int grid = std::min(a.pairs, nsm * per_sm);
+  kern<<<grid, threads, smem, (cudaStream_t)stream>>>(a);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return fail(OQ_ERR_CUDA, "composed rotate+quantize launch: %s", cudaGetErrorString(e));
+  return OQ_OK;
+}
+
+}  // namespace oq

@@ -33,6 +33,9 @@ _SIGS = {
     "oq_make_rpbh": (_c_int, [ctypes.c_uint64, _c_int, _c_int, ctypes.POINTER(_c_void_p)]),
     "oq_make_rotation": (_c_int, [ctypes.c_uint64, _c_int, _c_int, _c_int, ctypes.POINTER(_c_void_p)]),
     "oq_rotation_kind": (_c_int, [_c_void_p, ctypes.POINTER(_c_int)]),
+    "oq_make_composed_rpbh": (_c_int, [ctypes.c_uint64, _c_int, _c_int, _c_int, ctypes.POINTER(_c_void_p)]),
+    "oq_rotation_rounds": (_c_int, [_c_void_p, ctypes.POINTER(_c_int)]),
+    "oq_rpbh_export_round": (_c_int, [_c_void_p, _c_int, _c_void_p, _c_void_p]),
     "oq_rpbh_info": (_c_int, [_c_void_p, ctypes.POINTER(_c_int), ctypes.POINTER(_c_int)]),
     "oq_rpbh_export": (_c_int, [_c_void_p, _c_void_p, _c_void_p]),
     "oq_free_rpbh": (None, [_c_void_p]),
@@ -86,16 +89,23 @@ def _stream(stream):
 
 class Rpbh:
     """Handle of the RPBH rotation for one (seed, d, block); `kind` selects a
-    variant of the rotation ablation ("rpbh", "block_rht", "full_rht")."""
+    variant of the rotation ablation ("rpbh", "block_rht", "full_rht");
+    `rounds` > 1 composes that many RPBH rounds (oq_make_composed_rpbh)."""
 
-    def __init__(self, seed: int, d: int, block: int = 0, kind: str = "rpbh"):
+    def __init__(self, seed: int, d: int, block: int = 0, kind: str = "rpbh", rounds: int = 1):
         h = ctypes.c_void_p()
-        _check(_lib.oq_make_rotation(seed, d, block, ROTATIONS[kind], ctypes.byref(h)))
+        if rounds == 1:
+            _check(_lib.oq_make_rotation(seed, d, block, ROTATIONS[kind], ctypes.byref(h)))
+        else:
+            if kind != "rpbh":
+                raise ValueError("composed rounds are RPBH rounds")
+            _check(_lib.oq_make_composed_rpbh(seed, d, block, rounds, ctypes.byref(h)))
         self._h = h
-        dd, bb, kk = ctypes.c_int(), ctypes.c_int(), ctypes.c_int()
+        dd, bb, kk, rr = ctypes.c_int(), ctypes.c_int(), ctypes.c_int(), ctypes.c_int()
         _check(_lib.oq_rpbh_info(h, ctypes.byref(dd), ctypes.byref(bb)))
         _check(_lib.oq_rotation_kind(h, ctypes.byref(kk)))
-        self.seed, self.d, self.block = seed, dd.value, bb.value
+        _check(_lib.oq_rotation_rounds(h, ctypes.byref(rr)))
+        self.seed, self.d, self.block, self.rounds = seed, dd.value, bb.value, rr.value
         self.kind = {v: k for k, v in ROTATIONS.items()}[kk.value]
 
     @property
@@ -107,6 +117,14 @@ class Rpbh:
         perm = np.empty(self.d, dtype=np.int32)
         signs = np.empty((self.d + 31) // 32, dtype=np.uint32)
         _check(_lib.oq_rpbh_export(self._h, perm.ctypes.data, signs.ctypes.data))
+        return perm, signs
+
+    def export_round(self, rnd: int):
+        """(perm, sign words) of round `rnd` (1-based) of a composed rotation."""
+        import numpy as np
+        perm = np.empty(self.d, dtype=np.int32)
+        signs = np.empty((self.d + 31) // 32, dtype=np.uint32)
+        _check(_lib.oq_rpbh_export_round(self._h, rnd, perm.ctypes.data, signs.ctypes.data))
         return perm, signs
 
     def __del__(self):

@@ -113,6 +113,31 @@ OQ_API int oq_make_rotation(uint64_t seed, int d, int block, int kind, oq_rpbh_t
 /* Kind (OQ_ROT_*) of a rotation handle. */
 OQ_API int oq_rotation_kind(oq_rpbh_t r, int* kind);
 
+/* ---------------------------------------------------------------------------
+ * Composed RPBH rotation Pi^(k) = Pi_k ... Pi_1 of k = `rounds` rounds
+ * ("Quantizing With Randomized Hadamard Transforms: Efficient Heuristic Now
+ * Proven", Methodology: the composition of k randomized Hadamard transforms;
+ * Key contributions 1 and 3: two rounds make every coordinate of ANY input
+ * close to Gaussian, three also decorrelate the coordinates).  For a block
+ * rotation each round is a full RPBH round, Pi_r = blkdiag(H_h D_r) P_r with
+ * its own permutation and signs: the permutation is what lets a later round
+ * mix coordinates that an earlier one kept inside a block.
+ *   Round 1 is exactly oq_make_rpbh(seed, d, block); round r+1 continues the
+ *   same SplitMix64 stream after round r's draws (Fisher-Yates, then d signs).
+ * Every entry point accepts the handle (weights and activations rotated by the
+ * same Pi^(k), so it still cancels in oq_linear).  rounds = 1 is oq_make_rpbh;
+ * rounds 2 and 3 run a separate kernel that keeps the row pair in shared
+ * memory between rounds (d <= 16384, 32 <= block <= 1024).
+ * Errors: as oq_make_rpbh; OQ_ERR_ARG unless 1 <= rounds <= 3.
+ * ------------------------------------------------------------------------- */
+OQ_API int oq_make_composed_rpbh(uint64_t seed, int d, int block, int rounds, oq_rpbh_t* out);
+/* Rounds of a rotation handle (1 for every handle but a composed one). */
+OQ_API int oq_rotation_rounds(oq_rpbh_t r, int* rounds);
+/* Copies round `round` (1-based) of a handle: pi (int32[d], host) and its sign
+ * bits (uint32[ceil(d/32)], host), in oq_rpbh_export's layout.  Either output
+ * may be NULL.  OQ_ERR_ARG for a round outside 1..rounds. */
+OQ_API int oq_rpbh_export_round(oq_rpbh_t r, int round, int32_t* perm, uint32_t* sign_bits);
+
 /* d and h of a handle.  Either output may be NULL. */
 OQ_API int oq_rpbh_info(oq_rpbh_t r, int* d, int* block);
 

@@ -133,3 +133,34 @@ def test_rotation_variant_errors(oq):
     h = ctypes.c_void_p()
     assert oq.lib().oq_make_rotation(0, 256, 64, 7, ctypes.byref(h)) == oq.OQ_ERR_ARG
     assert oq.Rpbh(0, 3072, 1024, kind="full_rht").block == 1024
+
+
+@pytest.mark.parametrize("seed,d,block,rounds", [(0, 256, 64, 2), (3, 3072, 128, 3), (9, 1536, 0, 2)])
+def test_composed_rounds_match_the_oracle_draws(oq, seed, d, block, rounds):
+    # Composed rotation ([RHT] Methodology): round 1 is the RPBH draw, later
+    # rounds continue the same SplitMix64 stream; the library and the oracle
+    # implement the generator independently.
+    r = oq.Rpbh(seed, d, block, rounds=rounds)
+    assert r.rounds == rounds and r.kind == "rpbh"
+    ref = orpbh.draw_rounds(seed, d, rounds)
+    p1, s1 = oq.Rpbh(seed, d, block).export()
+    assert np.array_equal(r.export()[0], p1) and np.array_equal(r.export()[1], s1)
+    for k in range(rounds):
+        perm, words = r.export_round(k + 1)
+        assert np.array_equal(perm, ref[k][0])
+        bits = (words[np.arange(d) // 32] >> (np.arange(d) % 32).astype(np.uint32)) & 1
+        assert np.array_equal(np.where(bits == 1, -1.0, 1.0), ref[k][1])
+    assert oq.Rpbh(seed, d, block).rounds == 1
+
+
+def test_composed_rotation_errors(oq):
+    h = ctypes.c_void_p()
+    for bad in (0, 4, -1):
+        assert oq.lib().oq_make_composed_rpbh(0, 256, 64, bad, ctypes.byref(h)) == oq.OQ_ERR_ARG
+    r = oq.Rpbh(0, 256, 64, rounds=2)
+    with pytest.raises(oq.OQError):
+        r.export_round(3)
+    with pytest.raises(oq.OQError):
+        r.export_round(0)
+    with pytest.raises(ValueError):
+        oq.Rpbh(0, 256, 64, kind="block_rht", rounds=2)

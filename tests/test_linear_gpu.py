@@ -325,3 +325,27 @@ def test_bf16_only_output(oq, codebooks, ba, bw, epilogue, M, N):
                                  gelu=(epilogue == "gelu"))
     # bf16 output: the rounding adds up to 2^-9 relative per element
     assert _rel_fro(y16.double().cpu().numpy()[rows], ref) <= TOL + 2.0 ** -9
+
+
+def test_full_layer_with_composed_rotation(oq, codebooks):
+    # The composed rotation is orthogonal too, so it cancels in the product:
+    # oq_linear with a 2-round handle against the oracle on the same rounds.
+    d, h, M, N = 512, 64, 200, 272
+    r = oq.Rpbh(0, d, h, rounds=2)
+    X = inputs.to_bf16_bits(np.random.default_rng(8).standard_normal((M, d)))
+    W = inputs.weights(1, inputs.T_W, N, d)
+    cb = _lib_cb(oq, d, 4)
+    wc, wn = oq.quantize_weight(r, cb, _dev_bf16(W))
+    y, _ = oq.linear(r, cb, cb, _dev_bf16(X), wc, wn)
+    torch.cuda.synchronize()
+    oq.device_status()
+    R = orpbh.draw_rounds(0, d, 2)
+    c = codebooks(d, 4)["centroids"]
+    ca, s, _ = oqz.quantize_rows_composed(inputs.bf16_bits_to_f64(X), R, h, c)
+    cw, r16, _, _ = oqz.quantize_weight_rows_composed(inputs.bf16_bits_to_f64(W), R, h, c)
+    got_a = oqz.unpack_codes(oq.quantize_act(r, cb, _dev_bf16(X))[0].cpu().numpy(), 4, d)
+    got_w = oqz.unpack_codes(wc.cpu().numpy(), 4, d)
+    rows, cols = (got_a == ca).all(axis=1), (got_w == cw).all(axis=1)
+    assert rows.sum() > M // 2 and cols.sum() > N // 2
+    ref = olin.linear_from_codes(ca, s, cw, r16, c, c, d)
+    assert _rel_fro(y.double().cpu().numpy()[np.ix_(rows, cols)], ref[np.ix_(rows, cols)]) <= TOL

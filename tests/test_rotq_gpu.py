@@ -37,10 +37,10 @@ def oq():
 _handles = {}
 
 
-def _lib_handles(oq, seed, d, h, bits, kind="rpbh"):
-    key = (seed, d, h, bits, kind)
+def _lib_handles(oq, seed, d, h, bits, kind="rpbh", rounds=1):
+    key = (seed, d, h, bits, kind, rounds)
     if key not in _handles:
-        _handles[key] = (oq.Rpbh(seed, d, h, kind=kind), oq.Codebook(d, bits))
+        _handles[key] = (oq.Rpbh(seed, d, h, kind=kind, rounds=rounds), oq.Codebook(d, bits))
     return _handles[key]
 
 
@@ -48,9 +48,10 @@ def _to_dev(bits_u16):
     return torch.from_numpy(np.ascontiguousarray(bits_u16).view(np.int16)).cuda().view(torch.bfloat16)
 
 
-def _check_rows(oq, codebooks, X_bits, d, h, bits, seed=0, weight=False, rows=None, report=None, kind="rpbh"):
+def _check_rows(oq, codebooks, X_bits, d, h, bits, seed=0, weight=False, rows=None, report=None, kind="rpbh",
+                rounds=1):
     """Runs the kernel on all of X_bits; checks rows `rows` (default all) against the oracle."""
-    r, cb = _lib_handles(oq, seed, d, h, bits, kind)
+    r, cb = _lib_handles(oq, seed, d, h, bits, kind, rounds)
     X = _to_dev(X_bits)
     if weight:
         codes, norms = oq.quantize_weight(r, cb, X)
@@ -69,7 +70,13 @@ def _check_rows(oq, codebooks, X_bits, d, h, bits, seed=0, weight=False, rows=No
         perm = np.arange(d)
     ref = codebooks(d, bits)
     xs = inputs.bf16_bits_to_f64(X_bits[rows])
-    if weight:
+    if rounds > 1:
+        R = orpbh.draw_rounds(seed, d, rounds)
+        if weight:
+            ref_codes, r16, r_exact, T = oqz.quantize_weight_rows_composed(xs, R, h, ref["centroids"])
+        else:
+            ref_codes, s, T = oqz.quantize_rows_composed(xs, R, h, ref["centroids"])
+    elif weight:
         ref_codes, r16, r_exact, T = oqz.quantize_weight_rows(xs, perm, signs, h, ref["centroids"])
     else:
         ref_codes, s, T = oqz.quantize_rows(xs, perm, signs, h, ref["centroids"])
@@ -228,3 +235,63 @@ def test_empirical_distortion_matches_lloyd_max(oq, codebooks, d, h, bits):
     # N(0,1) rows: the error of a row is a mean over d coordinates; 1792 rows
     # bring the sampling spread well below 1%
     assert abs(err / theory - 1.0) < 0.01, (err, theory)
+
+
+@pytest.mark.parametrize("d,h,bits,rounds", [(256, 64, 4, 2), (3072, 128, 4, 2), (3072, 128, 2, 3), (1536, 256, 6, 2),
+                                              (12288, 128, 4, 2), (16384, 1024, 4, 3), (512, 32, 3, 2),
+                                              (8960, 128, 5, 3), (1024, 1024, 1, 2)])
+def test_composed_rounds(oq, codebooks, d, h, bits, rounds):
+    # [RHT] Methodology: Pi_k ... Pi_1, k RPBH rounds from one SplitMix64
+    # stream, against the oracle; ragged M, sparse rows and a zero row included
+    M = 301 if d >= 8192 else 999
+    X = inputs.sweep_activations(M, d)
+    rep = []
+    _check_rows(oq, codebooks, X, d, h, bits, rounds=rounds, report=rep)
+    assert rep[0][0] <= rep[0][1]
+    if d == 3072:
+        W = inputs.weights(2, inputs.T_W, 200, d)
+        _check_rows(oq, codebooks, W, d, h, bits, weight=True, rounds=rounds)
+
+
+def test_composed_edge_rows(oq, codebooks):
+    d, h = 3072, 128
+    rng = np.random.default_rng(1)
+    x = rng.standard_normal((7, d))
+    x[0] = 0.0
+    x[1] = 0.0
+    x[1, 17] = 2.0
+    x[2] *= 1e-18
+    x[3] *= 1e15
+    X = inputs.to_bf16_bits(x)
+    got, _ = _check_rows(oq, codebooks, X, d, h, 4, rounds=2)
+    assert np.all(got[0] == 7)
+    _check_rows(oq, codebooks, X[:1], d, h, 4, rounds=3)  # M = 1
+
+
+def test_composed_rounds_bring_one_hot_rows_to_the_lloyd_max_distortion(oq, codebooks):
+    # [RHT] Key contribution 1: two rounds make each coordinate of any input
+    # near-Gaussian, so the kernel's codes of one-hot and 8-sparse rows reach
+    # the Lloyd-Max distortion d * D(d, b); one round leaves them far above it.
+    d, h, b = 3072, 128, 4
+    rng = np.random.default_rng(2)
+    M = 512
+    x = np.zeros((M, d))
+    x[np.arange(M // 2), rng.integers(0, d, M // 2)] = rng.choice([-1.0, 1.0], M // 2)
+    for i in range(M // 2, M):
+        x[i, rng.choice(d, 8, replace=False)] = rng.standard_normal(8)
+    X = inputs.to_bf16_bits(x)
+    book = codebooks(d, b)
+    theory = d * book["distortion"]
+    ratios = {}
+    for k in (1, 2, 3):
+        r, cb = _lib_handles(oq, 0, d, h, b, rounds=k)
+        codes, _ = oq.quantize_act(r, cb, _to_dev(X))
+        torch.cuda.synchronize()
+        got = oqz.unpack_codes(codes.cpu().numpy(), b, d)
+        U = orpbh.rotate_composed(inputs.bf16_bits_to_f64(X), orpbh.draw_rounds(0, d, k), h)
+        T = U / np.linalg.norm(U, axis=1, keepdims=True)
+        e = np.sum((T - book["centroids"][got]) ** 2, axis=1)
+        ratios[k] = (e[: M // 2].mean() / theory, e[M // 2:].mean() / theory)
+    assert ratios[1][0] > 10.0 and ratios[1][1] > 2.5
+    for k in (2, 3):
+        assert 0.6 < ratios[k][0] < 1.3 and 0.8 < ratios[k][1] < 1.2, ratios
