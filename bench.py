@@ -405,7 +405,7 @@ def run_profile_case(args):
     torch.manual_seed(0)
     M, d, N = args.rows, args.d, args.n
     if args.profile == "rotq":
-        r = oq.Rpbh(0, d, args.block)
+        r = oq.Rpbh(0, d, args.block, rounds=args.rounds)
         cb = oq.Codebook(d, args.bits_a)
         X = torch.randn(M, d, device="cuda").to(torch.bfloat16)
         codes, norms = oq.quantize_act(r, cb, X)
@@ -444,7 +444,8 @@ def run_profile_case(args):
 def run_ablation(args):
     """Rotation ablation ([OQ] "Rotation Ablation (Table 3)", latency column):
     times oq_quantize_act (4-bit) under RPBH, Block-RHT (no permutation) and Full
-    RHT (d's largest power-of-two block) on N(0,1) bf16 rows.  L2 is flushed
+    RHT (d's largest power-of-two block) on N(0,1) bf16 rows, and the composed
+    RPBH of 2 and 3 rounds ([RHT] Methodology).  L2 is flushed
     (a 256 MB write) before every timed launch; CUDA events bracket the launch
     alone.  Prints one JSON line per (shape, rotation); not the contract line."""
     import torch
@@ -460,8 +461,9 @@ def run_ablation(args):
         codes = torch.empty(M, d // 2, dtype=torch.uint8, device="cuda")
         norms = torch.empty(M, dtype=torch.float32, device="cuda")
         cb = oq.Codebook(d, 4)
-        for kind, block in (("rpbh", args.block), ("block_rht", args.block), ("full_rht", 0)):
-            r = oq.Rpbh(0, d, block, kind=kind)
+        for kind, block, rounds in (("rpbh", args.block, 1), ("block_rht", args.block, 1), ("full_rht", 0, 1),
+                                    ("rpbh", args.block, 2), ("rpbh", args.block, 3)):
+            r = oq.Rpbh(0, d, block, kind=kind, rounds=rounds)
             for _ in range(args.warmup):
                 oq.quantize_act(r, cb, X, codes, norms)
             times = []
@@ -476,7 +478,8 @@ def run_ablation(args):
             oq.device_status()
             ms = statistics.median(times)
             gbs = algorithmic(M, d, 1, 4, 4)[0] / ms / 1e6
-            print(json.dumps({"ablation": "rotation", "kind": kind, "block": r.block, "rows": M, "d": d, "bits": 4,
+            print(json.dumps({"ablation": "rotation", "kind": kind, "rounds": rounds, "block": r.block, "rows": M,
+                              "d": d, "bits": 4,
                               "median_us": 1e3 * ms, "GB/s": gbs, "frac_hbm": gbs / peaks["hbm_gbs"],
                               "peak_source": src}), flush=True)
     return 0
@@ -592,16 +595,19 @@ def run_sweep(args):
             rows_dense = torch.arange(0, min(4096, M - n_adv), device=dev)
             rows_adv = torch.arange(M - n_adv, min(M - 1, M - n_adv + 4096), device=dev)  # not the zero row
             for h in (64, 128, 256):
-                r = oq.Rpbh(0, d, h)
-                perm, sbits = r.export()
-                sign = torch.tensor([-1.0 if (sbits[j >> 5] >> (j & 31)) & 1 else 1.0 for j in range(d)],
-                                    dtype=torch.float64, device=dev)
-                perm_t = torch.from_numpy(perm.astype(np.int64)).to(dev)
+                r = oq.Rpbh(0, d, h, rounds=args.rounds)
+                tables = []
+                for k in range(1, args.rounds + 1):
+                    perm, sbits = r.export_round(k)
+                    sign = torch.tensor([-1.0 if (sbits[j >> 5] >> (j & 31)) & 1 else 1.0 for j in range(d)],
+                                        dtype=torch.float64, device=dev)
+                    tables.append((torch.from_numpy(perm.astype(np.int64)).to(dev), sign))
                 H = _sylvester(h, dev) / math.sqrt(h)
 
                 def unit_rotated(rows):
-                    x = X[rows].double()[:, perm_t] * sign
-                    u = (x.view(len(rows), d // h, h) @ H.T).view(len(rows), d)
+                    u = X[rows].double()
+                    for perm_t, sign in tables:  # round 1 first
+                        u = ((u[:, perm_t] * sign).view(len(rows), d // h, h) @ H.T).view(len(rows), d)
                     return u / u.norm(dim=1, keepdim=True).clamp_min(1e-300)
 
                 T = {"dense": unit_rotated(rows_dense), "adversarial": unit_rotated(rows_adv)}
@@ -615,7 +621,8 @@ def run_sweep(args):
                                          args.warmup)
                     gbs = algorithmic(M, d, 1, bits, bits)[0] / ms / 1e6
                     cent = torch.from_numpy(np.asarray(c, dtype=np.float64)).to(dev)
-                    line = {"sweep": "rotate_quantize", "M": M, "d": d, "block": h, "bits": bits, "median_us": 1e3 * ms,
+                    line = {"sweep": "rotate_quantize", "M": M, "d": d, "block": h, "rounds": args.rounds, "bits": bits,
+                            "median_us": 1e3 * ms,
                             "GB/s": gbs, "frac_hbm": gbs / peaks["hbm_gbs"], "peak_source": src,
                             "mse_theory": d * D}
                     for key, rows in (("dense", rows_dense), ("adversarial", rows_adv)):
@@ -651,6 +658,7 @@ def main():
     ap.add_argument("--workload", choices=["flux_mlp", "wan_ffn"], help="per-kernel times of a two-layer workload")
     ap.add_argument("--sweep", action="store_true", help="the rotate+quantize sweep with empirical MSE")
     ap.add_argument("--sweep-rows", default="1024,16384,65536")
+    ap.add_argument("--rounds", type=int, default=1, help="composed RPBH rounds for --sweep and --profile rotq (1, 2 or 3)")
     ap.add_argument("--rows", type=int, default=4608)
     ap.add_argument("--d", type=int, default=3072)
     ap.add_argument("--n", type=int, default=9216)
