@@ -506,19 +506,41 @@ def run_workload(args):
     """Per-kernel times of the two-layer workloads (one JSON line each; not the
     contract line).  flux_mlp: X[4608 x 3072] -> fc1 [12288 x 3072] + GELU ->
     fc2 [3072 x 12288], W2A4, block 128.  wan_ffn: X[32760 x 1536] Student-t(3)
-    -> fc1 [8960 x 1536] + GELU -> fc2 [1536 x 8960], W4A6, block 128.  Every
-    launch is timed alone after a 256 MB L2 flush."""
+    -> fc1 [8960 x 1536] + GELU -> fc2 [1536 x 8960], W4A6, block 128.
+    flux_qkv_w3a3: the FLUX-like QKV projection (X[4608 x 3072] -> W[9216 x 3072]
+    + bias) at W3A3 ([OQ] Experiments, Qualitative Results).  Every launch is
+    timed alone after a 256 MB L2 flush."""
     import torch
     from calibration_free_rotated_b200 import build
     build.build()
     from calibration_free_rotated_b200 import inputs
     from calibration_free_rotated_b200 import orbitquant as oq
     peaks, src = load_peaks()
-    wl, M, d1, d2, bw, ba = {"flux_mlp": (3, 4608, 3072, 12288, 2, 4),
-                             "wan_ffn": (4, 32760, 1536, 8960, 4, 6)}[args.workload]
     h = 128
     dev = torch.device("cuda")
     bf = lambda bits: torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).to(dev).view(torch.bfloat16)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    if args.workload == "flux_qkv_w3a3":
+        M, d, N, b = 4608, 3072, 9216, 3
+        r, cb = oq.Rpbh(0, d, h), oq.Codebook(d, b)
+        X = bf(inputs.activations(2, M, d))
+        wc, wn = oq.quantize_weight(r, cb, bf(inputs.weights(2, inputs.T_W, N, d)))
+        bias = bf(inputs.bias(2, N))
+        ac, an = oq.quantize_act(r, cb, X)
+        Y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+        ms_q = _flush_and_time(lambda: oq.quantize_act(r, cb, X, ac, an), flush, args.steps, args.warmup)
+        ms_g = _flush_and_time(lambda: oq.linear_codes(d, cb, cb, ac, an, wc, wn, bias=bias, out_bf16=Y,
+                                                       want_f32=False, want_bf16=True), flush, args.steps, args.warmup)
+        oq.device_status()
+        gbs, tfs = algorithmic(M, d, N, b, b)[0] / ms_q / 1e6, 2.0 * M * N * d / ms_g / 1e9
+        print(json.dumps({"workload": args.workload, "M": M, "d": d, "N": N, "bits_w": b, "bits_a": b, "block": h,
+                          "kernels": {"act_quant": {"ms": ms_q, "GB/s": gbs, "frac": gbs / peaks["hbm_gbs"]},
+                                      "qkv": {"ms": ms_g, "TFLOP/s": tfs, "frac": tfs / peaks["bf16_tflops"]}},
+                          "peak_source": src, "step_ms": ms_q + ms_g,
+                          "TFLOP/s": 2.0 * M * N * d / (ms_q + ms_g) / 1e9}), flush=True)
+        return 0
+    wl, M, d1, d2, bw, ba = {"flux_mlp": (3, 4608, 3072, 12288, 2, 4),
+                             "wan_ffn": (4, 32760, 1536, 8960, 4, 6)}[args.workload]
     X = bf(inputs.activations(wl, M, d1))
     r1, r2 = oq.Rpbh(0, d1, h), oq.Rpbh(0, d2, h)
     ca1, cw1, ca2, cw2 = oq.Codebook(d1, ba), oq.Codebook(d1, bw), oq.Codebook(d2, ba), oq.Codebook(d2, bw)
@@ -529,7 +551,6 @@ def run_workload(args):
     a2c = torch.empty((M, d2 * ba // 8), dtype=torch.uint8, device=dev)
     a2n = torch.empty((M,), dtype=torch.float32, device=dev)
     Y2 = torch.empty((M, d1), dtype=torch.bfloat16, device=dev)
-    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
     steps = [
         ("act_quant_1", lambda: oq.quantize_act(r1, ca1, X, a1c, a1n), "hbm", algorithmic(M, d1, d2, ba, bw)[0]),
         ("fc1_gelu", lambda: oq.linear_codes(d1, ca1, cw1, a1c, a1n, w1c, w1n, epilogue="gelu", out_bf16=Y1,
@@ -655,7 +676,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--profile", choices=["rotq", "gemm"], help="launch one kernel only (for ncu captures)")
     ap.add_argument("--ablation", choices=["rotation"], help="time the rotation variants of the ablation table")
-    ap.add_argument("--workload", choices=["flux_mlp", "wan_ffn"], help="per-kernel times of a two-layer workload")
+    ap.add_argument("--workload", choices=["flux_mlp", "wan_ffn", "flux_qkv_w3a3"],
+                    help="per-kernel times of a layer workload")
     ap.add_argument("--sweep", action="store_true", help="the rotate+quantize sweep with empirical MSE")
     ap.add_argument("--sweep-rows", default="1024,16384,65536")
     ap.add_argument("--rounds", type=int, default=1, help="composed RPBH rounds for --sweep and --profile rotq (1, 2 or 3)")

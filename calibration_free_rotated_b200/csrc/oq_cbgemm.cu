@@ -80,6 +80,18 @@ struct PackedTile {
   static constexpr int kRowBytes = BK * BITS / 8;
 };
 
+// k-steps per packed ring stage (one TMA load of each operand): a tensor copy's
+// box must be a multiple of 16 bytes wide, so 3-bit rows (24 bytes per k-step)
+// travel two k-steps at a time; the two converter groups of those k-steps
+// share the stage.
+template <int BA, int BW>
+struct PackedUnit {
+  static constexpr int KP = (PackedTile<BA>::kRowBytes % 16 || PackedTile<BW>::kRowBytes % 16) ? 2 : 1;
+  static constexpr int kRowA = KP * PackedTile<BA>::kRowBytes;  // bytes of an A row in a stage
+  static constexpr int kRowB = KP * PackedTile<BW>::kRowBytes;
+  static_assert(kRowA % 16 == 0 && kRowB % 16 == 0, "TMA box width");
+};
+
 // ---- shared memory plan (offsets from a 1024-aligned base) -------------------
 // PAIR: two CTAs of a cluster share one 256 x 256 tile (cta_group::2); each holds
 // 128 rows of A and 128 of the 256 B rows.  Otherwise one CTA owns 128 x 256.
@@ -87,8 +99,8 @@ template <int BA, int BW, bool PAIR>
 struct Smem {
   static constexpr int kBnCta = PAIR ? BN / 2 : BN;
   static constexpr int kExpBBytes = kBnCta * BK * 2;
-  static constexpr int kPkA = BM * PackedTile<BA>::kRowBytes;
-  static constexpr int kPkB = kBnCta * PackedTile<BW>::kRowBytes;
+  static constexpr int kPkA = BM * PackedUnit<BA, BW>::kRowA;
+  static constexpr int kPkB = kBnCta * PackedUnit<BA, BW>::kRowB;
   static constexpr int kPkAStride = (kPkA + 127) / 128 * 128;
   static constexpr int kPkBStride = (kPkB + 127) / 128 * 128;
   // bytes that do not depend on the ring depth or the output staging
@@ -318,14 +330,21 @@ __device__ __forceinline__ void sts_v4(uint32_t addr, uint4 v) {
                : "memory");
 }
 
-// One packed row of a k-step (BYTES = 16, 32 or 48; 16-byte aligned) into registers.
+// One packed row of a k-step into registers: BYTES = 16, 32 or 48 (16-byte
+// aligned), or 24 for 3-bit codes (8-byte aligned).
 template <int BYTES>
 __device__ __forceinline__ void lds_row(uint32_t addr, uint32_t* w) {
+  if constexpr (BYTES % 16 == 0) {
 #pragma unroll
-  for (int i = 0; i < BYTES / 16; ++i)
-    asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
-                 : "=r"(w[4 * i]), "=r"(w[4 * i + 1]), "=r"(w[4 * i + 2]), "=r"(w[4 * i + 3])
-                 : "r"(addr + 16 * i));
+    for (int i = 0; i < BYTES / 16; ++i)
+      asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                   : "=r"(w[4 * i]), "=r"(w[4 * i + 1]), "=r"(w[4 * i + 2]), "=r"(w[4 * i + 3])
+                   : "r"(addr + 16 * i));
+  } else {
+#pragma unroll
+    for (int i = 0; i < BYTES / 8; ++i)
+      asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(w[2 * i]), "=r"(w[2 * i + 1]) : "r"(addr + 8 * i));
+  }
 }
 
 // Codes 8i .. 8i+7 of a packed row held in registers (little-endian bit stream).
@@ -335,6 +354,10 @@ __device__ __forceinline__ uint64_t row_chunk(const uint32_t* w, int i) {
     return w[i];
   } else if constexpr (BITS == 2) {
     return (w[i >> 1] >> (16 * (i & 1))) & 0xFFFFu;
+  } else if constexpr (BITS == 3) {  // 24 bits starting at byte 3 i
+    const int byte = 3 * i, wi = byte >> 2, sh = 8 * (byte & 3);
+    const uint64_t lo = w[wi], hi = (wi + 1 < 6) ? w[wi + 1] : 0u;
+    return (((hi << 32) | lo) >> sh) & 0xFFFFFFull;
   } else {  // 6 bits: 48 bits starting at byte 6 i
     const int byte = 6 * i, wi = byte >> 2, sh = 8 * (byte & 3);
     const uint64_t lo = w[wi], hi = (wi + 1 < 12) ? w[wi + 1] : 0u;
@@ -429,6 +452,23 @@ __device__ __forceinline__ uint4 expand8(uint64_t packed, const Lut8& t8, uint32
     r.y = prmt(lo, hi, 0x7362u);
     lo = prmt(q0, q0, n_hi);
     hi = prmt(q1, q1, n_hi);
+    r.z = prmt(lo, hi, 0x5140u);
+    r.w = prmt(lo, hi, 0x7362u);
+  } else if constexpr (BITS == 3) {
+    // t8 holds the byte planes of all eight entries (no sign folding).  The
+    // eight 3-bit codes are spread to one code per nibble in three
+    // shift-mask steps (shifts on the IMAD pipe): 12-bit halves to 16-bit
+    // halves, 6-bit pairs to bytes, codes to nibbles.
+    const uint32_t x = (uint32_t)packed;
+    uint32_t n = (x & 0x00000FFFu) | (mul_lo(x, 1u << 4) & 0x0FFF0000u);
+    n = (n & 0x003F003Fu) | (mul_lo(n, 1u << 2) & 0x3F003F00u);
+    n = (n & 0x07070707u) | (mul_lo(n, 1u << 1) & 0x70707070u);  // nibble i = code i
+    const uint32_t n_hi = shr_imad<16>(n);
+    uint32_t lo = prmt(t8.lo0, t8.lo1, n), hi = prmt(t8.hi0, t8.hi1, n);
+    r.x = prmt(lo, hi, 0x5140u);
+    r.y = prmt(lo, hi, 0x7362u);
+    lo = prmt(t8.lo0, t8.lo1, n_hi);
+    hi = prmt(t8.hi0, t8.hi1, n_hi);
     r.z = prmt(lo, hi, 0x5140u);
     r.w = prmt(lo, hi, 0x7362u);
   } else {  // 6 bits: shared 64-entry table
@@ -631,7 +671,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   if (threadIdx.x == 0) {
     for (int s = 0; s < PSTAGES; ++s) {
       mbar_init(bar(PK_FULL + s), 1);
-      mbar_init(bar(PK_EMPTY + s), GROUP_WARPS);           // the warps of one group
+      mbar_init(bar(PK_EMPTY + s), GROUP_WARPS * PackedUnit<BA, BW>::KP);  // the groups that read it
     }
     for (int s = 0; s < ESTAGES; ++s) {
       mbar_init(bar(EX_FULL + s), GROUP_WARPS * NCTA);     // one group in each CTA
@@ -673,12 +713,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   if (warp == TMA_WARP) {
     if (lane == 0) {
       constexpr uint32_t bytes = S::kPkA + S::kPkB;
-      uint32_t pc = 0;
+      constexpr int KP = PackedUnit<BA, BW>::KP;
+      uint32_t pc = 0;  // packed stages issued
       bool ok = true;
       for (int t = unit; t < num_tiles && ok; t += nunits) {
         const int m0 = (t % args.tiles_m) * TILE_M + (int)rank * BM;
         const int n0 = (t / args.tiles_m) * BN + (int)rank * BN_CTA;
-        for (int kb = 0; kb < KB; ++kb, ++pc) {
+        for (int kb = 0; kb < KB; kb += KP, ++pc) {
           const int s = pc % PSTAGES;
           const uint32_t ph = (pc / PSTAGES) & 1u;
           if (!wait_bounded(bar(PK_EMPTY + s), ph ^ 1u, abort_flag, args.status)) {
@@ -706,22 +747,26 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     // 2-bit tables as byte planes (low bytes of the 4 entries, high bytes)
     const uint32_t qa0 = prmt(args.lut_a[0], args.lut_a[1], 0x6420), qa1 = prmt(args.lut_a[0], args.lut_a[1], 0x7531);
     const uint32_t qw0 = prmt(args.lut_w[0], args.lut_w[1], 0x6420), qw1 = prmt(args.lut_w[0], args.lut_w[1], 0x7531);
-    if constexpr (BA == 4) ta = make_lut8(args.lut_a);
-    if constexpr (BW == 4) tw = make_lut8(args.lut_w);
+    if constexpr (BA == 4 || BA == 3) ta = make_lut8(args.lut_a);  // 4 bits: the negative half
+    if constexpr (BW == 4 || BW == 3) tw = make_lut8(args.lut_w);
     constexpr int RB_A = PackedTile<BA>::kRowBytes, RB_B = PackedTile<BW>::kRowBytes;
     constexpr int NB_ROWS = BN_CTA / BM;  // weight rows per thread: 1 (pair) or 2
     const uint32_t t_lane = tmem_base + ((uint32_t)(32 * q) << 16) + (uint32_t)(A_COL0 + 32 * g);
+    constexpr int KP = PackedUnit<BA, BW>::KP;
+    constexpr int ROW_A = PackedUnit<BA, BW>::kRowA, ROW_B = PackedUnit<BA, BW>::kRowB;
     for (uint32_t pc = (uint32_t)g, j = 0; pc < total_steps; pc += NUM_GROUPS, ++j) {
-      const int ps = pc % PSTAGES;
-      const uint32_t pph = (pc / PSTAGES) & 1u;
+      const uint32_t pu = pc / KP;  // packed stage that holds k-step pc
+      const int ps = pu % PSTAGES;
+      const uint32_t pph = (pu / PSTAGES) & 1u;
+      const uint32_t sub = pc % KP;  // this k-step's part of the stage's rows
       bool got = wait_bounded(bar(PK_FULL + ps), pph, abort_flag, args.status);
       __syncwarp();
       if (__any_sync(0xFFFFFFFFu, !got)) break;
       uint32_t wa[RB_A / 4], wb[NB_ROWS][RB_B / 4];
-      lds_row<RB_A>(sbase + S::kPackA + ps * S::kPkAStride + r * RB_A, wa);
+      lds_row<RB_A>(sbase + S::kPackA + ps * S::kPkAStride + r * ROW_A + sub * RB_A, wa);
 #pragma unroll
       for (int h = 0; h < NB_ROWS; ++h)
-        lds_row<RB_B>(sbase + S::kPackB + ps * S::kPkBStride + (r + BM * h) * RB_B, wb[h]);
+        lds_row<RB_B>(sbase + S::kPackB + ps * S::kPkBStride + (r + BM * h) * ROW_B + sub * RB_B, wb[h]);
       __syncwarp();
       if (lane == 0) mbar_arrive(bar(PK_EMPTY + ps));  // packed stage read by this warp
       uint32_t v[32];
@@ -1075,8 +1120,10 @@ template <int BA, int BW, bool PAIR>
 int launch_t(GemmArgs& a, const uint8_t* a_codes, const uint8_t* w_codes, int nsm, cudaStream_t stream) {
   using S = Smem<BA, BW, PAIR>;
   CUtensorMap ma, mb;
-  if (int rc = make_code_map(&ma, a_codes, a.M, a.K * BA / 8, BK * BA / 8, BM)) return rc;
-  if (int rc = make_code_map(&mb, w_codes, a.N, a.K * BW / 8, BK * BW / 8, S::kBnCta)) return rc;
+  if (int rc = make_code_map(&ma, a_codes, a.M, a.K * BA / 8, PackedUnit<BA, BW>::kRowA, BM)) return rc;
+  if (int rc = make_code_map(&mb, w_codes, a.N, a.K * BW / 8, PackedUnit<BA, BW>::kRowB, S::kBnCta)) return rc;
+  if ((a.K / BK) % PackedUnit<BA, BW>::KP != 0)
+    return fail(OQ_ERR_UNSUPPORTED, "3-bit codes need d %% 128 == 0 (d=%d)", a.K);
   CUtensorMap my16, my32;
   memset(&my16, 0, sizeof(my16));
   memset(&my32, 0, sizeof(my32));
@@ -1178,6 +1225,7 @@ int launch_cbgemm(int d, oq_codebook_t cb_a, oq_codebook_t cb_w, const uint8_t* 
   OQ_GEMM_CASE(6, 6)
   OQ_GEMM_CASE(6, 2)
   OQ_GEMM_CASE(2, 6)
+  OQ_GEMM_CASE(3, 3)
 #undef OQ_GEMM_CASE
   return fail(OQ_ERR_UNSUPPORTED, "no GEMM kernel for bits a=%d w=%d", ba, bw);
 }

@@ -702,8 +702,11 @@ static int check_linear_args(int d, oq_codebook_t cb_a, oq_codebook_t cb_w, int 
   if (d % 64 != 0) return fail(OQ_ERR_UNSUPPORTED, "the GEMM needs d %% 64 == 0 (d=%d)", d);
   if (N % 16 != 0) return fail(OQ_ERR_UNSUPPORTED, "the GEMM needs N %% 16 == 0 (N=%d)", N);
   auto ok_bits = [](int b) { return b == 2 || b == 4 || b == 6; };
-  if (!ok_bits(cb_a->bits) || !ok_bits(cb_w->bits))
-    return fail(OQ_ERR_UNSUPPORTED, "the GEMM needs bits in {2,4,6} (a=%d, w=%d)", cb_a->bits, cb_w->bits);
+  const bool w3a3 = cb_a->bits == 3 && cb_w->bits == 3;
+  if (!w3a3 && (!ok_bits(cb_a->bits) || !ok_bits(cb_w->bits)))
+    return fail(OQ_ERR_UNSUPPORTED, "the GEMM needs bits in {2,4,6}, or 3 for both (a=%d, w=%d)", cb_a->bits,
+                cb_w->bits);
+  if (w3a3 && d % 128 != 0) return fail(OQ_ERR_UNSUPPORTED, "3-bit codes need d %% 128 == 0 (d=%d)", d);
   if (M == 0 || N == 0) return OQ_OK;
   if (!Y_f32 && !Y_bf16) return fail(OQ_ERR_ARG, "at least one of Y_f32 / Y_bf16 is needed");
   if (!w_codes || !w_norm) return fail(OQ_ERR_ARG, "NULL weight buffer");

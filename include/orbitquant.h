@@ -208,7 +208,8 @@ OQ_API int oq_quantize_weight(oq_rpbh_t r, oq_codebook_t cb, const void* W, int 
  * epilogue    : OQ_EPI_NONE or OQ_EPI_GELU (exact erf form).
  * Y_f32       : device float [M][N] or NULL; Y_bf16: device bf16 [M][N] or
  *               NULL (at least one).  Row stride N elements.
- * Needs d % 64 == 0, N % 16 == 0, bits in {2, 4, 6} for both operands.
+ * Needs d % 64 == 0, N % 16 == 0, bits in {2, 4, 6} for both operands, or
+ * W3A3 (3 bits for both; [OQ] Experiments, Qualitative Results) with d % 128 == 0.
  * ------------------------------------------------------------------------- */
 OQ_API int oq_linear_codes(int d, oq_codebook_t cb_a, oq_codebook_t cb_w, const uint8_t* a_codes, const float* a_norm,
                     int M, const uint8_t* w_codes, const void* w_norm, int N, const void* bias, int epilogue,

@@ -164,3 +164,20 @@ def test_composed_rotation_errors(oq):
         r.export_round(0)
     with pytest.raises(ValueError):
         oq.Rpbh(0, 256, 64, kind="block_rht", rounds=2)
+
+
+def test_gemm_bit_width_checks(oq):
+    # W3A3 needs d % 128 == 0 (two 24-byte k-step rows per tensor copy); 3 bits
+    # only for both operands; argument errors are found before any launch.
+    lib = oq.lib()
+    cb3, cb4 = oq.Codebook(320, 3), oq.Codebook(320, 4)
+    null = ctypes.c_void_p()
+    assert lib.oq_linear_codes(320, cb3.handle, cb3.handle, null, null, 0, null, null, 0, null, 0, null, null,
+                               null) == oq.OQ_ERR_UNSUPPORTED
+    assert lib.oq_linear_codes(320, cb4.handle, cb3.handle, null, null, 0, null, null, 0, null, 0, null, null,
+                               null) == oq.OQ_ERR_UNSUPPORTED
+    cb3b, cb4b = oq.Codebook(384, 3), oq.Codebook(384, 4)
+    assert lib.oq_linear_codes(384, cb3b.handle, cb3b.handle, null, null, 0, null, null, 0, null, 0, null, null,
+                               null) == 0
+    assert lib.oq_linear_codes(384, cb4b.handle, cb4b.handle, null, null, 0, null, null, 0, null, 0, null, null,
+                               null) == 0

@@ -86,7 +86,7 @@ def _run_codes(oq, codebooks, ca, s, cw, r16, d, ba, bw, bias_bits=None, epilogu
     return y32.cpu().double().numpy(), (None if y16 is None else y16.float().cpu().double().numpy()), ref
 
 
-@pytest.mark.parametrize("ba,bw", [(4, 4), (4, 2), (6, 4), (2, 2), (6, 6), (2, 4)])
+@pytest.mark.parametrize("ba,bw", [(4, 4), (4, 2), (6, 4), (2, 2), (6, 6), (2, 4), (3, 3)])
 def test_codes_gemm_small_ragged(oq, codebooks, ba, bw):
     # several tiles in both M and N, M and N tails (M=200, N=272), K = 256
     d, h, M, N = 256, 64, 200, 272
@@ -298,7 +298,8 @@ def test_full_layer_with_rotation_variants(oq, codebooks, kind, h):
 
 
 @pytest.mark.parametrize("ba,bw,epilogue,M,N", [(4, 4, "none", 2048, 2560), (4, 2, "gelu", 1000, 2320),
-                                                 (6, 4, "gelu", 777, 1216), (2, 2, "none", 300, 272)])
+                                                 (6, 4, "gelu", 777, 1216), (2, 2, "none", 300, 272),
+                                                 (3, 3, "gelu", 1500, 2576)])
 def test_bf16_only_output(oq, codebooks, ba, bw, epilogue, M, N):
     # bf16-only output (the layer's usual call) takes the epilogue that first
     # evacuates the accumulator (spare TMEM columns + raw staging) and converts
@@ -349,3 +350,21 @@ def test_full_layer_with_composed_rotation(oq, codebooks):
     assert rows.sum() > M // 2 and cols.sum() > N // 2
     ref = olin.linear_from_codes(ca, s, cw, r16, c, c, d)
     assert _rel_fro(y.double().cpu().numpy()[np.ix_(rows, cols)], ref[np.ix_(rows, cols)]) <= TOL
+
+
+def test_w3a3_full_layer(oq, codebooks):
+    # W3A3 ([OQ] Experiments, Qualitative Results): 3-bit activation and weight
+    # codes, whose k-step rows (24 bytes) travel two k-steps per tensor copy.
+    # X[2000 x 3072] FLUX-like activations, W[1536 x 3072], bias; sampled rows.
+    M, N, d, h = 2000, 1536, 3072, 128
+    X = inputs.activations(2, M, d)
+    W = inputs.weights(2, inputs.T_W, N, d)
+    bias = inputs.bias(2, N)
+    y, y16 = _full_layer(oq, X, W, d, h, 3, 3, bias_bits=bias, want_bf16=True)
+    rows = np.linspace(0, M - 1, 24).astype(int)
+    ca, s = _oracle_act(codebooks, X[rows], d, h, 3)
+    cw, r16 = _oracle_weight(codebooks, W, d, h, 3)
+    c = codebooks(d, 3)["centroids"]
+    ref = olin.linear_from_codes(ca, s, cw, r16, c, c, d, bias=inputs.bf16_bits_to_f64(bias))
+    assert _rel_fro(y.cpu().double().numpy()[rows], ref) <= TOL
+    assert torch.equal(y16, y.to(torch.bfloat16))
