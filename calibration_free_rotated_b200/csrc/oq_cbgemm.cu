@@ -70,6 +70,7 @@ struct GemmArgs {
   int M, N, K;
   int tiles_m, num_tiles;
   int epilogue;
+  int stall;  // test hook: the producer issues no tensor copies (the waits run out)
   float inv_d;
   uint32_t lut_a[32];  // 64 fp16 entries, two per word (entry 2i in the low half)
   uint32_t lut_w[32];
@@ -711,7 +712,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   const uint32_t total_steps = my_tiles * (uint32_t)KB;
 
   if (warp == TMA_WARP) {
-    if (lane == 0) {
+    if (lane == 0 && !args.stall) {
       constexpr uint32_t bytes = S::kPkA + S::kPkB;
       constexpr int KP = PackedUnit<BA, BW>::KP;
       uint32_t pc = 0;  // packed stages issued
@@ -1197,6 +1198,7 @@ int launch_cbgemm(int d, oq_codebook_t cb_a, oq_codebook_t cb_w, const uint8_t* 
   a.K = d;
   a.epilogue = epilogue;
   a.inv_d = (float)(1.0 / (double)d);
+  a.stall = take_test_stall(2);
   for (int i = 0; i < 32; ++i) {
     auto entry = [](oq_codebook_t cb, int k) -> uint32_t {
       return k < (int)cb->lut.size() ? cb->lut[k] : 0u;

@@ -8,12 +8,15 @@
 // ([TQ]) slides 14-16 (sphere marginal, continuous k-means).
 #include <cuda_runtime.h>
 
+#include <atomic>
 #include <cmath>
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
 #include <new>
 #include <string>
+
+#include <nvtx3/nvToolsExt.h>
 
 #include "oq_internal.h"
 
@@ -413,6 +416,22 @@ int rpbh_device_tables(oq_rpbh_t r, const uint16_t** perm, const uint32_t** sign
   return OQ_OK;
 }
 
+// Host span of an entry point for timeline tools (NVTX; a no-op unless a tool
+// such as ncu --nvtx is attached).
+struct NvtxRange {
+  explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+  ~NvtxRange() { nvtxRangePop(); }
+  NvtxRange(const NvtxRange&) = delete;
+  NvtxRange& operator=(const NvtxRange&) = delete;
+};
+
+static std::atomic<int> g_test_stall{0};
+
+int take_test_stall(int kernel) {
+  int expected = kernel;
+  return g_test_stall.compare_exchange_strong(expected, 0) ? 1 : 0;
+}
+
 // One round of draws from the SplitMix64 stream `st`: the Fisher-Yates
 // permutation of 0..d-1 (for i = d-1 .. 1: j = next() mod (i+1), swap), then
 // d Rademacher signs (sign_j = -1 when the top bit of next() is set).
@@ -496,6 +515,13 @@ using namespace oq;
 extern "C" {
 
 int oq_version(void) { return OQ_VERSION; }
+
+int oq_test_stall_next(int kernel) {
+  clear_error();
+  if (kernel < 0 || kernel > 2) return fail(OQ_ERR_ARG, "kernel must be 0 (disarm), 1 or 2 (got %d)", kernel);
+  g_test_stall.store(kernel);
+  return OQ_OK;
+}
 
 const char* oq_last_error(void) { return g_last_error.c_str(); }
 
@@ -671,6 +697,7 @@ static int check_quant_args(oq_rpbh_t r, oq_codebook_t cb, const void* X, int M,
 int oq_quantize_act(oq_rpbh_t r, oq_codebook_t cb, const void* X, int M, uint8_t* codes, float* norms,
                     void* stream) {
   clear_error();
+  NvtxRange nvtx("oq_quantize_act");
   if (int rc = check_quant_args(r, cb, X, M, codes, norms)) return rc;
   if (M == 0) return OQ_OK;
   return launch_rotq(r, cb, X, M, codes, norms, nullptr, stream);
@@ -679,6 +706,7 @@ int oq_quantize_act(oq_rpbh_t r, oq_codebook_t cb, const void* X, int M, uint8_t
 int oq_quantize_weight(oq_rpbh_t r, oq_codebook_t cb, const void* W, int N, uint8_t* codes, void* norms_bf16,
                        void* stream) {
   clear_error();
+  NvtxRange nvtx("oq_quantize_weight");
   if (int rc = check_quant_args(r, cb, W, N, codes, norms_bf16)) return rc;
   if (N == 0) return OQ_OK;
   return launch_rotq(r, cb, W, N, codes, nullptr, (uint16_t*)norms_bf16, stream);
@@ -720,6 +748,7 @@ int oq_linear_codes(int d, oq_codebook_t cb_a, oq_codebook_t cb_w, const uint8_t
                     int M, const uint8_t* w_codes, const void* w_norm, int N, const void* bias, int epilogue,
                     float* Y_f32, void* Y_bf16, void* stream) {
   clear_error();
+  NvtxRange nvtx("oq_linear_codes");
   if (int rc = check_linear_args(d, cb_a, cb_w, M, w_codes, w_norm, N, bias, epilogue, Y_f32, Y_bf16)) return rc;
   if (M == 0 || N == 0) return OQ_OK;
   if (!a_codes || !a_norm) return fail(OQ_ERR_ARG, "NULL activation buffer");
@@ -732,6 +761,7 @@ int oq_linear(oq_rpbh_t r, oq_codebook_t cb_a, oq_codebook_t cb_w, const void* X
               const void* w_norm, int N, const void* bias, int epilogue, float* Y_f32, void* Y_bf16,
               void* workspace, size_t workspace_bytes, void* stream) {
   clear_error();
+  NvtxRange nvtx("oq_linear");
   if (!r) return fail(OQ_ERR_ARG, "NULL rpbh handle");
   if (int rc = check_linear_args(r->d, cb_a, cb_w, M, w_codes, w_norm, N, bias, epilogue, Y_f32, Y_bf16)) return rc;
   if (M == 0 || N == 0) return OQ_OK;

@@ -65,6 +65,8 @@ int device_status_word(int** status);
 int device_status_word_if_present(int** status);  // never allocates
 int sm_count(int* n);
 bool aligned16(const void* p);
+// Test hook (oq_test_stall_next): 1 exactly once, for the next launch of `kernel`.
+int take_test_stall(int kernel);
 
 // Kernel launchers.
 int launch_rotq(oq_rpbh_t r, oq_codebook_t cb, const void* X, int M, uint8_t* codes, float* norm_f32,

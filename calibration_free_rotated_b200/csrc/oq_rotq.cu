@@ -137,6 +137,7 @@ int launch_rotq(oq_rpbh_t r, oq_codebook_t cb, const void* X, int M, uint8_t* co
   a.ring_off = p.ring_off;
   a.alpha_h = (float)((double)cb->qt_alpha / std::sqrt((double)h));
   a.nb = (float)cb->qt_nb;
+  a.stall = take_test_stall(1);
 
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)p.smem);
   if (e != cudaSuccess) return fail(OQ_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(e));

@@ -29,6 +29,7 @@ struct Args {
   uint32_t bar_off, part_off, qt_off, ring_off;  // byte offsets in dynamic shared memory
   float alpha_h;                                 // alpha / sqrt(h)
   float nb;                                      // buckets of the search table
+  int stall;                                     // test hook: issue no copies (the waits run out)
 };
 
 // Kernel configurations: pair-buffer stride (IBS) and gather-address form.
@@ -83,7 +84,7 @@ static __device__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity, int* sta
 template <int CFG>
 __device__ __forceinline__ void issue_stage_load(const Args& a, uint32_t ring, uint32_t bars, int it, int lane) {
   const int grp = blockIdx.x + it * gridDim.x;
-  if (grp >= a.groups) return;
+  if (grp >= a.groups || a.stall) return;
   const int slot = it % Cfg<CFG>::STAGES;
   const int R = 2 * a.P;
   const int row0 = grp * R;

@@ -76,6 +76,15 @@ OQ_API const char* oq_last_error(void);
  * synchronising `stream`.  Returns OQ_OK, OQ_ERR_TIMEOUT, or OQ_ERR_CUDA. */
 OQ_API int oq_get_device_status(void* stream);
 
+/* Test hook for the failure path: the next launch of kernel 1 (rotate +
+ * quantize, one-round rotations) or kernel 2 (codebook GEMM), on any stream,
+ * issues none of its bulk / tensor copies.  Its bounded waits then run out
+ * (about 1 s), it records OQ_ERR_TIMEOUT in the device status word and every
+ * CTA leaves through its normal teardown, so the context stays usable; the
+ * launch's outputs are undefined.  kernel 0 disarms.  One launch consumes it.
+ * Errors: OQ_ERR_ARG for a kernel outside 0..2. */
+OQ_API int oq_test_stall_next(int kernel);
+
 /* ---------------------------------------------------------------------------
  * RPBH rotation  Pi_d = blkdiag(H_h D_1, ..., H_h D_{d/h}) P_pi
  * [OQ] Methodology, "Randomized Permuted Block-Hadamard (RPBH) Rotation".

@@ -181,3 +181,11 @@ def test_gemm_bit_width_checks(oq):
                                null) == 0
     assert lib.oq_linear_codes(384, cb4b.handle, cb4b.handle, null, null, 0, null, null, 0, null, 0, null, null,
                                null) == 0
+
+
+def test_stall_hook_arguments(oq):
+    lib = oq.lib()
+    assert lib.oq_test_stall_next(3) == oq.OQ_ERR_ARG
+    assert lib.oq_test_stall_next(-1) == oq.OQ_ERR_ARG
+    assert lib.oq_test_stall_next(2) == oq.OQ_OK
+    assert lib.oq_test_stall_next(0) == oq.OQ_OK  # disarmed again
