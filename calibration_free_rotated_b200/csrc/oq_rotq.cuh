@@ -468,6 +468,13 @@ __global__ void __launch_bounds__(CFG == 2 ? 512 : 384, 1) rotq_kernel(const __g
       asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(t.s_bars + 8u * s) : "memory");
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
+  // The first stages' copies start now, so their HBM latency overlaps the
+  // table loads below (only warp 0, which made the barriers, touches them
+  // before the CTA barrier).
+  if (warp == 0) {
+    __syncwarp();
+    for (int s = 0; s < Cfg<CFG>::STAGES; ++s) issue_stage_load<CFG>(a, t.s_ring, t.s_bars, s, t.lane);
+  }
   for (int k = t.tid; k < a.qtable_len; k += blockDim.x) qtab[k] = __ldg(a.qtable + k);
 
   // gather addresses: pair word of column c of pair pr sits at word
@@ -514,10 +521,6 @@ __global__ void __launch_bounds__(CFG == 2 ? 512 : 384, 1) rotq_kernel(const __g
     t.src_direct = t.s_ring + (uint32_t)t.pr * (uint32_t)d * 2u + (uint32_t)t.g * 64u;
   }
   __syncthreads();
-
-  if (warp == 0) {
-    for (int s = 0; s < Cfg<CFG>::STAGES; ++s) issue_stage_load<CFG>(a, t.s_ring, t.s_bars, s, t.lane);
-  }
 
   const int n_it = a.groups > (int)blockIdx.x ? (a.groups - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
   if (n_it == 0) return;
