@@ -73,3 +73,21 @@ def test_noalloc_rejects_sizes_beyond_the_static_scratch(oq):
         oq.linear_noalloc(r, cb, cb, X, w, wn, out_f32=y)
     assert e.value.code == oq.OQ_ERR_UNSUPPORTED
     assert "static scratch" in str(e.value)
+
+
+def test_noalloc_with_a_composed_rotation(oq):
+    # A 2-round composed rotation uploads its round tables when the handle is
+    # made (with the device current), so the no-allocation path runs with it.
+    torch.cuda.set_device(0)
+    d, h, N, M = 1536, 128, 512, 700
+    r = oq.Rpbh(0, d, h, rounds=2)
+    cb = oq.Codebook(d, 4)
+    W = _dev_bf16(inputs.weights(4, inputs.T_W, N, d))
+    w_codes, w_norm = oq.quantize_weight(r, cb, W)
+    X = _dev_bf16(inputs.activations(4, M, d))
+    ref, _ = oq.linear(r, cb, cb, X, w_codes, w_norm)
+    y32 = torch.full((M, N), float("nan"), device="cuda")
+    oq.linear_noalloc(r, cb, cb, X, w_codes, w_norm, out_f32=y32)
+    torch.cuda.synchronize()
+    oq.device_status()
+    assert torch.equal(y32, ref)  # same kernels on the same inputs
