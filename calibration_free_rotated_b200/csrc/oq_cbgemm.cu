@@ -10,13 +10,14 @@
 // sm_100a design (persistent; tiles of 256 x 256 shared by a CTA pair of a
 // cluster with tcgen05 cta_group::2, or 128 x 256 on one CTA when M <= 128):
 //   warp 20      TMA producer: 2-D tensor copies of the packed code tiles into a
-//                4-deep packed ring (each CTA: 128 rows of A, its B rows).
-//   warps 0..7   A converters: expand activation codes through the fp16 LUT and
-//                write them straight into TMEM with tcgen05.st (warp w owns TMEM
-//                lanes 32 (w % 4) .. +31 = its tile rows, half of K each).
-//   warps 8..15  B converters: expand weight codes into the canonical K-major
-//                128-byte-swizzled UMMA layout in shared memory.
-//                (Both use register byte-permute tables for 2 and 4 bits and a
+//                4- or 8-deep packed ring (each CTA: 128 rows of A, its B rows;
+//                3-bit codes travel two k-steps per copy).
+//   warps 0..15  converters, four groups of four warps running out of phase,
+//                group g expanding k-steps g, g+4, ...  Thread r of a group
+//                expands activation row r through the fp16 LUT straight into
+//                TMEM lane r with tcgen05.st, and its weight row(s) into the
+//                canonical K-major 128-byte-swizzled UMMA layout in shared
+//                memory.  (Register byte-permute tables for 2, 3 and 4 bits, a
 //                128-byte shared table for 6 bits.)
 //   warp 21      one elected lane of the leader CTA's warp issues tcgen05.mma (kind::f16,
 //                A from TMEM, B from shared memory, M = 256 across the pair,
