@@ -368,3 +368,34 @@ def test_w3a3_full_layer(oq, codebooks):
     ref = olin.linear_from_codes(ca, s, cw, r16, c, c, d, bias=inputs.bf16_bits_to_f64(bias))
     assert _rel_fro(y.cpu().double().numpy()[rows], ref) <= TOL
     assert torch.equal(y16, y.to(torch.bfloat16))
+
+
+def test_full_layer_replays_from_a_cuda_graph(oq, codebooks):
+    # The full layer captured once in a CUDA graph (outputs, workspace and
+    # inputs preallocated; one eager call first so that every device table
+    # exists) and replayed on new inputs written into the same buffers: the
+    # replay equals eager calls bit for bit.
+    d, h, M, N = 3072, 128, 640, 1024
+    r, cb = oq.Rpbh(0, d, h), oq.Codebook(d, 4)
+    wc, wn = oq.quantize_weight(r, cb, _dev_bf16(inputs.weights(2, inputs.T_W, N, d)))
+    bias = _dev_bf16(inputs.bias(2, N))
+    X = _dev_bf16(inputs.activations(2, 4608, d, rows=(0, M)))
+    y16 = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+    ws = torch.empty((oq.workspace_bytes(M, d, 4),), dtype=torch.uint8, device="cuda")
+    s = torch.cuda.Stream()
+    with torch.cuda.stream(s):
+        oq.linear(r, cb, cb, X, wc, wn, bias=bias, out_bf16=y16, want_f32=False, want_bf16=True, workspace=ws,
+                  stream=s)
+    s.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=s):
+        oq.linear(r, cb, cb, X, wc, wn, bias=bias, out_bf16=y16, want_f32=False, want_bf16=True, workspace=ws,
+                  stream=s)
+    for rows in ((1000, 1000 + M), (3000, 3000 + M)):
+        X.copy_(_dev_bf16(inputs.activations(2, 4608, d, rows=rows)))
+        g.replay()
+        torch.cuda.synchronize()
+        _, ref = oq.linear(r, cb, cb, X, wc, wn, bias=bias, want_f32=False, want_bf16=True)
+        torch.cuda.synchronize()
+        oq.device_status()
+        assert torch.equal(y16, ref)
