@@ -12,6 +12,7 @@
 #include <cmath>
 #include <cstdarg>
 #include <cstdio>
+#include <cstdlib>
 #include <cstring>
 #include <new>
 #include <string>
@@ -516,6 +517,35 @@ extern "C" {
 
 int oq_version(void) { return OQ_VERSION; }
 
+// Synchronous checking (OQ_DEBUG=1 in the environment, or oq_set_debug): each
+// launching entry point then waits for its stream and returns the device status
+// word itself, so an asynchronous give-up is reported by the call that caused
+// it.  Off by default, when the calls stay asynchronous.
+static std::atomic<int> g_debug{-1};  // -1: the environment is not read yet
+
+static bool debug_on() {
+  int v = g_debug.load();
+  if (v < 0) {
+    const char* e = std::getenv("OQ_DEBUG");
+    v = (e && e[0] && e[0] != '0') ? 1 : 0;
+    int expected = -1;
+    g_debug.compare_exchange_strong(expected, v);
+    v = g_debug.load();
+  }
+  return v != 0;
+}
+
+static int finish(int rc, void* stream) {
+  if (rc != OQ_OK || !debug_on()) return rc;
+  return oq_get_device_status(stream);
+}
+
+int oq_set_debug(int on) {
+  clear_error();
+  g_debug.store(on ? 1 : 0);
+  return OQ_OK;
+}
+
 int oq_test_stall_next(int kernel) {
   clear_error();
   if (kernel < 0 || kernel > 2) return fail(OQ_ERR_ARG, "kernel must be 0 (disarm), 1 or 2 (got %d)", kernel);
@@ -700,7 +730,7 @@ int oq_quantize_act(oq_rpbh_t r, oq_codebook_t cb, const void* X, int M, uint8_t
   NvtxRange nvtx("oq_quantize_act");
   if (int rc = check_quant_args(r, cb, X, M, codes, norms)) return rc;
   if (M == 0) return OQ_OK;
-  return launch_rotq(r, cb, X, M, codes, norms, nullptr, stream);
+  return finish(launch_rotq(r, cb, X, M, codes, norms, nullptr, stream), stream);
 }
 
 int oq_quantize_weight(oq_rpbh_t r, oq_codebook_t cb, const void* W, int N, uint8_t* codes, void* norms_bf16,
@@ -709,7 +739,7 @@ int oq_quantize_weight(oq_rpbh_t r, oq_codebook_t cb, const void* W, int N, uint
   NvtxRange nvtx("oq_quantize_weight");
   if (int rc = check_quant_args(r, cb, W, N, codes, norms_bf16)) return rc;
   if (N == 0) return OQ_OK;
-  return launch_rotq(r, cb, W, N, codes, nullptr, (uint16_t*)norms_bf16, stream);
+  return finish(launch_rotq(r, cb, W, N, codes, nullptr, (uint16_t*)norms_bf16, stream), stream);
 }
 
 size_t oq_linear_workspace_bytes(int M, int d, int bits_a) {
@@ -753,8 +783,9 @@ int oq_linear_codes(int d, oq_codebook_t cb_a, oq_codebook_t cb_w, const uint8_t
   if (M == 0 || N == 0) return OQ_OK;
   if (!a_codes || !a_norm) return fail(OQ_ERR_ARG, "NULL activation buffer");
   if (!aligned16(a_codes) || !aligned16(a_norm)) return fail(OQ_ERR_ALIGN, "activation buffers must be 16-byte aligned");
-  return launch_cbgemm(d, cb_a, cb_w, a_codes, a_norm, M, w_codes, (const uint16_t*)w_norm, N,
-                       (const uint16_t*)bias, epilogue, Y_f32, (uint16_t*)Y_bf16, stream);
+  return finish(launch_cbgemm(d, cb_a, cb_w, a_codes, a_norm, M, w_codes, (const uint16_t*)w_norm, N,
+                              (const uint16_t*)bias, epilogue, Y_f32, (uint16_t*)Y_bf16, stream),
+                stream);
 }
 
 int oq_linear(oq_rpbh_t r, oq_codebook_t cb_a, oq_codebook_t cb_w, const void* X, int M, const uint8_t* w_codes,
@@ -773,9 +804,10 @@ int oq_linear(oq_rpbh_t r, oq_codebook_t cb_a, oq_codebook_t cb_w, const void* X
   size_t code_bytes = need - 4 * (size_t)M;
   float* a_norm = (float*)((uint8_t*)workspace + code_bytes);
   if (int rc = check_quant_args(r, cb_a, X, M, a_codes, a_norm)) return rc;
-  if (int rc = launch_rotq(r, cb_a, X, M, a_codes, a_norm, nullptr, stream)) return rc;
-  return launch_cbgemm(r->d, cb_a, cb_w, a_codes, a_norm, M, w_codes, (const uint16_t*)w_norm, N,
-                       (const uint16_t*)bias, epilogue, Y_f32, (uint16_t*)Y_bf16, stream);
+  if (int rc = finish(launch_rotq(r, cb_a, X, M, a_codes, a_norm, nullptr, stream), stream)) return rc;
+  return finish(launch_cbgemm(r->d, cb_a, cb_w, a_codes, a_norm, M, w_codes, (const uint16_t*)w_norm, N,
+                              (const uint16_t*)bias, epilogue, Y_f32, (uint16_t*)Y_bf16, stream),
+                stream);
 }
 
 }  // extern "C"

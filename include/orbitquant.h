@@ -76,6 +76,13 @@ OQ_API const char* oq_last_error(void);
  * synchronising `stream`.  Returns OQ_OK, OQ_ERR_TIMEOUT, or OQ_ERR_CUDA. */
 OQ_API int oq_get_device_status(void* stream);
 
+/* Synchronous checking, for debugging: when on, every launching entry point
+ * waits for its stream and returns the device status word itself (so a kernel
+ * that gave up is reported by the call that launched it, as OQ_ERR_TIMEOUT).
+ * Off by default; the environment variable OQ_DEBUG=1 turns it on at first
+ * use.  Not for use inside CUDA graph capture (it synchronises). */
+OQ_API int oq_set_debug(int on);
+
 /* Test hook for the failure path: the next launch of kernel 1 (rotate +
  * quantize, one-round rotations) or kernel 2 (codebook GEMM), on any stream,
  * issues none of its bulk / tensor copies.  Its bounded waits then run out

@@ -81,3 +81,36 @@ def test_gemm_wait_runs_out_and_context_survives(oq, codebooks):
     ref = olin.linear_from_codes(ca, an.cpu().double().numpy(), cw, r16, c, c, d)
     yy = y.double().cpu().numpy()
     assert np.linalg.norm(yy - ref) / np.linalg.norm(ref) <= 2e-3
+
+
+def test_debug_mode_reports_the_timeout_at_the_launching_call(oq):
+    # With synchronous checking on (oq_set_debug / OQ_DEBUG=1), the entry point
+    # that launched the kernel returns its give-up itself; normal calls in the
+    # same mode return OQ_OK with the same results as asynchronous calls.
+    d, M, N = 512, 300, 272
+    torch.manual_seed(7)
+    cb = oq.Codebook(d, 4)
+    a = torch.randint(0, 256, (M, d // 2), dtype=torch.uint8, device="cuda")
+    w = torch.randint(0, 256, (N, d // 2), dtype=torch.uint8, device="cuda")
+    an = torch.rand(M, device="cuda")
+    wn = torch.rand(N, device="cuda").to(torch.bfloat16)
+    ref, _ = oq.linear_codes(d, cb, cb, a, an, w, wn)
+    torch.cuda.synchronize()
+    oq.device_status()
+    lib = oq.lib()
+    assert lib.oq_set_debug(1) == oq.OQ_OK
+    try:
+        y, _ = oq.linear_codes(d, cb, cb, a, an, w, wn)
+        assert torch.equal(y, ref)
+        assert lib.oq_test_stall_next(2) == oq.OQ_OK
+        with pytest.raises(oq.OQError) as e:
+            oq.linear_codes(d, cb, cb, a, an, w, wn)
+        assert e.value.code == oq.OQ_ERR_TIMEOUT
+    finally:
+        lib.oq_test_stall_next(0)
+        lib.oq_set_debug(0)
+    oq.device_status()
+    y, _ = oq.linear_codes(d, cb, cb, a, an, w, wn)
+    torch.cuda.synchronize()
+    oq.device_status()
+    assert torch.equal(y, ref)

@@ -189,3 +189,9 @@ def test_stall_hook_arguments(oq):
     assert lib.oq_test_stall_next(-1) == oq.OQ_ERR_ARG
     assert lib.oq_test_stall_next(2) == oq.OQ_OK
     assert lib.oq_test_stall_next(0) == oq.OQ_OK  # disarmed again
+
+
+def test_debug_switch(oq):
+    lib = oq.lib()
+    assert lib.oq_set_debug(1) == oq.OQ_OK
+    assert lib.oq_set_debug(0) == oq.OQ_OK
