@@ -364,11 +364,18 @@ int codebook_device_qtable(oq_codebook_t cb, const uint32_t** qtable) {
   return OQ_OK;
 }
 
-// Shared-memory slot of coordinate c in the composed kernel's array of f32
-// pairs: thread c / 32 owns a run of 32 slots whose 2-slot chunks are rotated
-// by the thread index (chunk (c / 2) % 16 at position chunk ^ (thread % 16)).
-static uint16_t composed_slot(uint32_t c) {
-  const uint32_t g = c >> 5, ch = (c >> 1) & 15u;
+// Shared-memory slot of coordinate c in the composed kernel: thread c / 32
+// owns a run of 32 slots whose 16-byte chunks are rotated by the thread index.
+// Round 1 reads 4-byte bf16 pair words (chunk (c / 4) % 8 at position
+// chunk ^ (thread % 8)); later rounds 8-byte f32 pairs (chunk (c / 2) % 16 at
+// position chunk ^ (thread % 16)).
+static uint16_t composed_slot(uint32_t c, bool first_round) {
+  const uint32_t g = c >> 5;
+  if (first_round) {
+    const uint32_t ch = (c >> 2) & 7u;
+    return (uint16_t)((g << 5) | ((ch ^ (g & 7u)) << 2) | (c & 3u));
+  }
+  const uint32_t ch = (c >> 1) & 15u;
   return (uint16_t)((g << 5) | ((ch ^ (g & 15u)) << 1) | (c & 1u));
 }
 
@@ -383,7 +390,7 @@ int rpbh_composed_tables(oq_rpbh_t r, const uint16_t** slots, const uint32_t** s
     for (int k = 0; k < r->rounds; ++k) {
       const int32_t* perm = k == 0 ? r->perm.data() : r->perm_more.data() + (size_t)(k - 1) * d;
       const uint32_t* bits = k == 0 ? r->sign_bits.data() : r->sign_bits_more.data() + (size_t)(k - 1) * words;
-      for (int j = 0; j < d; ++j) sl[(size_t)k * d + j] = composed_slot((uint32_t)perm[j]);
+      for (int j = 0; j < d; ++j) sl[(size_t)k * d + j] = composed_slot((uint32_t)perm[j], k == 0);
       std::memcpy(sg.data() + (size_t)k * words, bits, sizeof(uint32_t) * words);
     }
     uint16_t* dsl = nullptr;

@@ -12,15 +12,17 @@
 // One CTA works on one row pair at a time (persistent over pairs); thread g
 // owns coordinates 32 g .. 32 g + 31 of both rows, the layout the butterflies
 // and the search of the one-round kernel use:
-//   * the pair is loaded from global memory (128-bit loads), widened to f32
-//     pairs and written to a shared array F of d 8-byte slots (row a, row b);
-//     a thread's 32 slots form a 256-byte run whose 16-byte chunks are rotated
+//   * the pair is loaded from global memory (128-bit loads) and written to a
+//     shared array of d 4-byte words, word j holding (x_a[j], x_b[j]) as bf16;
+//     a thread's 32 words form a 128-byte run whose 16-byte chunks are rotated
 //     by the thread index, so the 128-bit writes are free of bank conflicts;
-//   * each round gathers its input from F through a table of precomputed slot
-//     indices (the permutation composed with the chunk rotation), flips the
-//     signs of its Rademacher word, runs the unnormalised block transform in
-//     registers and, unless it is the last round, writes the result back to F
-//     between two CTA barriers;
+//   * round 1 gathers those words (one 32-bit load feeds both rows) and widens
+//     them to f32 while flipping its signs; later rounds gather f32 pairs from
+//     a shared array F of d 8-byte slots (256-byte runs, rotated the same
+//     way), which the previous round wrote between two CTA barriers; each
+//     round reads through a table of precomputed slot indices (the
+//     permutation composed with the chunk rotation) and runs the unnormalised
+//     block transform in registers;
 //   * the sum of squares comes from round 1's gathered input (the rotation is
 //     orthogonal); the k factors sqrt(h) of the unnormalised transforms are
 //     folded into the search multiplier.
@@ -40,7 +42,7 @@ struct ComposedArgs {
   uint8_t* codes;
   float* norm_f32;
   uint16_t* norm_bf16;
-  const uint16_t* slots;  // [rounds][d]: F slot that round r's coordinate j reads
+  const uint16_t* slots;  // [rounds][d]: slot that round r's coordinate j reads (round 1: 4-byte words)
   const uint32_t* signs;  // [rounds][d / 32]: sign words
   const uint32_t* qtable;
   int M, d, rounds, pairs, qtable_len;
@@ -90,19 +92,16 @@ __global__ void __launch_bounds__(512, 1) rotq_composed_kernel(const __grid_cons
       const uint4* ra = reinterpret_cast<const uint4*>(reinterpret_cast<const unsigned char*>(a.X) + row * rowb) +
                         4 * tid;
       const uint4* rb = ra + rowb / 16;
-      unsigned long long v[32];
+      const uint32_t run1 = fbase + 128u * (uint32_t)tid, rot1 = (uint32_t)tid & 7u;
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
+      for (int q = 0; q < 4; ++q) {  // 8 columns -> two 16-byte chunks of pair words
         const uint4 A = ra[q];
         const uint4 B = has_b ? rb[q] : make_uint4(0u, 0u, 0u, 0u);
-        const uint32_t wa[4] = {A.x, A.y, A.z, A.w}, wb[4] = {B.x, B.y, B.z, B.w};
-#pragma unroll
-        for (int m = 0; m < 4; ++m) {
-          v[8 * q + 2 * m] = u2_pack(wa[m] << 16, wb[m] << 16);
-          v[8 * q + 2 * m + 1] = u2_pack(wa[m] & 0xFFFF0000u, wb[m] & 0xFFFF0000u);
-        }
+        sts_u128(run1 + ((((uint32_t)(2 * q)) ^ rot1) << 4), __byte_perm(A.x, B.x, 0x5410), __byte_perm(A.x, B.x, 0x7632),
+                 __byte_perm(A.y, B.y, 0x5410), __byte_perm(A.y, B.y, 0x7632));
+        sts_u128(run1 + ((((uint32_t)(2 * q + 1)) ^ rot1) << 4), __byte_perm(A.z, B.z, 0x5410),
+                 __byte_perm(A.z, B.z, 0x7632), __byte_perm(A.w, B.w, 0x5410), __byte_perm(A.w, B.w, 0x7632));
       }
-      store_run(run, rot, v);
     }
     __syncthreads();
 
@@ -120,10 +119,15 @@ __global__ void __launch_bounds__(512, 1) rotq_composed_kernel(const __grid_cons
           for (int m = 0; m < 8; ++m) {
             const int i = 8 * q + m;
             const uint32_t slot = (s4[m >> 1] >> (16 * (m & 1))) & 0xFFFFu;
-            uint32_t lo, hi;
-            u2_unpack(lds_u64(fbase + 8u * slot), lo, hi);
             const uint32_t flip = (sw << (31 - i)) & 0x80000000u;  // sign of coordinate i
-            v[i] = u2_pack(lo ^ flip, hi ^ flip);
+            if (r == 0) {  // bf16 pair word (row a low, row b high)
+              const uint32_t w = lds_u32(fbase + 4u * slot);
+              v[i] = u2_pack((w << 16) ^ flip, (w & 0xFFFF0000u) ^ flip);
+            } else {
+              uint32_t lo, hi;
+              u2_unpack(lds_u64(fbase + 8u * slot), lo, hi);
+              v[i] = u2_pack(lo ^ flip, hi ^ flip);
+            }
           }
         }
       } else {
@@ -250,7 +254,7 @@ int launch_rotq_composed(oq_rpbh_t r, oq_codebook_t cb, const void* X, int M, ui
   a.rounds = r->rounds;
   a.pairs = (M + 1) / 2;
   a.qtable_len = qlen;
-  a.qt_off = (uint32_t)threads * 256u;  // F: one 256-byte run per thread (inactive runs unused)
+  a.qt_off = (uint32_t)threads * 256u;  // F: one 256-byte run per thread (round 1 uses the first half)
   a.part_off = (a.qt_off + 4u * (uint32_t)qlen + 15u) & ~15u;
   a.alpha = (float)((double)cb->qt_alpha / std::pow((double)h, 0.5 * r->rounds));
   a.nb = (float)cb->qt_nb;
