@@ -69,6 +69,33 @@ __device__ __forceinline__ void store_run(uint32_t run, uint32_t rot, const unsi
   }
 }
 
+// One round's gather of this thread's 32 coordinates with its signs applied:
+// round 1 (FIRST) from bf16 pair words (row a low, row b high), later rounds
+// from f32 pairs.  sl: the thread's 32 slot indices, sw: its sign word.
+template <bool FIRST>
+__device__ __forceinline__ void gather_round(unsigned long long (&v)[32], const uint4* sl, uint32_t sw,
+                                             uint32_t fbase) {
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const uint4 S = sl[q];
+    const uint32_t s4[4] = {S.x, S.y, S.z, S.w};
+#pragma unroll
+    for (int m = 0; m < 8; ++m) {
+      const int i = 8 * q + m;
+      const uint32_t slot = (s4[m >> 1] >> (16 * (m & 1))) & 0xFFFFu;
+      const uint32_t flip = (sw << (31 - i)) & 0x80000000u;  // sign of coordinate i
+      if constexpr (FIRST) {
+        const uint32_t w = lds_u32(fbase + 4u * slot);
+        v[i] = u2_pack((w << 16) ^ flip, (w & 0xFFFF0000u) ^ flip);
+      } else {
+        uint32_t lo, hi;
+        u2_unpack(lds_u64(fbase + 8u * slot), lo, hi);
+        v[i] = u2_pack(lo ^ flip, hi ^ flip);
+      }
+    }
+  }
+}
+
 template <int BITS, int LOGHB>
 __global__ void __launch_bounds__(512, 1) rotq_composed_kernel(const __grid_constant__ ComposedArgs a) {
   extern __shared__ __align__(1024) unsigned char smem[];
@@ -111,25 +138,10 @@ __global__ void __launch_bounds__(512, 1) rotq_composed_kernel(const __grid_cons
       if (active) {
         const uint4* sl = reinterpret_cast<const uint4*>(a.slots + (size_t)r * a.d) + 4 * tid;
         const uint32_t sw = a.signs[(size_t)r * T + tid];
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const uint4 S = sl[q];
-          const uint32_t s4[4] = {S.x, S.y, S.z, S.w};
-#pragma unroll
-          for (int m = 0; m < 8; ++m) {
-            const int i = 8 * q + m;
-            const uint32_t slot = (s4[m >> 1] >> (16 * (m & 1))) & 0xFFFFu;
-            const uint32_t flip = (sw << (31 - i)) & 0x80000000u;  // sign of coordinate i
-            if (r == 0) {  // bf16 pair word (row a low, row b high)
-              const uint32_t w = lds_u32(fbase + 4u * slot);
-              v[i] = u2_pack((w << 16) ^ flip, (w & 0xFFFF0000u) ^ flip);
-            } else {
-              uint32_t lo, hi;
-              u2_unpack(lds_u64(fbase + 8u * slot), lo, hi);
-              v[i] = u2_pack(lo ^ flip, hi ^ flip);
-            }
-          }
-        }
+        if (r == 0)
+          gather_round<true>(v, sl, sw, fbase);
+        else
+          gather_round<false>(v, sl, sw, fbase);
       } else {
 #pragma unroll
         for (int i = 0; i < 32; ++i) v[i] = 0ull;
