@@ -166,3 +166,64 @@ def test_gelu_erf_values():
     x = np.linspace(-4, 4, 17)
     assert np.allclose(olin.gelu_erf(x) - olin.gelu_erf(-x), x, atol=1e-15)
     assert abs(olin.gelu_erf(np.array([1.0]))[0] - 0.8413447460685429) < 1e-15
+
+
+# ---- boundary_distance: decides which code mismatches fall inside the 1e-5 band ----
+# The parity rule forgives a code difference only when t lies within 1e-5 of a
+# decision boundary beta_k (the midpoints between consecutive centroids that
+# define q_hat, OrbitQuant "Theoretical Basis").  These pins fix the distance
+# itself: hand-computed values, then brute force against every boundary.
+
+def test_boundary_distance_hand_values():
+    b = np.array([-0.5, 0.0, 0.25])
+    t = np.array([0.0, -0.5, 0.25,      # exactly on a boundary
+                  -1.0, -0.75,          # below the first boundary
+                  1.0, 0.5,             # above the last boundary
+                  0.125, -0.25,         # midway between two boundaries
+                  0.2, -0.1, 0.05])     # nearer one neighbour than the other
+    want = [0.0, 0.0, 0.0,
+            0.5, 0.25,
+            0.75, 0.25,
+            0.125, 0.25,
+            0.05, 0.1, 0.05]
+    got = oq.boundary_distance(t, b)
+    assert np.allclose(got, want, rtol=0, atol=1e-15)
+    # the boundaries' order must not matter
+    assert np.array_equal(oq.boundary_distance(t, b[[2, 0, 1]]), got)
+    # shape is kept (a rows x columns matrix of t)
+    assert oq.boundary_distance(t.reshape(3, 4), b).shape == (3, 4)
+
+
+def test_boundary_distance_single_boundary():
+    # 1-bit codebook: one boundary at 0, distance is |t|
+    t = np.array([-3.0, -1e-7, 0.0, 2e-9, 5.0])
+    assert np.array_equal(oq.boundary_distance(t, np.array([0.0])), np.abs(t))
+
+
+@pytest.mark.parametrize("bits", [1, 2, 3, 4, 5, 6])
+def test_boundary_distance_equals_brute_force(bits, codebooks):
+    d = 256
+    beta = codebooks(d, bits)["boundaries"]
+    rng = np.random.default_rng(100 + bits)
+    # t spread over and beyond the boundaries' range, plus the boundaries
+    # themselves and points a hair either side of them
+    t = np.concatenate([rng.uniform(-1.0, 1.0, 50000),
+                        rng.standard_normal(50000) / math.sqrt(d),
+                        beta, np.nextafter(beta, 2.0), np.nextafter(beta, -2.0)])
+    brute = np.min(np.abs(t[:, None] - beta[None, :]), axis=1)
+    shuffled = beta[rng.permutation(len(beta))]
+    assert np.array_equal(oq.boundary_distance(t, beta), brute)
+    assert np.array_equal(oq.boundary_distance(t, shuffled), brute)
+    assert np.all(oq.boundary_distance(beta, beta) == 0.0)
+
+
+def test_band_rule_flags_exactly_the_near_ties(codebooks):
+    # the parity tests forgive a mismatch where boundary_distance < 1e-5: put
+    # points at known offsets from each boundary and check which are flagged
+    beta = codebooks(3072, 4)["boundaries"]
+    offs = np.array([0.0, 3e-6, -9.9e-6, 1.01e-5, -2e-5, 1e-3])
+    t = (beta[:, None] + offs[None, :]).reshape(-1)
+    near = oq.boundary_distance(t, beta) < 1e-5
+    spacing = np.min(np.diff(beta))
+    assert spacing > 2e-3                      # each point's nearest boundary is its own
+    assert near.reshape(len(beta), -1).tolist() == [[True, True, True, False, False, False]] * len(beta)
