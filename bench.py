@@ -185,6 +185,43 @@ def oracle_sample(rows, W_state=None):
     return dt, W_state
 
 
+def parity_report(oq, cb, bufs, w_norm, W_state, K, bias):
+    """Parity of one bench set's outputs against the oracle on sampled rows.
+
+    Codes: the kernel's codes of the sampled rows against the oracle's
+    nearest-centroid codes; mismatches are counted with the entries whose t lies
+    within 1e-5 of a decision boundary (the band the parity rule forgives).
+    Norms: max relative error of s.  Linear: relative Frobenius error of the
+    GEMM's fp32 output (one extra launch on the same codes) and of the bench's
+    bf16 output against the oracle's fp64 layer on its own codes."""
+    import torch
+    from calibration_free_rotated_b200 import inputs
+    from oracle import linear as olin
+    from oracle import quantize as oqz
+    w = WORKLOAD
+    M, h = w["M"], w["block"]
+    rows = np.unique(np.concatenate([np.linspace(0, M - 1, 64).astype(int), [M - 1]]))
+    st = W_state
+    X = inputs.bf16_bits_to_f64(inputs.activations(2, M, K)[rows])
+    ca, s, T = oqz.quantize_rows(X, st["perm"], st["signs"], h, st["cb"]["centroids"])
+    got = oqz.unpack_codes(bufs["codes"].cpu().numpy()[rows], 4, K)
+    mism = got != ca
+    band = oqz.boundary_distance(T, st["cb"]["boundaries"]) < 1e-5
+    s_gpu = bufs["norms"].cpu().numpy()[rows].astype(np.float64)
+    ref = olin.linear_from_codes(ca, s, st["cw"], st["r16"], st["cb"]["centroids"], st["cb"]["centroids"], K,
+                                 bias=st["bias"])
+    y32, _ = oq.linear_codes(K, cb, cb, bufs["codes"], bufs["norms"], bufs["wc"], w_norm, bias=bias)
+    torch.cuda.synchronize()
+    y32 = y32.double().cpu().numpy()[rows]
+    y16 = bufs["Y"].double().cpu().numpy()[rows]
+    rel = lambda y: float(np.linalg.norm(y - ref) / np.linalg.norm(ref))
+    return {"rows_sampled": int(len(rows)), "codes_checked": int(mism.size), "code_mismatches": int(mism.sum()),
+            "in_band": int(band.sum()), "mismatches_outside_band": int((mism & ~band).sum()), "band": 1e-5,
+            "norm_max_rel": float(np.max(np.abs(s_gpu - s) / np.maximum(s, 1e-300))),
+            "rel_fro_f32": rel(y32), "rel_fro_bf16_out": rel(y16), "tol": 2e-3,
+            "weights": "oracle-quantized weights for the reference; the GPU's own weight codes for the GEMM"}
+
+
 def cpu_threads():
     try:
         from threadpoolctl import threadpool_info
@@ -380,9 +417,17 @@ def run_ours(args, world, rank, local):
         "gpu_launches": 2 * args.steps,
         "clocks": clk.summary(),
     }
+    st = None
+    if rank == 0 and not args.no_parity:
+        # parity of this run's own outputs, outside the timed region: sampled
+        # rows of set 0 (codes, norms and Y from the timed steps) against the
+        # oracle, with the boundary ties counted
+        _, st = oracle_sample(8)
+        line["parity"] = parity_report(oq, cb, sets[0], wn, st, K, bias)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         rows = 2048
-        _, st = oracle_sample(8)
+        if st is None:
+            _, st = oracle_sample(8)
         dt, _ = oracle_sample(rows, st)
         _, sflops = algorithmic(rows, K, N, 4, 4)
         line["cpu_baseline"] = {"value": sflops / dt / 1e12, "unit": UNIT, "cores": cpu_threads(), "kind": "oracle",
@@ -674,6 +719,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-parity", action="store_true", help="skip the sampled-row parity check of the bench line")
     ap.add_argument("--profile", choices=["rotq", "gemm"], help="launch one kernel only (for ncu captures)")
     ap.add_argument("--ablation", choices=["rotation"], help="time the rotation variants of the ablation table")
     ap.add_argument("--workload", choices=["flux_mlp", "wan_ffn", "flux_qkv_w3a3"],

@@ -1086,34 +1086,37 @@ int get_encode_fn(EncodeTiledFn* fn) {
   return OQ_OK;
 }
 
-// 2-D map over packed codes: [rows][row_bytes] uint8, box = (64 codes, box_rows).
-int make_code_map(CUtensorMap* map, const void* base, int rows, int row_bytes, int box_bytes, int box_rows) {
+// Encodes a 2-D map from its cache key (no interleave, unit element strides).
+int encode_2d(const TmapKey& k, void* out) {
   EncodeTiledFn enc;
   if (int rc = get_encode_fn(&enc)) return rc;
-  cuuint64_t dims[2] = {(cuuint64_t)row_bytes, (cuuint64_t)rows};
-  cuuint64_t strides[1] = {(cuuint64_t)row_bytes};
-  cuuint32_t box[2] = {(cuuint32_t)box_bytes, (cuuint32_t)box_rows};
+  cuuint64_t dims[2] = {(cuuint64_t)k.dim0, (cuuint64_t)k.dim1};
+  cuuint64_t strides[1] = {(cuuint64_t)k.stride1};
+  cuuint32_t box[2] = {(cuuint32_t)k.box0, (cuuint32_t)k.box1};
   cuuint32_t estr[2] = {1, 1};
-  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
-                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
-                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  CUresult r = enc(static_cast<CUtensorMap*>(out), (CUtensorMapDataType)k.type, 2, const_cast<void*>(k.base), dims,
+                   strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, (CUtensorMapSwizzle)k.swizzle,
+                   (CUtensorMapL2promotion)k.promo, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return fail(OQ_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
   return OQ_OK;
+}
+
+// 2-D map over packed codes: [rows][row_bytes] uint8, box = (64 codes, box_rows).
+int make_code_map(CUtensorMap* map, const void* base, int rows, int row_bytes, int box_bytes, int box_rows) {
+  static_assert(sizeof(CUtensorMap) == 128, "tensor map size");
+  TmapKey k{base, (unsigned long long)row_bytes, (unsigned long long)rows, (unsigned long long)row_bytes,
+            (unsigned)box_bytes, (unsigned)box_rows, (int)CU_TENSOR_MAP_DATA_TYPE_UINT8,
+            (int)CU_TENSOR_MAP_SWIZZLE_NONE, (int)CU_TENSOR_MAP_L2_PROMOTION_L2_128B};
+  return cached_tensor_map(k, map, encode_2d);
 }
 
 // Row-major M x N output, written in 128-row boxes of 128 bytes with the
 // 128-byte swizzle that the epilogue's staging layout uses.
 int make_out_map(CUtensorMap* map, void* base, int M, int N, CUtensorMapDataType type, int esize) {
-  EncodeTiledFn enc;
-  if (int rc = get_encode_fn(&enc)) return rc;
-  cuuint64_t dims[2] = {(cuuint64_t)N, (cuuint64_t)M};
-  cuuint64_t strides[1] = {(cuuint64_t)N * (cuuint64_t)esize};
-  cuuint32_t box[2] = {(cuuint32_t)(128 / esize), 128u};
-  cuuint32_t estr[2] = {1, 1};
-  CUresult r = enc(map, type, 2, base, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                   CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  if (r != CUDA_SUCCESS) return fail(OQ_ERR_CUDA, "cuTensorMapEncodeTiled (output) failed (%d)", (int)r);
-  return OQ_OK;
+  TmapKey k{base, (unsigned long long)N, (unsigned long long)M, (unsigned long long)N * (unsigned long long)esize,
+            (unsigned)(128 / esize), 128u, (int)type, (int)CU_TENSOR_MAP_SWIZZLE_128B,
+            (int)CU_TENSOR_MAP_L2_PROMOTION_NONE};
+  return cached_tensor_map(k, map, encode_2d);
 }
 
 using GemmKernel = void (*)(GemmArgs, CUtensorMap, CUtensorMap, CUtensorMap, CUtensorMap);
@@ -1135,8 +1138,6 @@ int launch_t(GemmArgs& a, const uint8_t* a_codes, const uint8_t* w_codes, int ns
     if (int rc = make_out_map(&my32, a.y32, a.M, a.N, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4)) return rc;
   GemmKernel k = cbgemm_kernel<BA, BW, PAIR>;
   const int smem = S::kAlloc;
-  cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-  if (e != cudaSuccess) return fail(OQ_ERR_CUDA, "cudaFuncSetAttribute(GEMM): %s", cudaGetErrorString(e));
   const int tile_m = PAIR ? 2 * BM : BM;
   a.tiles_m = (a.M + tile_m - 1) / tile_m;
   a.num_tiles = a.tiles_m * ((a.N + BN - 1) / BN);
@@ -1154,17 +1155,18 @@ int launch_t(GemmArgs& a, const uint8_t* a_codes, const uint8_t* w_codes, int ns
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    cfg.gridDim = dim3(2 * std::min(a.num_tiles, nsm / 2), 1, 1);
     int max_clusters = 0;
-    e = cudaOccupancyMaxActiveClusters(&max_clusters, k, &cfg);
-    if (e != cudaSuccess) return fail(OQ_ERR_CUDA, "cluster occupancy query: %s", cudaGetErrorString(e));
+    if (int rc = occupancy(reinterpret_cast<const void*>(k), smem, NUM_THREADS, 2, &max_clusters)) return rc;
     if (max_clusters < 1) return fail(OQ_ERR_UNSUPPORTED, "no CTA pair of the GEMM fits on this device");
     units = std::min(std::min(a.num_tiles, max_clusters), nsm / 2);  // one CTA per SM
     cfg.gridDim = dim3(2 * units, 1, 1);
   } else {
+    int per_sm = 0;
+    if (int rc = occupancy(reinterpret_cast<const void*>(k), smem, NUM_THREADS, 0, &per_sm)) return rc;
+    if (per_sm < 1) return fail(OQ_ERR_UNSUPPORTED, "the GEMM's CTA does not fit on this device");
     cfg.gridDim = dim3(units, 1, 1);
   }
-  e = cudaLaunchKernelEx(&cfg, k, a, ma, mb, my16, my32);
+  cudaError_t e = cudaLaunchKernelEx(&cfg, k, a, ma, mb, my16, my32);
   if (e != cudaSuccess) return fail(OQ_ERR_CUDA, "GEMM launch: %s", cudaGetErrorString(e));
   return OQ_OK;
 }

@@ -275,6 +275,16 @@ void build_qtable(oq_codebook_t cb) {
 // ---------------------------------------------------------------------------
 // Device state
 // ---------------------------------------------------------------------------
+static std::atomic<long long> g_dev_allocs{0};
+
+// Every device allocation of the library goes through here, so that
+// oq_device_allocations() can report how many there have been.
+static cudaError_t dev_malloc(void** p, size_t bytes) {
+  cudaError_t e = cudaMalloc(p, bytes);
+  if (e == cudaSuccess) g_dev_allocs.fetch_add(1, std::memory_order_relaxed);
+  return e;
+}
+
 static std::mutex g_dev_mu;
 static int* g_status[OQ_MAX_DEVICES] = {};
 static int g_sms[OQ_MAX_DEVICES] = {};
@@ -292,7 +302,7 @@ int device_status_word(int** status) {
   std::lock_guard<std::mutex> lk(g_dev_mu);
   if (!g_status[dev]) {
     int* p = nullptr;
-    cudaError_t e = cudaMalloc(&p, sizeof(int));
+    cudaError_t e = dev_malloc(reinterpret_cast<void**>(&p), sizeof(int));
     if (e != cudaSuccess) return fail(OQ_ERR_CUDA, "cudaMalloc(status): %s", cudaGetErrorString(e));
     e = cudaMemset(p, 0, sizeof(int));
     if (e != cudaSuccess) return fail(OQ_ERR_CUDA, "cudaMemset(status): %s", cudaGetErrorString(e));
@@ -325,13 +335,98 @@ int sm_count(int* n) {
   return OQ_OK;
 }
 
+namespace {
+struct OccEntry {
+  const void* fn;
+  int dev, smem, threads, cluster, value;
+};
+std::mutex g_occ_mu;
+std::vector<OccEntry> g_occ;
+std::vector<std::pair<const void*, int>> g_smem_raised;  // (kernel, device)
+
+struct TmapEntry {
+  TmapKey key;
+  int dev;
+  alignas(64) unsigned char map[128];
+};
+constexpr int kTmapSlots = 64;
+std::mutex g_tmap_mu;
+TmapEntry g_tmap[kTmapSlots];
+int g_tmap_used = 0, g_tmap_next = 0;
+}  // namespace
+
+int occupancy(const void* kernel, int smem, int threads, int cluster, int* value) {
+  int dev;
+  if (int rc = current_device(&dev)) return rc;
+  std::lock_guard<std::mutex> lk(g_occ_mu);
+  for (const OccEntry& e : g_occ)
+    if (e.fn == kernel && e.dev == dev && e.smem == smem && e.threads == threads && e.cluster == cluster) {
+      *value = e.value;
+      return OQ_OK;
+    }
+  bool raised = false;
+  for (const auto& p : g_smem_raised) raised |= p.first == kernel && p.second == dev;
+  if (!raised) {
+    int optin = 0;
+    cudaFuncAttributes fa;
+    cudaError_t e = cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+    if (e == cudaSuccess) e = cudaFuncGetAttributes(&fa, kernel);
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, optin - (int)fa.sharedSizeBytes);
+    if (e != cudaSuccess) return fail(OQ_ERR_CUDA, "raising the shared-memory limit: %s", cudaGetErrorString(e));
+    g_smem_raised.emplace_back(kernel, dev);
+  }
+  int v = 0;
+  cudaError_t e;
+  if (cluster == 0) {
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&v, kernel, threads, (size_t)smem);
+  } else {
+    cudaLaunchConfig_t cfg;
+    std::memset(&cfg, 0, sizeof(cfg));
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = (unsigned)cluster;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cfg.blockDim = dim3((unsigned)threads, 1, 1);
+    cfg.gridDim = dim3((unsigned)cluster, 1, 1);
+    cfg.dynamicSmemBytes = (size_t)smem;
+    e = cudaOccupancyMaxActiveClusters(&v, kernel, &cfg);
+  }
+  if (e != cudaSuccess) return fail(OQ_ERR_CUDA, "occupancy query: %s", cudaGetErrorString(e));
+  g_occ.push_back(OccEntry{kernel, dev, smem, threads, cluster, v});
+  *value = v;
+  return OQ_OK;
+}
+
+int cached_tensor_map(const TmapKey& key, void* map128, int (*encode)(const TmapKey&, void*)) {
+  int dev;
+  if (int rc = current_device(&dev)) return rc;
+  std::lock_guard<std::mutex> lk(g_tmap_mu);
+  for (int i = 0; i < g_tmap_used; ++i)
+    if (g_tmap[i].dev == dev && g_tmap[i].key == key) {
+      std::memcpy(map128, g_tmap[i].map, 128);
+      return OQ_OK;
+    }
+  if (int rc = encode(key, map128)) return rc;
+  TmapEntry& slot = g_tmap[g_tmap_next];  // round-robin replacement
+  slot.key = key;
+  slot.dev = dev;
+  std::memcpy(slot.map, map128, 128);
+  g_tmap_next = (g_tmap_next + 1) % kTmapSlots;
+  if (g_tmap_used < kTmapSlots) ++g_tmap_used;
+  return OQ_OK;
+}
+
 static int upload_rpbh(oq_rpbh_t r, int dev) {
   std::vector<uint16_t> p16(r->d);
   for (int j = 0; j < r->d; ++j) p16[j] = (uint16_t)r->perm[j];
   uint16_t* dp = nullptr;
   uint32_t* ds = nullptr;
-  cudaError_t e = cudaMalloc(&dp, sizeof(uint16_t) * r->d);
-  if (e == cudaSuccess) e = cudaMalloc(&ds, sizeof(uint32_t) * r->sign_bits.size());
+  cudaError_t e = dev_malloc(reinterpret_cast<void**>(&dp), sizeof(uint16_t) * r->d);
+  if (e == cudaSuccess) e = dev_malloc(reinterpret_cast<void**>(&ds), sizeof(uint32_t) * r->sign_bits.size());
   if (e == cudaSuccess) e = cudaMemcpy(dp, p16.data(), sizeof(uint16_t) * r->d, cudaMemcpyHostToDevice);
   if (e == cudaSuccess)
     e = cudaMemcpy(ds, r->sign_bits.data(), sizeof(uint32_t) * r->sign_bits.size(), cudaMemcpyHostToDevice);
@@ -352,7 +447,7 @@ int codebook_device_qtable(oq_codebook_t cb, const uint32_t** qtable) {
   if (!cb->dev_qtable[dev]) {
     uint32_t* p = nullptr;
     const size_t bytes = sizeof(uint32_t) * cb->qtable.size();
-    cudaError_t e = cudaMalloc(&p, bytes);
+    cudaError_t e = dev_malloc(reinterpret_cast<void**>(&p), bytes);
     if (e == cudaSuccess) e = cudaMemcpy(p, cb->qtable.data(), bytes, cudaMemcpyHostToDevice);
     if (e != cudaSuccess) {
       cudaFree(p);
@@ -395,8 +490,8 @@ int rpbh_composed_tables(oq_rpbh_t r, const uint16_t** slots, const uint32_t** s
     }
     uint16_t* dsl = nullptr;
     uint32_t* dsg = nullptr;
-    cudaError_t e = cudaMalloc(&dsl, sizeof(uint16_t) * sl.size());
-    if (e == cudaSuccess) e = cudaMalloc(&dsg, sizeof(uint32_t) * sg.size());
+    cudaError_t e = dev_malloc(reinterpret_cast<void**>(&dsl), sizeof(uint16_t) * sl.size());
+    if (e == cudaSuccess) e = dev_malloc(reinterpret_cast<void**>(&dsg), sizeof(uint32_t) * sg.size());
     if (e == cudaSuccess) e = cudaMemcpy(dsl, sl.data(), sizeof(uint16_t) * sl.size(), cudaMemcpyHostToDevice);
     if (e == cudaSuccess) e = cudaMemcpy(dsg, sg.data(), sizeof(uint32_t) * sg.size(), cudaMemcpyHostToDevice);
     if (e != cudaSuccess) {
@@ -410,6 +505,16 @@ int rpbh_composed_tables(oq_rpbh_t r, const uint16_t** slots, const uint32_t** s
   *slots = r->dev_slots[dev];
   *signs = r->dev_csigns[dev];
   return OQ_OK;
+}
+
+int rpbh_tables_if_present(oq_rpbh_t r, int dev) {
+  std::lock_guard<std::mutex> lk(r->mu);
+  return r->dev_perm[dev] && (r->rounds == 1 || r->dev_slots[dev]) ? OQ_OK : OQ_ERR_ARG;
+}
+
+int codebook_qtable_if_present(oq_codebook_t cb, int dev) {
+  std::lock_guard<std::mutex> lk(cb->mu);
+  return cb->dev_qtable[dev] ? OQ_OK : OQ_ERR_ARG;
 }
 
 int rpbh_device_tables(oq_rpbh_t r, const uint16_t** perm, const uint32_t** signs) {
@@ -468,7 +573,10 @@ static int make_rotation(uint64_t seed, int d, int block, int kind, int rounds, 
   int h = block == 0 ? (d & -d) : block;
   if (h < 1 || (h & (h - 1)) != 0 || d % h != 0)
     return fail(OQ_ERR_ARG, "block %d must be a power of two dividing d=%d", block, d);
-  if (rounds > 1 && d > 65536) return fail(OQ_ERR_ARG, "composed rotations need d <= 65536 (got %d)", d);
+  // the composed kernel's limits, checked here so that no handle is made (and
+  // uploaded) that no kernel can run
+  if (rounds > 1 && (h < 32 || d % 32 != 0 || d > 16384))
+    return fail(OQ_ERR_UNSUPPORTED, "composed rotation kernel: d=%d h=%d (needs h >= 32, d <= 16384)", d, h);
   oq_rpbh_t r = new (std::nothrow) oq_rpbh_s;
   if (!r) return fail(OQ_ERR_NOMEM, "allocating the RPBH handle");
   r->seed = seed;
@@ -523,6 +631,8 @@ using namespace oq;
 extern "C" {
 
 int oq_version(void) { return OQ_VERSION; }
+
+long long oq_device_allocations(void) { return g_dev_allocs.load(std::memory_order_relaxed); }
 
 // Synchronous checking (OQ_DEBUG=1 in the environment, or oq_set_debug): each
 // launching entry point then waits for its stream and returns the device status

@@ -63,10 +63,38 @@ int codebook_device_qtable(oq_codebook_t cb, const uint32_t** qtable);
 void build_qtable(oq_codebook_t cb);
 int device_status_word(int** status);
 int device_status_word_if_present(int** status);  // never allocates
+// OQ_OK when the handle's tables exist on device `dev`, else OQ_ERR_ARG (no
+// message); they take the handle's lock and never allocate.
+int rpbh_tables_if_present(oq_rpbh_t r, int dev);
+int codebook_qtable_if_present(oq_codebook_t cb, int dev);
 int sm_count(int* n);
 bool aligned16(const void* p);
 // Test hook (oq_test_stall_next): 1 exactly once, for the next launch of `kernel`.
 int take_test_stall(int kernel);
+
+// Launch preparation cached per device (oq_host.cpp).  On the first use of a
+// kernel on a device its dynamic shared-memory limit is raised to the device's
+// opt-in maximum; `occupancy` then returns the kernel's resident CTAs per SM
+// (cluster == 0) or its resident clusters of `cluster` CTAs per device, queried
+// once per (kernel, dynamic shared memory, block size, cluster) and device.
+// Steady-state launches therefore make no attribute or occupancy calls.
+int occupancy(const void* kernel, int smem, int threads, int cluster, int* value);
+
+// Encoded 2-D tensor maps cached by everything that defines them (base
+// address, sizes, strides, box, element type, swizzle, promotion); a launch on
+// the same buffers reuses the encoding instead of re-encoding.  `encode`
+// fills the map on a miss and returns OQ_OK or an error code.
+struct TmapKey {
+  const void* base;
+  unsigned long long dim0, dim1, stride1;
+  unsigned box0, box1;
+  int type, swizzle, promo;
+  bool operator==(const TmapKey& o) const {
+    return base == o.base && dim0 == o.dim0 && dim1 == o.dim1 && stride1 == o.stride1 && box0 == o.box0 &&
+           box1 == o.box1 && type == o.type && swizzle == o.swizzle && promo == o.promo;
+  }
+};
+int cached_tensor_map(const TmapKey& key, void* map128, int (*encode)(const TmapKey&, void*));
 
 // Kernel launchers.
 int launch_rotq(oq_rpbh_t r, oq_codebook_t cb, const void* X, int M, uint8_t* codes, float* norm_f32,

@@ -58,10 +58,10 @@ extern "C" int oq_linear_noalloc(oq_rpbh_t r, oq_codebook_t cb_a, oq_codebook_t 
   // handle was created with this device current) and the status word (made
   // by the first kernel launch of any other entry point, or by
   // oq_get_device_status).
-  if (!r->dev_perm[dev] || (r->rounds > 1 && !r->dev_slots[dev]))
+  if (oq::rpbh_tables_if_present(r, dev) != OQ_OK)
     return oq::fail(OQ_ERR_ARG, "the RPBH handle has no tables on device %d: create it with that device current",
                     dev);
-  if (!cb_a->dev_qtable[dev])
+  if (oq::codebook_qtable_if_present(cb_a, dev) != OQ_OK)
     return oq::fail(OQ_ERR_ARG,
                     "the activation codebook has no tables on device %d: build it with that device current", dev);
   int* status = nullptr;

@@ -139,15 +139,13 @@ int launch_rotq(oq_rpbh_t r, oq_codebook_t cb, const void* X, int M, uint8_t* co
   a.nb = (float)cb->qt_nb;
   a.stall = take_test_stall(1);
 
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)p.smem);
-  if (e != cudaSuccess) return fail(OQ_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(e));
   int per_sm = 0;
-  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, p.threads, p.smem);
-  if (e != cudaSuccess) return fail(OQ_ERR_CUDA, "occupancy query: %s", cudaGetErrorString(e));
+  if (int rc = occupancy(reinterpret_cast<const void*>(kern), (int)p.smem, p.threads, 0, &per_sm)) return rc;
   if (per_sm < 1) return fail(OQ_ERR_UNSUPPORTED, "rotate+quantize kernel does not fit (d=%d)", d);
+  if (a.groups == 0) return OQ_OK;
   const int grid = std::min(a.groups, nsm * per_sm);
   kern<<<grid, p.threads, p.smem, (cudaStream_t)stream>>>(a);
-  e = cudaGetLastError();
+  cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return fail(OQ_ERR_CUDA, "rotate+quantize launch: %s", cudaGetErrorString(e));
   return OQ_OK;
 }

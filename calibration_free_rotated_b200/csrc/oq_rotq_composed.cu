@@ -272,15 +272,12 @@ int launch_rotq_composed(oq_rpbh_t r, oq_codebook_t cb, const void* X, int M, ui
   a.nb = (float)cb->qt_nb;
   const size_t smem = a.part_off + (size_t)(threads / 32) * 8;
 
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-  if (e != cudaSuccess) return fail(OQ_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(e));
   int per_sm = 0;
-  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, threads, smem);
-  if (e != cudaSuccess) return fail(OQ_ERR_CUDA, "occupancy query: %s", cudaGetErrorString(e));
+  if (int rc = occupancy(reinterpret_cast<const void*>(kern), (int)smem, threads, 0, &per_sm)) return rc;
   if (per_sm < 1) return fail(OQ_ERR_UNSUPPORTED, "composed rotate+quantize kernel does not fit (d=%d)", d);
   const int grid = std::min(a.pairs, nsm * per_sm);
   kern<<<grid, threads, smem, (cudaStream_t)stream>>>(a);
-  e = cudaGetLastError();
+  cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return fail(OQ_ERR_CUDA, "composed rotate+quantize launch: %s", cudaGetErrorString(e));
   return OQ_OK;
 }

@@ -28,6 +28,7 @@ _lib = ctypes.CDLL(LIB_PATH)
 _c_int, _c_void_p, _c_size_t = ctypes.c_int, ctypes.c_void_p, ctypes.c_size_t
 _SIGS = {
     "oq_version": (_c_int, []),
+    "oq_device_allocations": (ctypes.c_longlong, []),
     "oq_last_error": (ctypes.c_char_p, []),
     "oq_get_device_status": (_c_int, [_c_void_p]),
     "oq_make_rpbh": (_c_int, [ctypes.c_uint64, _c_int, _c_int, ctypes.POINTER(_c_void_p)]),
@@ -230,6 +231,11 @@ def linear(rpbh: Rpbh, cb_a: Codebook, cb_w: Codebook, X, w_codes, w_norm, bias=
 def device_status(stream=None):
     """Raises OQError if a kernel's bounded wait gave up since the last call."""
     _check(_lib.oq_get_device_status(_stream(stream)))
+
+
+def device_allocations() -> int:
+    """How many device allocations the library has made in this process."""
+    return int(_lib.oq_device_allocations())
 
 
 def linear_noalloc(rpbh: Rpbh, cb_a: Codebook, cb_w: Codebook, X, w_codes, w_norm, bias=None, epilogue="none",

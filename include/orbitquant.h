@@ -69,6 +69,12 @@ typedef struct oq_codebook_s* oq_codebook_t;
 /* Version of this ABI (major*100 + minor). */
 OQ_API int oq_version(void);
 
+/* Number of device allocations (cudaMalloc) the library has made in this
+ * process, on every device: the status words and the handles' device tables,
+ * which are the only device memory it allocates.  A diagnostic: a call that
+ * leaves it unchanged allocated nothing.  Never fails. */
+OQ_API long long oq_device_allocations(void);
+
 /* Message for the last error returned on this host thread ("" if none). */
 OQ_API const char* oq_last_error(void);
 
@@ -144,7 +150,9 @@ OQ_API int oq_rotation_kind(oq_rpbh_t r, int* kind);
  * same Pi^(k), so it still cancels in oq_linear).  rounds = 1 is oq_make_rpbh;
  * rounds 2 and 3 run a separate kernel that keeps the row pair in shared
  * memory between rounds (d <= 16384, 32 <= block <= 1024).
- * Errors: as oq_make_rpbh; OQ_ERR_ARG unless 1 <= rounds <= 3.
+ * Errors: as oq_make_rpbh; OQ_ERR_ARG unless 1 <= rounds <= 3;
+ * OQ_ERR_UNSUPPORTED for rounds >= 2 unless d % 32 == 0, d <= 16384 and
+ * block >= 32 (the limits of the composed kernel, checked before any upload).
  * ------------------------------------------------------------------------- */
 OQ_API int oq_make_composed_rpbh(uint64_t seed, int d, int block, int rounds, oq_rpbh_t* out);
 /* Rounds of a rotation handle (1 for every handle but a composed one). */

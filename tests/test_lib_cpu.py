@@ -164,6 +164,15 @@ def test_composed_rotation_errors(oq):
         r.export_round(0)
     with pytest.raises(ValueError):
         oq.Rpbh(0, 256, 64, kind="block_rht", rounds=2)
+    # widths and blocks the composed kernel cannot run are refused when the
+    # handle is made, with the kernel's own limits (one round has no such limit)
+    for d, block in ((32768, 128), (65536, 256), (16416, 32), (240, 16), (4096, 16)):
+        assert oq.lib().oq_make_composed_rpbh(0, d, block, 2, ctypes.byref(h)) == oq.OQ_ERR_UNSUPPORTED
+        assert "d <= 16384" in oq.lib().oq_last_error().decode()
+        assert oq.lib().oq_make_composed_rpbh(0, d, block, 1, ctypes.byref(h)) == oq.OQ_OK
+        oq.lib().oq_free_rpbh(h)
+    assert oq.lib().oq_make_composed_rpbh(0, 16384, 32, 3, ctypes.byref(h)) == oq.OQ_OK
+    oq.lib().oq_free_rpbh(h)
 
 
 def test_gemm_bit_width_checks(oq):
@@ -195,3 +204,8 @@ def test_debug_switch(oq):
     lib = oq.lib()
     assert lib.oq_set_debug(1) == oq.OQ_OK
     assert lib.oq_set_debug(0) == oq.OQ_OK
+
+
+def test_device_allocation_counter_is_exported(oq):
+    # no device here, so nothing has been allocated; the counter never fails
+    assert oq.device_allocations() == 0

@@ -233,6 +233,46 @@ def test_wan_ffn_w4a6_sampled(oq, codebooks):
     assert _rel_fro(y1.cpu().double().numpy()[rows], ref) <= TOL
 
 
+def test_wan_ffn_fc2_w4a6_chain(oq, codebooks):
+    # Wan FFN fc2: input width d = 8960 (fc1's GELU output), 6-bit activations,
+    # W2 [1536 x 8960] with 4-bit weights.  fc2's input is the oracle's own
+    # bf16 fc1 output on 1201 tokens sampled across all 32760 (each layer is
+    # judged on its own inputs; 1201 is ragged against the GEMM's 256-row
+    # tiles).  Checks, in order: the GPU's 6-bit activation codes at d = 8960
+    # against the oracle's (band rule), the (6,4) GEMM on the oracle's codes
+    # at K = 8960, and the full fc2 layer (GPU act-quant -> GEMM).
+    M, d1, d2, h = 32760, 1536, 8960, 128
+    rows = np.linspace(0, M - 1, 1201).astype(int)
+    X = inputs.activations(4, M, d1)[rows]
+    W1 = inputs.weights(4, inputs.T_W, d2, d1)
+    W2 = inputs.weights(4, inputs.T_W2, d1, d2)
+    ca1, s1 = _oracle_act(codebooks, X, d1, h, 6)
+    cw1, r1 = _oracle_weight(codebooks, W1, d1, h, 4)
+    ref1 = olin.linear_from_codes(ca1, s1, cw1, r1, codebooks(d1, 6)["centroids"], codebooks(d1, 4)["centroids"],
+                                  d1, gelu=True)
+    h1 = inputs.to_bf16_bits(ref1)
+    # act-quant of the fc2 input
+    perm, signs = orpbh.draw_permutation_and_signs(0, d2)
+    book6 = codebooks(d2, 6)
+    ca2, s2, T2 = oqz.quantize_rows(inputs.bf16_bits_to_f64(h1), perm, signs, h, book6["centroids"])
+    r = oq.Rpbh(0, d2, h)
+    cb6 = _lib_cb(oq, d2, 6)
+    got_codes, got_norm = oq.quantize_act(r, cb6, _dev_bf16(h1))
+    torch.cuda.synchronize()
+    oq.device_status()
+    got = oqz.unpack_codes(got_codes.cpu().numpy(), 6, d2)
+    near = oqz.boundary_distance(T2, book6["boundaries"]) < 1e-5
+    assert not np.any((got != ca2) & ~near)
+    assert np.max(np.abs(got_norm.cpu().numpy() - s2) / s2) < 1e-6
+    # the (6,4) GEMM at K = 8960 on the oracle's codes
+    cw2, r2 = _oracle_weight(codebooks, W2, d2, h, 4)
+    y, _, ref2 = _run_codes(oq, codebooks, ca2, s2, cw2, r2, d2, 6, 4)
+    assert _rel_fro(y, ref2) <= TOL
+    # the whole fc2 layer on the GPU
+    y2, _ = _full_layer(oq, h1, W2, d2, h, 6, 4)
+    assert _rel_fro(y2.cpu().double().numpy(), ref2) <= TOL
+
+
 def test_empty_shapes(oq):
     cb = _lib_cb(oq, 256, 4)
     a = torch.empty((0, 128), dtype=torch.uint8, device="cuda")

@@ -107,17 +107,33 @@ def test_single_linear_workload_act_and_weight(oq, codebooks, bits):
     _check_rows(oq, codebooks, W, 256, 64, bits, weight=True)
 
 
-@pytest.mark.parametrize("d,h", [(256, 64), (1536, 128), (3072, 128), (3072, 256), (8960, 128), (12288, 128),
-                                 (1024, 1024), (512, 32), (1536, 512)])
+@pytest.mark.parametrize("d,h", [(256, 64), (8960, 128), (1024, 1024), (512, 32), (1536, 512)])
 @pytest.mark.parametrize("bits", [2, 4, 6])
 def test_sweep_shapes_with_ragged_tail(oq, codebooks, d, h, bits):
-    # several stages and CTAs, M not a multiple of the rows per stage, sparse tail rows
+    # widths and blocks beyond the sweep grid: several stages and CTAs, M not
+    # a multiple of the rows per stage, sparse tail rows
     M = 300 if d >= 8192 else 1000
     X = inputs.sweep_activations(M, d)
     rep = []
     _check_rows(oq, codebooks, X, d, h, bits, report=rep)
     mism, inband, total = rep[0]
     assert mism <= inband
+
+
+@pytest.mark.parametrize("d", [1536, 3072, 12288])
+@pytest.mark.parametrize("h", [64, 128, 256])
+@pytest.mark.parametrize("bits", [2, 4, 6])
+def test_sweep_grid(oq, codebooks, d, h, bits):
+    # The rotate+quantize sweep's whole grid of widths, blocks and code widths
+    # (every kernel configuration the sweep launches), each on M = 999 rows:
+    # ragged for every rows-per-stage, N(0,1) rows followed by the one-hot and
+    # k-sparse tail and a zero last row.
+    M = 999
+    X = inputs.sweep_activations(M, d)
+    rep = []
+    _check_rows(oq, codebooks, X, d, h, bits, report=rep)
+    mism, inband, total = rep[0]
+    assert total == M * d and mism <= inband
 
 
 @pytest.mark.parametrize("bits", [1, 3, 5])

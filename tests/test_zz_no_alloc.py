@@ -53,7 +53,9 @@ def test_noalloc_matches_linear_on_two_calls(oq):
         ref, _ = oq.linear(r, cb, cb, X, w_codes, w_norm, bias=bias)
         y32 = torch.full((M, N), float("nan"), device="cuda")
         y16 = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+        allocs = oq.device_allocations()
         oq.linear_noalloc(r, cb, cb, X, w_codes, w_norm, bias=bias, out_f32=y32, out_bf16=y16)
+        assert oq.device_allocations() == allocs, "the no-allocation entry point allocated device memory"
         torch.cuda.synchronize()
         oq.device_status()
         assert _rel(y32, ref) <= TOL, f"call {call}"
