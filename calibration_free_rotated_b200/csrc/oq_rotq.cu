@@ -28,9 +28,20 @@
 //     addresses each); the Rademacher signs sit in 8 registers as sign bytes
 //     and are applied while splitting the gathered word into two floats
 //     (one byte-permute, one shift-add, one logic op per pair).
-//   * The two rows travel as f32x2 pairs: the sum of squares and the five
-//     in-thread FWHT stages are packed f32x2 instructions; the remaining
-//     log2(h/32) stages are xor-shuffles across the lanes of a block.
+//   * The two rows travel as f32x2 pairs: the sum of squares and the FWHT
+//     stages are packed f32x2 instructions.  For blocks of h = 64, 128, 256
+//     (L = h/32 lanes) every stage runs in-thread: the gather fills layout A,
+//     where lane l's register group t holds coordinates 32 (t ^ l) + (32/L) l
+//     + [0, 32/L), so A's stages cover the block bits above 5; one transpose
+//     (register group t xor-shuffled with lane l ^ t, group 0 staying put)
+//     then gives layout B, where group u holds 32 l + (32/L)(u ^ l) + [0,
+//     32/L), for the stages over bits 0..4.  The XOR relabelling keeps every
+//     register index a compile-time constant and turns the swapped roles of
+//     the butterflies into a per-lane sign (one FMA per output); the packed
+//     codes' groups are moved back from u to u ^ l before the store.  At
+//     h = 128 this moves 24 pairs per thread through shuffles instead of 64.
+//     Wider blocks, and code widths whose groups are not whole bytes, words or
+//     three-word halves, keep log2(h/32) xor-shuffle butterfly stages.
 //   * Row norms: lane-segment shuffle reductions, per-segment partials in
 //     shared memory, summed in a fixed order (deterministic).
 //   * Centroid search in the unit interval: y = sat(t * alpha + 1/2) (the row

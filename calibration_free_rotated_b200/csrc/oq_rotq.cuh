@@ -264,6 +264,52 @@ struct Direct {
   }
 };
 
+// Gather step without a permutation for the block-transposed FWHT: group t of
+// lane bl is columns 32 (t ^ bl) + R bl + [0, R) of the block, read for both
+// rows of the pair straight from ring slot SLOT (src = the block's first
+// column + 2 R bl bytes in slot 0).
+template <int CFG, int LOGHB>
+struct DirectX {
+  template <int SLOT>
+  static __device__ __forceinline__ void run(unsigned long long (&v)[32], unsigned long long& ss2, uint32_t src, int bl,
+                                             const uint32_t (&sb)[8]) {
+    constexpr int L = 1 << LOGHB, R = 32 / L;
+    constexpr uint32_t OFF = SLOT * Cfg<CFG>::IBS, HALF = Cfg<CFG>::HALF;
+    unsigned long long sq[4] = {0ull, 0ull, 0ull, 0ull};
+#pragma unroll
+    for (int t = 0; t < L; ++t) {
+      const uint32_t at = src + OFF + 64u * (uint32_t)(t ^ bl);
+      uint32_t wa[R / 2], wb[R / 2];  // R bf16 of each row
+      if constexpr (R >= 8) {
+#pragma unroll
+        for (int c = 0; c < R / 8; ++c) {
+          const uint4 A = lds_u128(at + 16u * c), B = lds_u128(at + HALF + 16u * c);
+          wa[4 * c] = A.x, wa[4 * c + 1] = A.y, wa[4 * c + 2] = A.z, wa[4 * c + 3] = A.w;
+          wb[4 * c] = B.x, wb[4 * c + 1] = B.y, wb[4 * c + 2] = B.z, wb[4 * c + 3] = B.w;
+        }
+      } else {
+        uint32_t x0, x1, y0, y1;
+        asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(x0), "=r"(x1) : "r"(at));
+        asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(y0), "=r"(y1) : "r"(at + HALF));
+        wa[0] = x0, wa[1] = x1, wb[0] = y0, wb[1] = y1;
+      }
+#pragma unroll
+      for (int m = 0; m < R / 2; ++m) {
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          const int i = R * t + 2 * m + e;
+          const uint32_t sgb = __byte_perm(sb[i >> 2], 0u, 0x0444u | ((uint32_t)(i & 3) << 12));
+          const uint32_t ra = e ? ((wa[m] & 0xFFFF0000u) ^ sgb) : ((wa[m] << 16) + sgb);
+          const uint32_t rb = e ? ((wb[m] & 0xFFFF0000u) ^ sgb) : ((wb[m] << 16) + sgb);
+          v[i] = u2_pack(ra, rb);
+          sq[i & 3] = f2_fma(v[i], v[i], sq[i & 3]);
+        }
+      }
+    }
+    ss2 = f2_add(f2_add(sq[0], sq[1]), f2_add(sq[2], sq[3]));
+  }
+};
+
 // Unnormalised Walsh-Hadamard transform (Sylvester order) of the blocks of h =
 // 32 << LOGHB coordinates that span lanes 2^LOGHB-aligned: coordinate 32 l + i
 // of the block sits in v[i] of lane l (f32x2: both rows of a pair).  Five
@@ -294,6 +340,137 @@ __device__ __forceinline__ void fwht_pairs(unsigned long long (&v)[32], int lane
       const float ohi = __shfl_xor_sync(0xFFFFFFFFu, hi, 1 << k);
       v[i] = f2_fma(v[i], sg2, f2_pack(olo, ohi));
     }
+  }
+}
+
+// ---- block-transposed FWHT ------------------------------------------------------
+// For blocks of h = 32 L coordinates (L = 2^LOGHB lanes) the lane-crossing
+// stages run in-thread too, with one register transpose between two layouts.
+// Registers come in L groups of R = 32 / L pairs; lane l of the block holds
+//   layout A (after the gather): group t = coordinates 32 (t ^ l) + R l + [0, R)
+//   layout B (after the transpose): group u = coordinates 32 l + R (u ^ l) + [0, R)
+// A's stages run over bits 5.. of the block coordinate (its group index, XOR-
+// relabelled by l), B's over bits 0..4.  Group t of lane l is exactly what lane
+// l ^ t needs in B's group t, so the transpose is one xor-shuffle per pair of
+// groups t != 0 and group 0 stays in place: (L - 1) R pairs move instead of
+// 32 LOGHB, with compile-time register indices.  A stage over a relabelled
+// bit s swaps the roles of the two inputs in lanes whose bit s of l is set;
+// that is folded into a sign, so both outputs are one FMA each:
+//   x0' = x0 * sg + x1,   x1' = x0 - x1 * sg   (sg = -1 where bit s of l is 1).
+template <int BITS, int LOGHB>
+struct Xch {
+  static constexpr int L = 1 << LOGHB, R = 32 / L, LOGR = 5 - LOGHB;
+  static constexpr int CB = R * BITS;  // bits of one group's codes
+  // The packed codes of a group are moved between positions u and u ^ l; each
+  // level k swaps neighbouring runs of CB << k bits, which this supports when
+  // every run is whole words, a half / byte / nibble of a word, or half of a
+  // three-word group (48 bits, 3- and 6-bit codes).
+  static constexpr bool level_ok(int S) {
+    return S % 32 == 0 || S == 16 || S == 8 || S == 4 || (S == 48 && BITS % 3 == 0);
+  }
+  static constexpr bool ok() {
+    bool r = LOGHB >= 1 && LOGHB <= 3;
+    for (int k = 0; k < 3; ++k) r = r && (k >= LOGHB || level_ok(CB << k));
+    return r;
+  }
+};
+
+// The relabelled stages over the group index of a layout (A or B).
+template <int LOGHB>
+__device__ __forceinline__ void groups_stages(unsigned long long (&v)[32], const unsigned long long (&sg)[3],
+                                              const unsigned long long (&nsg)[3]) {
+  constexpr int L = 1 << LOGHB, R = 32 / L;
+#pragma unroll
+  for (int s = 0; s < LOGHB; ++s) {
+#pragma unroll
+    for (int t = 0; t < L; ++t) {
+      if ((t >> s) & 1) continue;
+      const int t1 = t | (1 << s);
+#pragma unroll
+      for (int b = 0; b < R; ++b) {
+        const unsigned long long x0 = v[R * t + b], x1 = v[R * t1 + b];
+        v[R * t + b] = f2_fma(x0, sg[s], x1);
+        v[R * t1 + b] = f2_fma(x1, nsg[s], x0);
+      }
+    }
+  }
+}
+
+template <int LOGHB>
+__device__ __forceinline__ void fwht_xch(unsigned long long (&v)[32], const unsigned long long (&sg)[3],
+                                         const unsigned long long (&nsg)[3]) {
+  constexpr int L = 1 << LOGHB, R = 32 / L;
+  groups_stages<LOGHB>(v, sg, nsg);  // layout A: coordinate bits 5 .. 4 + LOGHB
+#pragma unroll
+  for (int t = 1; t < L; ++t) {
+#pragma unroll
+    for (int b = 0; b < R; ++b) {
+      float lo, hi;
+      f2_unpack(v[R * t + b], lo, hi);
+      lo = __shfl_xor_sync(0xFFFFFFFFu, lo, t);
+      hi = __shfl_xor_sync(0xFFFFFFFFu, hi, t);
+      v[R * t + b] = f2_pack(lo, hi);
+    }
+  }
+  // layout B: coordinate bits 0 .. 4 - LOGHB (standard), then the group bits
+#pragma unroll
+  for (int s = 1; s < R; s <<= 1) {
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+      if ((i & s) == 0) {
+        const unsigned long long x0 = v[i], x1 = v[i + s];
+        v[i] = f2_add(x0, x1);
+        v[i + s] = f2_sub(x0, x1);
+      }
+    }
+  }
+  groups_stages<LOGHB>(v, sg, nsg);
+}
+
+// Swaps every pair of neighbouring runs of S bits of the packed row when sw.
+template <int BITS, int S>
+__device__ __forceinline__ void swap_runs(uint32_t (&w)[BITS], bool sw) {
+  if constexpr (S % 32 == 0) {
+    constexpr int WS = S / 32;
+#pragma unroll
+    for (int c = 0; c < BITS; c += 2 * WS) {
+#pragma unroll
+      for (int j = 0; j < WS; ++j) {
+        const uint32_t a = w[c + j], b = w[c + WS + j];
+        w[c + j] = sw ? b : a;
+        w[c + WS + j] = sw ? a : b;
+      }
+    }
+  } else if constexpr (S == 48) {  // halves of each three-word group
+#pragma unroll
+    for (int c = 0; c < BITS; c += 3) {
+      const uint32_t m0 = __byte_perm(w[c + 1], w[c + 2], 0x5432), m1 = __byte_perm(w[c + 2], w[c], 0x5432),
+                     m2 = __byte_perm(w[c], w[c + 1], 0x5432);
+      w[c] = sw ? m0 : w[c];
+      w[c + 1] = sw ? m1 : w[c + 1];
+      w[c + 2] = sw ? m2 : w[c + 2];
+    }
+  } else if constexpr (S == 16 || S == 8) {
+    const uint32_t sel = sw ? (S == 16 ? 0x1032u : 0x2301u) : 0x3210u;
+#pragma unroll
+    for (int j = 0; j < BITS; ++j) w[j] = __byte_perm(w[j], 0u, sel);
+  } else {
+    static_assert(S == 4, "unsupported run width");
+#pragma unroll
+    for (int j = 0; j < BITS; ++j) {
+      const uint32_t x = ((w[j] >> 4) & 0x0F0F0F0Fu) | ((w[j] & 0x0F0F0F0Fu) << 4);
+      w[j] = sw ? x : w[j];
+    }
+  }
+}
+
+// Moves the packed codes of group u (CB bits at u * CB) to group u ^ l: level
+// k swaps runs of CB << k bits where bit k of l is set.
+template <int BITS, int LOGHB, int K = 0>
+__device__ __forceinline__ void xor_groups(uint32_t (&w)[BITS], int l) {
+  if constexpr (K < LOGHB) {
+    swap_runs<BITS, (Xch<BITS, LOGHB>::CB << K)>(w, ((l >> K) & 1) != 0);
+    xor_groups<BITS, LOGHB, K + 1>(w, l);
   }
 }
 
@@ -336,6 +513,9 @@ struct Thread {
   uint32_t src_direct;  // ring slot 0: row 2pr, columns 32g.. (no rotation)
   uint32_t ib_w0, ib_w1;
   float2* partial;
+  int bl;                          // lane within the Hadamard block (block-transposed FWHT)
+  uint32_t src_blk;                // ring slot 0: row 2pr, start of the block + 2 R bl (no permutation)
+  unsigned long long sg[3], nsg[3];  // (s, s) and (-s, -s), s = -1 where bit k of bl is set
 };
 
 // Interleave stage `it` (ring slot it % STAGES) into pair buffer it & 1.
@@ -361,15 +541,22 @@ __device__ __forceinline__ bool interleave(const Args& a, const Thread& t, int i
 }
 
 // Gather + signs + FWHT of stage `it`, and the segment partials of its squared norms.
-template <int LOGHB, int CFG, bool PERM>
+template <int BITS, int LOGHB, int CFG, bool PERM>
 __device__ __forceinline__ void transform(const Args& a, const Thread& t, int it, unsigned long long (&v)[32],
                                           const uint32_t (&offw)[16], const uint32_t (&sb)[8]) {
+  constexpr bool XCH = Xch<BITS, LOGHB>::ok();
   unsigned long long ss2;
   if constexpr (PERM) {
     if (it & 1)
       Gather<CFG, LOGHB>::template run<1>(v, ss2, offw, sb, t.s_base);
     else
       Gather<CFG, LOGHB>::template run<0>(v, ss2, offw, sb, t.s_base);
+  } else if constexpr (XCH) {
+    static_assert(Cfg<CFG>::STAGES <= 2, "slot offsets are unrolled for two slots");
+    if (it % Cfg<CFG>::STAGES == 1)
+      DirectX<CFG, LOGHB>::template run<1>(v, ss2, t.src_blk, t.bl, sb);
+    else
+      DirectX<CFG, LOGHB>::template run<0>(v, ss2, t.src_blk, t.bl, sb);
   } else {
     static_assert(Cfg<CFG>::STAGES <= 2, "slot offsets are unrolled for two slots");
     if (it % Cfg<CFG>::STAGES == 1)
@@ -391,12 +578,16 @@ __device__ __forceinline__ void transform(const Args& a, const Thread& t, int it
     if ((t.lane & ((1 << a.seg_log) - 1)) == 0)
       t.partial[(it & 1) * t.nparts + (t.tid >> a.seg_log)] = make_float2(lo, hi);
   }
-  fwht_pairs<LOGHB>(v, t.lane);
+  if constexpr (XCH)
+    fwht_xch<LOGHB>(v, t.sg, t.nsg);
+  else
+    fwht_pairs<LOGHB>(v, t.lane);
 }
 
 // Normalise, search, pack and store stage `it`.
-template <int BITS>
+template <int BITS, int LOGHB>
 __device__ __forceinline__ void quantize(const Args& a, const Thread& t, int it, const unsigned long long (&v)[32]) {
+  constexpr bool XCH = Xch<BITS, LOGHB>::ok();
   const int R = 2 * a.P;
   const int grp = blockIdx.x + it * gridDim.x;
   const int row0 = grp * R;
@@ -417,6 +608,10 @@ __device__ __forceinline__ void quantize(const Args& a, const Thread& t, int it,
   const float A_b = sum_b > 0.0f ? a.alpha_h * rsqrtf(sum_b) : 0.0f;
   uint32_t wa[BITS], wb[BITS];
   search_pack<BITS>(v, A_a, A_b, a.nb, t.qkey, wa, wb);
+  if constexpr (XCH) {  // register group u holds the codes of group u ^ bl
+    xor_groups<BITS, LOGHB>(wa, t.bl);
+    xor_groups<BITS, LOGHB>(wb, t.bl);
+  }
   const int row = row0 + 2 * t.pr;
   const size_t rb = (size_t)(a.d / 8 * BITS);
   uint8_t* dst = a.codes + (size_t)row * rb + (size_t)t.g * (4 * BITS);
@@ -480,12 +675,28 @@ __global__ void __launch_bounds__(CFG == 2 ? 512 : 384, 1) rotq_kernel(const __g
   // gather addresses: pair word of column c of pair pr sits at word
   // pr*d + swz(c) of a pair buffer, swz swapping the 16-byte halves of odd
   // 32-column segments (conflict-free interleave stores)
+  // Register r of a thread holds coordinate col(r) of its row pair: 32 g + r,
+  // or, with the block-transposed FWHT, layout A's
+  // 32 (g - bl) + 32 ((r / XR) ^ bl) + XR bl + r % XR.
+  constexpr bool XCH = Xch<BITS, LOGHB>::ok();
+  constexpr int XR = XCH ? (32 >> LOGHB) : 32;
+  t.bl = XCH ? (t.g & ((1 << LOGHB) - 1)) : 0;
+  auto col = [&](int r) -> uint32_t {
+    return 32u * (uint32_t)(t.g - t.bl) + 32u * (uint32_t)((r / XR) ^ t.bl) + (uint32_t)(XR * t.bl + r % XR);
+  };
+#pragma unroll
+  for (int k = 0; k < 3; ++k) {
+    const float sgn = ((t.bl >> k) & 1) ? -1.0f : 1.0f;
+    t.sg[k] = f2_pack(sgn, sgn);
+    t.nsg[k] = f2_pack(-sgn, -sgn);
+  }
+  t.src_blk = t.s_ring + (uint32_t)t.pr * (uint32_t)d * 2u + 64u * (uint32_t)(t.g - t.bl) + 2u * (uint32_t)(XR * t.bl);
   uint32_t offw[16];
   if constexpr (PERM) {
     const uint32_t rowbase = (uint32_t)t.pr * (uint32_t)d;
 #pragma unroll
     for (int k = 0; k < 16; ++k) {
-      const uint32_t pw = __ldg(a.perm2 + 16 * t.g + k);
+      const uint32_t pw = __ldg(a.perm2 + (col(2 * k) >> 1));  // col(2k) is even, col(2k + 1) = col(2k) + 1
       uint32_t c0 = pw & 0xFFFFu, c1 = pw >> 16;
       c0 ^= ((c0 >> 5) & 1u) << 2;
       c1 ^= ((c1 >> 5) & 1u) << 2;
@@ -497,17 +708,17 @@ __global__ void __launch_bounds__(CFG == 2 ? 512 : 384, 1) rotq_kernel(const __g
       offw[k] = (o0 & 0xFFFFu) | (o1 << 16);
     }
   }
-  // sign bytes: byte m of sb[q] is 0x80 when coordinate 32g + 4q + m is negated
+  // sign bytes: byte m of sb[q] is 0x80 when coordinate col(4q + m) is negated
   uint32_t sb[8];
-  {
-    const uint32_t sw = __ldg(a.signs + t.g);
 #pragma unroll
-    for (int q = 0; q < 8; ++q) {
-      uint32_t x = 0;
+  for (int q = 0; q < 8; ++q) {
+    uint32_t x = 0;
 #pragma unroll
-      for (int m = 0; m < 4; ++m) x |= ((sw >> (4 * q + m)) & 1u) << (8 * m + 7);
-      sb[q] = x;
+    for (int m = 0; m < 4; ++m) {
+      const uint32_t c = col(4 * q + m);
+      x |= ((__ldg(a.signs + (c >> 5)) >> (c & 31u)) & 1u) << (8 * m + 7);
     }
+    sb[q] = x;
   }
   // interleave addresses: 16-byte chunk c = n ^ rot of the thread's 32 columns
   // (lane-rotated, conflict-free ring reads); odd segments swap halves
@@ -534,7 +745,7 @@ __global__ void __launch_bounds__(CFG == 2 ? 512 : 384, 1) rotq_kernel(const __g
       asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
       issue_stage_load<CFG>(a, t.s_ring, t.s_bars, Cfg<CFG>::STAGES, t.lane);
     }
-    transform<LOGHB, CFG, PERM>(a, t, 0, v, offw, sb);
+    transform<BITS, LOGHB, CFG, PERM>(a, t, 0, v, offw, sb);
     for (int it = 0; it < n_it; ++it) {
       const bool more = it + 1 < n_it;
       ok = more ? interleave<CFG>(a, t, it + 1) : true;
@@ -543,26 +754,26 @@ __global__ void __launch_bounds__(CFG == 2 ? 512 : 384, 1) rotq_kernel(const __g
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
         issue_stage_load<CFG>(a, t.s_ring, t.s_bars, it + 1 + Cfg<CFG>::STAGES, t.lane);
       }
-      quantize<BITS>(a, t, it, v);
-      if (more) transform<LOGHB, CFG, PERM>(a, t, it + 1, v, offw, sb);
+      quantize<BITS, LOGHB>(a, t, it, v);
+      if (more) transform<BITS, LOGHB, CFG, PERM>(a, t, it + 1, v, offw, sb);
     }
   } else {
     // no permutation: each stage is read straight from its ring slot, which is
     // released at the barrier that follows its transform
     bool ok = mbar_wait_bounded(t.s_bars, 0u, a.status);
-    if (ok) transform<LOGHB, CFG, PERM>(a, t, 0, v, offw, sb);
+    if (ok) transform<BITS, LOGHB, CFG, PERM>(a, t, 0, v, offw, sb);
     for (int it = 0; it < n_it; ++it) {
       if (__syncthreads_or(!ok)) return;  // partials of `it`; ring slot of `it` released
       if (warp == 0) {
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
         issue_stage_load<CFG>(a, t.s_ring, t.s_bars, it + Cfg<CFG>::STAGES, t.lane);
       }
-      quantize<BITS>(a, t, it, v);
+      quantize<BITS, LOGHB>(a, t, it, v);
       if (it + 1 < n_it) {
         const int nx = it + 1;
         ok = mbar_wait_bounded(t.s_bars + 8u * (nx % Cfg<CFG>::STAGES), (uint32_t)(nx / Cfg<CFG>::STAGES) & 1u,
                                a.status);
-        if (ok) transform<LOGHB, CFG, PERM>(a, t, nx, v, offw, sb);
+        if (ok) transform<BITS, LOGHB, CFG, PERM>(a, t, nx, v, offw, sb);
       }
     }
   }
