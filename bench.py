@@ -417,17 +417,15 @@ def run_ours(args, world, rank, local):
         "gpu_launches": 2 * args.steps,
         "clocks": clk.summary(),
     }
-    st = None
-    if rank == 0 and not args.no_parity:
-        # parity of this run's own outputs, outside the timed region: sampled
-        # rows of set 0 (codes, norms and Y from the timed steps) against the
-        # oracle, with the boundary ties counted
-        _, st = oracle_sample(8)
-        line["parity"] = parity_report(oq, cb, sets[0], wn, st, K, bias)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        # the host-side oracle leg: the timed CPU baseline, and (untimed) the
+        # parity of this run's own outputs -- sampled rows of set 0 (codes,
+        # norms and Y from the timed steps) against the oracle, with the
+        # boundary ties counted
         rows = 2048
-        if st is None:
-            _, st = oracle_sample(8)
+        _, st = oracle_sample(8)
+        if not args.no_parity:
+            line["parity"] = parity_report(oq, cb, sets[0], wn, st, K, bias)
         dt, _ = oracle_sample(rows, st)
         _, sflops = algorithmic(rows, K, N, 4, 4)
         line["cpu_baseline"] = {"value": sflops / dt / 1e12, "unit": UNIT, "cores": cpu_threads(), "kind": "oracle",
@@ -623,12 +621,57 @@ def run_workload(args):
     return 0
 
 
+def run_flatness(args):
+    """The flatness check ([RHT] Key contribution 4: rho3 and rhoinf of every
+    row, and the batch maxima) timed alone after a 256 MB L2 flush, with per-row
+    outputs and with the batch maxima only, on N(0,1) bf16 rows.  Algorithmic
+    bytes: the rows once (2 M d) plus 8 bytes per row written (4 per measure)
+    and the maxima.  One JSON line per shape; not the contract line."""
+    import torch
+    from calibration_free_rotated_b200 import build
+    build.build()
+    from calibration_free_rotated_b200 import orbitquant as oq
+    peaks, src = load_peaks()
+    torch.manual_seed(0)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+    for M, d in ((4608, 3072), (32768, 3072), (32760, 8960), (16384, 12288)):
+        X = torch.randn(M, d, device="cuda").to(torch.bfloat16)
+        r3 = torch.empty(M, device="cuda")
+        ri = torch.empty(M, device="cuda")
+        bm = torch.empty(2, device="cuda")
+        ms_rows = _flush_and_time(lambda: oq.row_flatness(X, r3, ri, bm), flush, args.steps, args.warmup)
+        ms_batch = _flush_and_time(lambda: oq.row_flatness(X, batch_max=bm, want_rows=False), flush, args.steps,
+                                   args.warmup)
+        oq.device_status()
+        byt_rows, byt_batch = 2.0 * M * d + 8.0 * M + 8, 2.0 * M * d + 8
+        out = {"flatness": "row_flatness", "M": M, "d": d, "peak_source": src,
+               "with_rows": {"us": 1e3 * ms_rows, "GB/s": byt_rows / ms_rows / 1e6,
+                             "frac_hbm": byt_rows / ms_rows / 1e6 / peaks["hbm_gbs"]},
+               "batch_only": {"us": 1e3 * ms_batch, "GB/s": byt_batch / ms_batch / 1e6,
+                              "frac_hbm": byt_batch / ms_batch / 1e6 / peaks["hbm_gbs"]}}
+        print(json.dumps(out), flush=True)
+        del X
+    return 0
+
+
 def _sylvester(h, device):
     import torch
     H = torch.ones((1, 1), dtype=torch.float64, device=device)
     while H.shape[0] < h:
         H = torch.cat([torch.cat([H, H], 1), torch.cat([H, -H], 1)], 0)
     return H
+
+
+def rotate_rows_f64(U, tables, h):
+    """The (composed) RPBH rotation of fp64 rows U [n, d] for the sweep's error
+    measurement: per round (round 1 first), gather by the round's permutation,
+    multiply by its signs, then each block of h by the normalised Sylvester
+    Hadamard matrix.  tables: [(perm int64 [d], sign float64 [d]), ...]."""
+    n, d = U.shape
+    H = _sylvester(h, U.device) / math.sqrt(h)
+    for perm_t, sign in tables:
+        U = ((U[:, perm_t] * sign).view(n, d // h, h) @ H.T).view(n, d)
+    return U
 
 
 def run_sweep(args):
@@ -660,6 +703,9 @@ def run_sweep(args):
             n_adv = M // 8
             rows_dense = torch.arange(0, min(4096, M - n_adv), device=dev)
             rows_adv = torch.arange(M - n_adv, min(M - 1, M - n_adv + 4096), device=dev)  # not the zero row
+            # the flatness check's batch maxima ([RHT] Key contribution 4) of each row set
+            flat = {k: oq.row_flatness(X[rows].contiguous(), want_rows=False)[2].tolist()
+                    for k, rows in (("dense", rows_dense), ("adversarial", rows_adv))}
             for h in (64, 128, 256):
                 r = oq.Rpbh(0, d, h, rounds=args.rounds)
                 tables = []
@@ -668,12 +714,8 @@ def run_sweep(args):
                     sign = torch.tensor([-1.0 if (sbits[j >> 5] >> (j & 31)) & 1 else 1.0 for j in range(d)],
                                         dtype=torch.float64, device=dev)
                     tables.append((torch.from_numpy(perm.astype(np.int64)).to(dev), sign))
-                H = _sylvester(h, dev) / math.sqrt(h)
-
                 def unit_rotated(rows):
-                    u = X[rows].double()
-                    for perm_t, sign in tables:  # round 1 first
-                        u = ((u[:, perm_t] * sign).view(len(rows), d // h, h) @ H.T).view(len(rows), d)
+                    u = rotate_rows_f64(X[rows].double(), tables, h)
                     return u / u.norm(dim=1, keepdim=True).clamp_min(1e-300)
 
                 T = {"dense": unit_rotated(rows_dense), "adversarial": unit_rotated(rows_adv)}
@@ -695,6 +737,7 @@ def run_sweep(args):
                         k = _unpack_codes_torch(codes[rows], bits, d)
                         err = ((T[key] - cent[k]) ** 2).sum(dim=1)
                         line["mse_" + key] = float(err.mean())
+                        line["rho3_max_" + key], line["rhoinf_max_" + key] = flat[key]
                     print(json.dumps(line), flush=True)
             del X
     oq.device_status()
@@ -725,6 +768,7 @@ def main():
     ap.add_argument("--workload", choices=["flux_mlp", "wan_ffn", "flux_qkv_w3a3"],
                     help="per-kernel times of a layer workload")
     ap.add_argument("--sweep", action="store_true", help="the rotate+quantize sweep with empirical MSE")
+    ap.add_argument("--flatness", action="store_true", help="time the flatness check (rho3, rhoinf per row)")
     ap.add_argument("--sweep-rows", default="1024,16384,65536")
     ap.add_argument("--rounds", type=int, default=1, help="composed RPBH rounds for --sweep and --profile rotq (1, 2 or 3)")
     ap.add_argument("--rows", type=int, default=4608)
@@ -742,6 +786,8 @@ def main():
         return run_workload(args)
     if args.sweep:
         return run_sweep(args)
+    if args.flatness:
+        return run_flatness(args)
     if args.warmup < 3:
         args.warmup = 3
     world, rank, local = dist_setup()

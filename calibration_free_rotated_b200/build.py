@@ -18,7 +18,7 @@ CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "liborbitquant.so")
 SOURCES = ["oq_host.cpp", "oq_rotq.cu", "oq_rotq_cfg0.cu", "oq_rotq_cfg1.cu", "oq_rotq_cfg2.cu",
            "oq_rotq_cfg0_np.cu", "oq_rotq_cfg1_np.cu", "oq_rotq_cfg2_np.cu", "oq_rotq_composed.cu", "oq_cbgemm.cu",
-           "oq_noalloc.cu"]
+           "oq_noalloc.cu", "oq_flatness.cu"]
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",
     "-lineinfo", "-O3", "-std=c++17",

@@ -850,6 +850,20 @@ int oq_quantize_act(oq_rpbh_t r, oq_codebook_t cb, const void* X, int M, uint8_t
   return finish(launch_rotq(r, cb, X, M, codes, norms, nullptr, stream), stream);
 }
 
+int oq_row_flatness(const void* X, int M, int d, float* rho3, float* rhoinf, float* batch_max, void* stream) {
+  clear_error();
+  NvtxRange nvtx("oq_row_flatness");
+  if (M < 0) return fail(OQ_ERR_ARG, "M must be >= 0 (got %d)", M);
+  if (d < 8 || d % 8 != 0) return fail(OQ_ERR_UNSUPPORTED, "the flatness check needs d %% 8 == 0 (d=%d)", d);
+  if (M > 0 && !X) return fail(OQ_ERR_ARG, "X is NULL");
+  if (!aligned16(X)) return fail(OQ_ERR_ALIGN, "X must be 16-byte aligned");
+  if (!rho3 && !rhoinf && !batch_max) return fail(OQ_ERR_ARG, "no output requested");
+  if ((rho3 && ((uintptr_t)rho3 & 3u)) || (rhoinf && ((uintptr_t)rhoinf & 3u)) ||
+      (batch_max && ((uintptr_t)batch_max & 3u)))
+    return fail(OQ_ERR_ALIGN, "outputs must be 4-byte aligned");
+  return finish(launch_flatness(X, M, d, rho3, rhoinf, batch_max, stream), stream);
+}
+
 int oq_quantize_weight(oq_rpbh_t r, oq_codebook_t cb, const void* W, int N, uint8_t* codes, void* norms_bf16,
                        void* stream) {
   clear_error();

@@ -101,6 +101,7 @@ int launch_rotq(oq_rpbh_t r, oq_codebook_t cb, const void* X, int M, uint8_t* co
                 uint16_t* norm_bf16, void* stream);
 int launch_rotq_composed(oq_rpbh_t r, oq_codebook_t cb, const void* X, int M, uint8_t* codes, float* norm_f32,
                          uint16_t* norm_bf16, void* stream);
+int launch_flatness(const void* X, int M, int d, float* rho3, float* rhoinf, float* batch_max, void* stream);
 int launch_cbgemm(int d, oq_codebook_t cb_a, oq_codebook_t cb_w, const uint8_t* a_codes, const float* a_norm, int M,
                   const uint8_t* w_codes, const uint16_t* w_norm, int N, const uint16_t* bias, int epilogue,
                   float* Y_f32, uint16_t* Y_bf16, void* stream);

@@ -709,16 +709,22 @@ __global__ void __launch_bounds__(CFG == 2 ? 512 : 384, 1) rotq_kernel(const __g
     }
   }
   // sign bytes: byte m of sb[q] is 0x80 when coordinate col(4q + m) is negated
+  // (a register group's coordinates share one sign word)
   uint32_t sb[8];
+  {
+    uint32_t sw[32 / XR];
 #pragma unroll
-  for (int q = 0; q < 8; ++q) {
-    uint32_t x = 0;
+    for (int t2 = 0; t2 < 32 / XR; ++t2) sw[t2] = __ldg(a.signs + (col(XR * t2) >> 5));
 #pragma unroll
-    for (int m = 0; m < 4; ++m) {
-      const uint32_t c = col(4 * q + m);
-      x |= ((__ldg(a.signs + (c >> 5)) >> (c & 31u)) & 1u) << (8 * m + 7);
+    for (int q = 0; q < 8; ++q) {
+      uint32_t x = 0;
+#pragma unroll
+      for (int m = 0; m < 4; ++m) {
+        const int r = 4 * q + m;
+        x |= ((sw[r / XR] >> (col(r) & 31u)) & 1u) << (8 * m + 7);
+      }
+      sb[q] = x;
     }
-    sb[q] = x;
   }
   // interleave addresses: 16-byte chunk c = n ^ rot of the thread's 32 columns
   // (lane-rotated, conflict-free ring reads); odd segments swap halves

@@ -50,6 +50,7 @@ _SIGS = {
     "oq_linear_codes": (_c_int, [_c_int, _c_void_p, _c_void_p, _c_void_p, _c_void_p, _c_int, _c_void_p, _c_void_p,
                                  _c_int, _c_void_p, _c_int, _c_void_p, _c_void_p, _c_void_p]),
     "oq_linear_workspace_bytes": (_c_size_t, [_c_int, _c_int, _c_int]),
+    "oq_row_flatness": (_c_int, [_c_void_p, _c_int, _c_int, _c_void_p, _c_void_p, _c_void_p, _c_void_p]),
     "oq_linear": (_c_int, [_c_void_p, _c_void_p, _c_void_p, _c_void_p, _c_int, _c_void_p, _c_void_p, _c_int,
                            _c_void_p, _c_int, _c_void_p, _c_void_p, _c_void_p, _c_size_t, _c_void_p]),
     "oq_linear_noalloc": (_c_int, [_c_void_p, _c_void_p, _c_void_p, _c_void_p, _c_int, _c_void_p, _c_void_p,
@@ -204,6 +205,20 @@ def linear_codes(d, cb_a: Codebook, cb_w: Codebook, a_codes, a_norm, w_codes, w_
                                 _ptr(w_norm), N, _ptr(bias), EPILOGUES[epilogue], _ptr(out_f32), _ptr(out_bf16),
                                 _stream(stream)))
     return out_f32, out_bf16
+
+
+def row_flatness(X, rho3=None, rhoinf=None, batch_max=None, want_rows=True, stream=None):
+    """Flatness check of the rows of X (cuda bf16 [M, d]): per-row rho3 and
+    rhoinf (float [M] each, unless want_rows is False) and their batch maxima
+    (float [2])."""
+    M, d = X.shape
+    dev = X.device
+    if want_rows:
+        rho3 = torch.empty((M,), dtype=torch.float32, device=dev) if rho3 is None else rho3
+        rhoinf = torch.empty((M,), dtype=torch.float32, device=dev) if rhoinf is None else rhoinf
+    batch_max = torch.empty((2,), dtype=torch.float32, device=dev) if batch_max is None else batch_max
+    _check(_lib.oq_row_flatness(_ptr(X), M, d, _ptr(rho3), _ptr(rhoinf), _ptr(batch_max), _stream(stream)))
+    return rho3, rhoinf, batch_max
 
 
 def workspace_bytes(M: int, d: int, bits_a: int) -> int:

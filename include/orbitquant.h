@@ -220,6 +220,33 @@ OQ_API int oq_quantize_weight(oq_rpbh_t r, oq_codebook_t cb, const void* W, int 
                        void* stream);
 
 /* ---------------------------------------------------------------------------
+ * Flatness check of a batch of rows  ("Quantizing With Randomized Hadamard
+ * Transforms: Efficient Heuristic Now Proven", Methodology, adaptive
+ * verification, and Key contribution 4: an O(d) pass measuring the l3 norm
+ * (scalar quantization) and the l_inf norm (vector quantization) of the unit
+ * input, which tells whether one randomized Hadamard round suffices or the
+ * input needs the two or three rounds of oq_make_composed_rpbh)
+ *   rho3[m]   = sum_i |x_mi|^3 / (sum_i x_mi^2)^(3/2)
+ *   rhoinf[m] = max_i |x_mi| / (sum_i x_mi^2)^(1/2)
+ * Both are scale-free and lie in [d^-1/2, 1] (equal magnitudes .. one-hot);
+ * a zero row gives 0 and 0.  rho3 is the Berry-Esseen ratio of one
+ * randomized Hadamard coordinate of the row.  The page prints no thresholds:
+ * the choice of the round count is the caller's.  One rotation serves a whole
+ * layer, so the check reports the batch's maxima as well.
+ * X         : device bf16 [M][d], 16-byte aligned, d % 8 == 0, finite values.
+ * rho3, rhoinf : device float [M] each, or NULL (not written).
+ * batch_max : device float [2] = {max_m rho3, max_m rhoinf}, or NULL; the call
+ *             clears it on `stream` before the kernel runs (so it reads 0, 0
+ *             for M == 0).
+ * Outputs are fp32, from fp32 sums of exactly rescaled values (each row is
+ * divided by the power of two at its maximum first), so no finite bf16 row
+ * overflows or underflows.  One launch, HBM-bound (each row is read from
+ * memory once).  Errors: OQ_ERR_ARG (M < 0, NULL X with M > 0, no output),
+ * OQ_ERR_UNSUPPORTED (d), OQ_ERR_ALIGN.
+ * ------------------------------------------------------------------------- */
+OQ_API int oq_row_flatness(const void* X, int M, int d, float* rho3, float* rhoinf, float* batch_max, void* stream);
+
+/* ---------------------------------------------------------------------------
  * Codebook linear on codes  ([OQ] "Online Activation Quantization", last
  * paragraph: W^' x^' ~= W Pi^T Pi x = W x, no inverse rotation)
  *   y[m][n] = s_m r'_n sum_k v_a[ca[m][k]] v_w[cw[n][k]]  (+ bias_n) (-> GELU)

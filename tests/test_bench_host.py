@@ -51,3 +51,23 @@ def test_reference_arm_prints_contract_line():
                 "cpu_baseline", "e2e", "config"):
         assert key in line
     assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["cpu_baseline"]["kind"] == "oracle"
+
+
+@pytest.mark.parametrize("d,h,rounds", [(256, 64, 1), (512, 128, 2), (384, 128, 3), (1024, 256, 1)])
+def test_sweep_rotation_equals_the_oracle(d, h, rounds):
+    # the sweep's own fp64 torch rotation (used for its MSE figures) against the
+    # oracle's dense composed rotation, on the oracle's draws of the same seed
+    import numpy as np
+    import torch
+    sys.path.insert(0, ROOT)
+    import bench
+    from oracle import rpbh
+    R = rpbh.draw_rounds(0, d, rounds)
+    X = np.random.default_rng(d + rounds).standard_normal((7, d))
+    X[3] = 0.0
+    X[3, 11] = 2.0                              # a one-hot row
+    tables = [(torch.from_numpy(np.asarray(p, dtype=np.int64)), torch.from_numpy(np.asarray(s, dtype=np.float64)))
+              for p, s in R]
+    got = bench.rotate_rows_f64(torch.from_numpy(X), tables, h).numpy()
+    ref = rpbh.rotate_composed(X, R, h)
+    assert np.allclose(got, ref, rtol=0, atol=1e-12)

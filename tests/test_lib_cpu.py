@@ -209,3 +209,18 @@ def test_debug_switch(oq):
 def test_device_allocation_counter_is_exported(oq):
     # no device here, so nothing has been allocated; the counter never fails
     assert oq.device_allocations() == 0
+
+
+def test_row_flatness_argument_errors(oq):
+    # argument errors are found on the host, before any launch (no GPU here)
+    lib = oq.lib()
+    out = ctypes.c_void_p(16)
+    null = ctypes.c_void_p()
+    assert lib.oq_row_flatness(ctypes.c_void_p(16), -1, 256, out, out, out, null) == oq.OQ_ERR_ARG
+    assert lib.oq_row_flatness(ctypes.c_void_p(16), 4, 252, out, out, out, null) == oq.OQ_ERR_UNSUPPORTED
+    assert lib.oq_row_flatness(ctypes.c_void_p(16), 4, 0, out, out, out, null) == oq.OQ_ERR_UNSUPPORTED
+    assert lib.oq_row_flatness(null, 4, 256, out, out, out, null) == oq.OQ_ERR_ARG
+    assert lib.oq_row_flatness(ctypes.c_void_p(24), 4, 256, out, out, out, null) == oq.OQ_ERR_ALIGN
+    assert lib.oq_row_flatness(ctypes.c_void_p(16), 4, 256, null, null, null, null) == oq.OQ_ERR_ARG
+    assert lib.oq_row_flatness(ctypes.c_void_p(16), 4, 256, ctypes.c_void_p(18), null, null, null) == oq.OQ_ERR_ALIGN
+    assert "d % 8" in lib.oq_last_error().decode() or "aligned" in lib.oq_last_error().decode()
