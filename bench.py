@@ -460,7 +460,8 @@ def run_profile_case(args):
         an = torch.rand(M, device="cuda")
         wn = torch.rand(N, device="cuda").to(torch.bfloat16)
         y = torch.empty(M, N, device="cuda", dtype=torch.bfloat16)
-        run = lambda: oq.linear_codes(d, cba, cbw, a, an, w, wn, out_bf16=y, want_f32=False, want_bf16=True)
+        run = lambda: oq.linear_codes(d, cba, cbw, a, an, w, wn, epilogue=args.epilogue, out_bf16=y, want_f32=False,
+                                      want_bf16=True)
     for _ in range(args.warmup):
         run()
     torch.cuda.synchronize()
@@ -587,10 +588,19 @@ def run_workload(args):
     X = bf(inputs.activations(wl, M, d1))
     r1, r2 = oq.Rpbh(0, d1, h), oq.Rpbh(0, d2, h)
     ca1, cw1, ca2, cw2 = oq.Codebook(d1, ba), oq.Codebook(d1, bw), oq.Codebook(d2, ba), oq.Codebook(d2, bw)
-    w1c, w1n = oq.quantize_weight(r1, cw1, bf(inputs.weights(wl, inputs.T_W, d2, d1)))
+    W1 = bf(inputs.weights(wl, inputs.T_W, d2, d1))
+    w1c, w1n = oq.quantize_weight(r1, cw1, W1)
     w2c, w2n = oq.quantize_weight(r2, cw2, bf(inputs.weights(wl, inputs.T_W2, d1, d2)))
+    # fc2's permutation folded into fc1 (offline): W1's rows in the order pi_2,
+    # so fc1 emits P_2 GELU(.) and fc2's act-quant needs only blkdiag(H D_2),
+    # the Block-RHT handle of the same seed (same signs, no permutation)
+    perm2 = torch.from_numpy(r2.export()[0].astype(np.int64)).to(dev)
+    w1fc, w1fn = oq.quantize_weight(r1, cw1, W1[perm2].contiguous())
+    del W1
+    r2b = oq.Rpbh(0, d2, h, kind="block_rht")
     a1c, a1n = oq.quantize_act(r1, ca1, X)
     Y1 = torch.empty((M, d2), dtype=torch.bfloat16, device=dev)
+    Y1f = torch.empty((M, d2), dtype=torch.bfloat16, device=dev)
     a2c = torch.empty((M, d2 * ba // 8), dtype=torch.uint8, device=dev)
     a2n = torch.empty((M,), dtype=torch.float32, device=dev)
     Y2 = torch.empty((M, d1), dtype=torch.bfloat16, device=dev)
@@ -601,13 +611,22 @@ def run_workload(args):
         ("act_quant_2", lambda: oq.quantize_act(r2, ca2, Y1, a2c, a2n), "hbm", algorithmic(M, d2, d1, ba, bw)[0]),
         ("fc2", lambda: oq.linear_codes(d2, ca2, cw2, a2c, a2n, w2c, w2n, out_bf16=Y2, want_f32=False,
                                         want_bf16=True), "tensor", 2.0 * M * d1 * d2),
+        ("fc1_gelu_folded", lambda: oq.linear_codes(d1, ca1, cw1, a1c, a1n, w1fc, w1fn, epilogue="gelu",
+                                                    out_bf16=Y1f, want_f32=False, want_bf16=True),
+         "tensor", 2.0 * M * d1 * d2),
+        ("act_quant_2_folded", lambda: oq.quantize_act(r2b, ca2, Y1f, a2c, a2n), "hbm",
+         algorithmic(M, d2, d1, ba, bw)[0]),
     ]
     out = {"workload": args.workload, "M": M, "d_in": d1, "d_hidden": d2, "bits_w": bw, "bits_a": ba, "block": h,
            "kernels": {}, "peak_source": src}
     total = 0.0
+    folded = 0.0
     for name, fn, bound, work in steps:
         ms = _flush_and_time(fn, flush, args.steps, args.warmup)
-        total += ms
+        if name in ("act_quant_1", "fc2") or name.endswith("_folded"):
+            folded += ms
+        if not name.endswith("_folded"):
+            total += ms
         if bound == "hbm":
             ach = work / ms / 1e6
             out["kernels"][name] = {"ms": ms, "GB/s": ach, "frac": ach / peaks["hbm_gbs"]}
@@ -617,6 +636,8 @@ def run_workload(args):
     oq.device_status()
     out["step_ms"] = total
     out["TFLOP/s"] = 4.0 * M * d1 * d2 / total / 1e9
+    out["step_ms_folded_permutation"] = folded
+    out["TFLOP/s_folded_permutation"] = 4.0 * M * d1 * d2 / folded / 1e9
     print(json.dumps(out), flush=True)
     return 0
 
@@ -777,6 +798,7 @@ def main():
     ap.add_argument("--block", type=int, default=128)
     ap.add_argument("--bits-a", type=int, default=4)
     ap.add_argument("--bits-w", type=int, default=4)
+    ap.add_argument("--epilogue", choices=["none", "gelu"], default="none", help="GEMM epilogue for --profile gemm")
     args = ap.parse_args()
     if args.profile:
         return run_profile_case(args)

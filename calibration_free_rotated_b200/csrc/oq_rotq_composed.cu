@@ -12,10 +12,14 @@
 // One CTA works on one row pair at a time (persistent over pairs); thread g
 // owns coordinates 32 g .. 32 g + 31 of both rows, the layout the butterflies
 // and the search of the one-round kernel use:
-//   * the pair is loaded from global memory (128-bit loads) and written to a
-//     shared array of d 4-byte words, word j holding (x_a[j], x_b[j]) as bf16;
-//     a thread's 32 words form a 128-byte run whose 16-byte chunks are rotated
-//     by the thread index, so the 128-bit writes are free of bank conflicts;
+//   * the rows of the CTA's next pairs stream into a ring of shared-memory
+//     slots by 1-D bulk async copies with mbarrier transaction counts (two
+//     slots, one for the widest rows), so HBM latency overlaps the rounds of
+//     the pair at hand; a slot is refilled as soon as its pair is unpacked;
+//   * the pair is unpacked from its slot (128-bit loads) into a shared array
+//     of d 4-byte words, word j holding (x_a[j], x_b[j]) as bf16; a thread's
+//     32 words form a 128-byte run whose 16-byte chunks are rotated by the
+//     thread index, so the 128-bit writes are free of bank conflicts;
 //   * round 1 gathers those words (one 32-bit load feeds both rows) and widens
 //     them to f32 while flipping its signs; later rounds gather f32 pairs from
 //     a shared array F of d 8-byte slots (256-byte runs, rotated the same
@@ -45,8 +49,9 @@ struct ComposedArgs {
   const uint16_t* slots;  // [rounds][d]: slot that round r's coordinate j reads (round 1: 4-byte words)
   const uint32_t* signs;  // [rounds][d / 32]: sign words
   const uint32_t* qtable;
-  int M, d, rounds, pairs, qtable_len;
-  uint32_t qt_off, part_off;  // byte offsets in dynamic shared memory
+  int* status;
+  int M, d, rounds, pairs, qtable_len, stages;
+  uint32_t qt_off, part_off, bar_off, ring_off;  // byte offsets in dynamic shared memory
   float alpha;                // search multiplier / h^(rounds / 2)
   float nb;
 };
@@ -96,6 +101,30 @@ __device__ __forceinline__ void gather_round(unsigned long long (&v)[32], const 
   }
 }
 
+// Copies CTA-local pair k (rows 2 pk, 2 pk + 1 with pk = blockIdx + k grid)
+// into ring slot k % stages: lane 0 posts the byte count, lanes 0 and 1 issue
+// one row each.  Called by warp 0 only.
+__device__ __forceinline__ void issue_pair(const ComposedArgs& a, uint32_t ring, uint32_t bars, int k, int lane) {
+  const int pk = blockIdx.x + k * gridDim.x;
+  if (pk >= a.pairs) return;
+  const int slot = k % a.stages;
+  const int row = 2 * pk, nrows = min(2, a.M - row);
+  const uint32_t rowb = (uint32_t)a.d * 2u;
+  const uint32_t bar = bars + 8u * (uint32_t)slot;
+  if (lane == 0)
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"((uint32_t)nrows * rowb)
+                 : "memory");
+  __syncwarp();
+  if (lane < nrows) {
+    const uint32_t dst = ring + (uint32_t)slot * 2u * rowb + (uint32_t)lane * rowb;
+    const uint16_t* src = a.X + (size_t)(row + lane) * a.d;
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+        "l"(src), "r"(rowb), "r"(bar)
+        : "memory");
+  }
+}
+
 template <int BITS, int LOGHB>
 __global__ void __launch_bounds__(512, 1) rotq_composed_kernel(const __grid_constant__ ComposedArgs a) {
   extern __shared__ __align__(1024) unsigned char smem[];
@@ -109,28 +138,48 @@ __global__ void __launch_bounds__(512, 1) rotq_composed_kernel(const __grid_cons
   const uint32_t qkey = smem_u32(qtab) - 0x2D000000u;  // = qtab - 4 * bits(1.5 * 2^23)
   const uint32_t run = fbase + 256u * (uint32_t)tid, rot = (uint32_t)tid & 15u;
   const int nwarps = blockDim.x >> 5;
-  const size_t rowb = (size_t)a.d * 2;  // bytes of a bf16 row
+  const uint32_t rowb = (uint32_t)a.d * 2u;  // bytes of a bf16 row
+  const uint32_t ring = fbase + a.ring_off, bars = fbase + a.bar_off;
 
-  for (int pr = blockIdx.x; pr < a.pairs; pr += gridDim.x) {
+  if (tid == 0) {
+    for (int s = 0; s < a.stages; ++s)
+      asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(bars + 8u * (uint32_t)s) : "memory");
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 0) {  // the first pairs' copies start now, before the CTA barrier
+    __syncwarp();
+    for (int k = 0; k < a.stages; ++k) issue_pair(a, ring, bars, k, lane);
+  }
+  __syncthreads();  // barriers initialised and the search table loaded before any thread waits or reads
+
+  int it = 0;
+  for (int pr = blockIdx.x; pr < a.pairs; pr += gridDim.x, ++it) {
     const int row = 2 * pr;
     const bool has_b = row + 1 < a.M;
-    __syncthreads();  // the previous pair's readers of F and of the partials are done
+    const int slot = it % a.stages;
+    // the previous pair's readers of F and of the partials are done, and this
+    // pair's rows have landed (a give-up anywhere is agreed on and ends the CTA)
+    const bool ok = mbar_wait_bounded(bars + 8u * (uint32_t)slot, (uint32_t)(it / a.stages) & 1u, a.status);
+    if (__syncthreads_or(!ok)) return;
     if (active) {
-      const uint4* ra = reinterpret_cast<const uint4*>(reinterpret_cast<const unsigned char*>(a.X) + row * rowb) +
-                        4 * tid;
-      const uint4* rb = ra + rowb / 16;
+      const uint32_t ra = ring + (uint32_t)slot * 2u * rowb + 64u * (uint32_t)tid, rb = ra + rowb;
       const uint32_t run1 = fbase + 128u * (uint32_t)tid, rot1 = (uint32_t)tid & 7u;
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {  // 8 columns -> two 16-byte chunks of pair words
-        const uint4 A = ra[q];
-        const uint4 B = has_b ? rb[q] : make_uint4(0u, 0u, 0u, 0u);
-        sts_u128(run1 + ((((uint32_t)(2 * q)) ^ rot1) << 4), __byte_perm(A.x, B.x, 0x5410), __byte_perm(A.x, B.x, 0x7632),
+      for (int n = 0; n < 4; ++n) {  // 8 columns -> two 16-byte chunks of pair words
+        const uint32_t q = ((uint32_t)n + (uint32_t)tid) & 3u;  // rotated: 2-way conflicts at most
+        const uint4 A = lds_u128(ra + 16u * q);
+        const uint4 B = has_b ? lds_u128(rb + 16u * q) : make_uint4(0u, 0u, 0u, 0u);
+        sts_u128(run1 + (((2u * q) ^ rot1) << 4), __byte_perm(A.x, B.x, 0x5410), __byte_perm(A.x, B.x, 0x7632),
                  __byte_perm(A.y, B.y, 0x5410), __byte_perm(A.y, B.y, 0x7632));
-        sts_u128(run1 + ((((uint32_t)(2 * q + 1)) ^ rot1) << 4), __byte_perm(A.z, B.z, 0x5410),
-                 __byte_perm(A.z, B.z, 0x7632), __byte_perm(A.w, B.w, 0x5410), __byte_perm(A.w, B.w, 0x7632));
+        sts_u128(run1 + (((2u * q + 1u) ^ rot1) << 4), __byte_perm(A.z, B.z, 0x5410), __byte_perm(A.z, B.z, 0x7632),
+                 __byte_perm(A.w, B.w, 0x5410), __byte_perm(A.w, B.w, 0x7632));
       }
     }
-    __syncthreads();
+    __syncthreads();  // pair words ready; the ring slot is free
+    if (warp == 0) {
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      issue_pair(a, ring, bars, it + a.stages, lane);
+    }
 
     unsigned long long v[32];
     unsigned long long sq[4] = {0ull, 0ull, 0ull, 0ull};
@@ -266,14 +315,26 @@ int launch_rotq_composed(oq_rpbh_t r, oq_codebook_t cb, const void* X, int M, ui
   a.rounds = r->rounds;
   a.pairs = (M + 1) / 2;
   a.qtable_len = qlen;
+  int* status;
+  if (int rc = device_status_word(&status)) return rc;
+  a.status = status;
   a.qt_off = (uint32_t)threads * 256u;  // F: one 256-byte run per thread (round 1 uses the first half)
   a.part_off = (a.qt_off + 4u * (uint32_t)qlen + 15u) & ~15u;
+  a.bar_off = (a.part_off + (uint32_t)(threads / 32) * 8u + 15u) & ~15u;
+  a.ring_off = (a.bar_off + 16u + 127u) & ~127u;
+  // Ring slots of a row pair each: two where the second costs no resident CTA
+  // (the kernel is bound by its rounds, so residency matters more than depth).
+  const uint32_t slot_bytes = 4u * (uint32_t)d;
+  const size_t smem1 = (size_t)a.ring_off + slot_bytes, smem2 = smem1 + slot_bytes;
+  int occ1 = 0, occ2 = 0;
+  if (int rc = occupancy(reinterpret_cast<const void*>(kern), (int)smem1, threads, 0, &occ1)) return rc;
+  if (smem2 <= 200u * 1024u)
+    if (int rc = occupancy(reinterpret_cast<const void*>(kern), (int)smem2, threads, 0, &occ2)) return rc;
+  a.stages = occ2 >= occ1 && occ2 > 0 ? 2 : 1;
   a.alpha = (float)((double)cb->qt_alpha / std::pow((double)h, 0.5 * r->rounds));
   a.nb = (float)cb->qt_nb;
-  const size_t smem = a.part_off + (size_t)(threads / 32) * 8;
-
-  int per_sm = 0;
-  if (int rc = occupancy(reinterpret_cast<const void*>(kern), (int)smem, threads, 0, &per_sm)) return rc;
+  const size_t smem = a.stages == 2 ? smem2 : smem1;
+  const int per_sm = a.stages == 2 ? occ2 : occ1;
   if (per_sm < 1) return fail(OQ_ERR_UNSUPPORTED, "composed rotate+quantize kernel does not fit (d=%d)", d);
   const int grid = std::min(a.pairs, nsm * per_sm);
   kern<<<grid, threads, smem, (cudaStream_t)stream>>>(a);

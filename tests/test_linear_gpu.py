@@ -439,3 +439,55 @@ def test_full_layer_replays_from_a_cuda_graph(oq, codebooks):
         torch.cuda.synchronize()
         oq.device_status()
         assert torch.equal(y16, ref)
+
+
+@pytest.mark.parametrize("wl,M,d1,d2,bw,ba", [(3, 4608, 3072, 12288, 2, 4), (4, 3001, 1536, 8960, 4, 6)])
+def test_fc2_permutation_folded_into_fc1(oq, codebooks, wl, M, d1, d2, bw, ba):
+    # Partial fc1 -> fc2 fusion by reparametrisation: W1's rows (one per fc1
+    # output) taken in the order pi_2 of fc2's rotation, so fc1 emits
+    # P_2 GELU(.) directly; GELU and bf16 rounding act elementwise, so this is
+    # the unfused fc1 output with its columns permuted.  fc2's act-quant then
+    # needs blkdiag(H_h D_2) only: the Block-RHT handle of the same seed, with
+    # the same signs and no permutation.  The codes, norms and fc2 output must
+    # equal the unfused chain's bit for bit (FLUX MLP at full size, Wan FFN on
+    # 3001 tokens); the folded fc2 is also checked against the oracle.
+    h = 128
+    X = _dev_bf16(inputs.activations(wl, M, d1))
+    W1 = _dev_bf16(inputs.weights(wl, inputs.T_W, d2, d1))
+    W2b = inputs.weights(wl, inputs.T_W2, d1, d2)
+    r1, r2 = oq.Rpbh(0, d1, h), oq.Rpbh(0, d2, h)
+    r2b = oq.Rpbh(0, d2, h, kind="block_rht")
+    ca1, cw1, ca2, cw2 = _lib_cb(oq, d1, ba), _lib_cb(oq, d1, bw), _lib_cb(oq, d2, ba), _lib_cb(oq, d2, bw)
+    perm2 = torch.from_numpy(r2.export()[0].astype(np.int64)).cuda()
+    w1c, w1n = oq.quantize_weight(r1, cw1, W1)
+    w1fc, w1fn = oq.quantize_weight(r1, cw1, W1[perm2].contiguous())
+    w2c, w2n = oq.quantize_weight(r2, cw2, _dev_bf16(W2b))
+    _, y1 = oq.linear(r1, ca1, cw1, X, w1c, w1n, epilogue="gelu", want_f32=False, want_bf16=True)
+    _, y1f = oq.linear(r1, ca1, cw1, X, w1fc, w1fn, epilogue="gelu", want_f32=False, want_bf16=True)
+    c2, n2 = oq.quantize_act(r2, ca2, y1)
+    c2f, n2f = oq.quantize_act(r2b, ca2, y1f)
+    y2, _ = oq.linear_codes(d2, ca2, cw2, c2, n2, w2c, w2n)
+    y2f, _ = oq.linear_codes(d2, ca2, cw2, c2f, n2f, w2c, w2n)
+    torch.cuda.synchronize()
+    oq.device_status()
+    assert torch.equal(y1f, y1[:, perm2])
+    assert torch.equal(c2f, c2) and torch.equal(n2f, n2)
+    assert torch.equal(y2f, y2)
+    # the folded fc2 layer against the oracle on sampled rows; its input is the
+    # oracle's own bf16 fc1 output, in the folded column order
+    rows = np.linspace(0, M - 1, 8).astype(int)
+    Xb = inputs.activations(wl, M, d1)[rows]
+    ca, s = _oracle_act(codebooks, Xb, d1, h, ba)
+    cw1o, r1o = _oracle_weight(codebooks, inputs.weights(wl, inputs.T_W, d2, d1), d1, h, bw)
+    h1 = inputs.to_bf16_bits(olin.linear_from_codes(ca, s, cw1o, r1o, codebooks(d1, ba)["centroids"],
+                                                     codebooks(d1, bw)["centroids"], d1, gelu=True))
+    p2 = perm2.cpu().numpy()
+    h1f = h1[:, p2]                                  # what the folded fc1 emits for these rows
+    c2o, s2o = _oracle_act(codebooks, h1, d2, h, ba)  # the oracle's fc2 input codes (unfolded, RPBH)
+    cw2o, r2o = _oracle_weight(codebooks, W2b, d2, h, bw)
+    ref = olin.linear_from_codes(c2o, s2o, cw2o, r2o, codebooks(d2, ba)["centroids"], codebooks(d2, bw)["centroids"],
+                                 d2)
+    gc, gn = oq.quantize_act(r2b, ca2, _dev_bf16(h1f))
+    got, _ = oq.linear_codes(d2, ca2, cw2, gc, gn, w2c, w2n)
+    torch.cuda.synchronize()
+    assert _rel_fro(got.cpu().double().numpy(), ref) <= TOL
