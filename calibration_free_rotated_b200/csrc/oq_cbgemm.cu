@@ -661,6 +661,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   uint16_t* lut_a_s = reinterpret_cast<uint16_t*>(smem + S::kLut);
   uint16_t* lut_w_s = lut_a_s + 64;
 
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");  // the next kernel may launch
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t rank = PAIR ? cluster_ctarank() : 0u;   // 0 = leader (issues the MMAs)
   const int unit = PAIR ? (int)(blockIdx.x >> 1) : (int)blockIdx.x;
@@ -705,6 +706,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   if constexpr (PAIR) cluster_sync(); else __syncthreads();   // barriers initialised in both CTAs
   tc_fence_after();
   const uint32_t tmem_base = *tmem_holder;
+  // The set-up above overlaps the previous kernel in the stream (programmatic
+  // dependent launch); the codes, norms and bias may be its outputs, and Y
+  // may be its input: wait for it to complete before any global access.
+  asm volatile("griddepcontrol.wait;" ::: "memory");
 
   const int KB = args.K / BK;
   const int num_tiles = args.num_tiles;
@@ -1143,18 +1148,21 @@ int launch_t(GemmArgs& a, const uint8_t* a_codes, const uint8_t* w_codes, int ns
   a.num_tiles = a.tiles_m * ((a.N + BN - 1) / BN);
   cudaLaunchConfig_t cfg;
   memset(&cfg, 0, sizeof(cfg));
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   cfg.blockDim = dim3(NUM_THREADS, 1, 1);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = stream;
+  cfg.attrs = attr;
   int units = std::min(a.num_tiles, nsm);
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.numAttrs = pdl_enabled() ? 1 : 0;
   if (PAIR) {
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = 2;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    attr[cfg.numAttrs].id = cudaLaunchAttributeClusterDimension;
+    attr[cfg.numAttrs].val.clusterDim.x = 2;
+    attr[cfg.numAttrs].val.clusterDim.y = 1;
+    attr[cfg.numAttrs].val.clusterDim.z = 1;
+    cfg.numAttrs += 1;
     int max_clusters = 0;
     if (int rc = occupancy(reinterpret_cast<const void*>(k), smem, NUM_THREADS, 2, &max_clusters)) return rc;
     if (max_clusters < 1) return fail(OQ_ERR_UNSUPPORTED, "no CTA pair of the GEMM fits on this device");

@@ -355,6 +355,14 @@ TmapEntry g_tmap[kTmapSlots];
 int g_tmap_used = 0, g_tmap_next = 0;
 }  // namespace
 
+bool pdl_enabled() {
+  static const bool on = [] {
+    const char* e = std::getenv("OQ_NO_PDL");
+    return !(e && e[0] == '1');
+  }();
+  return on;
+}
+
 int occupancy(const void* kernel, int smem, int threads, int cluster, int* value) {
   int dev;
   if (int rc = current_device(&dev)) return rc;

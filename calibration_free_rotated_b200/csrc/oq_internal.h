@@ -80,6 +80,15 @@ int take_test_stall(int kernel);
 // Steady-state launches therefore make no attribute or occupancy calls.
 int occupancy(const void* kernel, int smem, int threads, int cluster, int* value);
 
+// Programmatic dependent launch (oq_host.cpp): whether launches carry the
+// programmatic-serialisation attribute (on unless OQ_NO_PDL=1 is set).  A
+// kernel so launched may start while the previous kernel in the stream
+// finishes; it runs `griddepcontrol.wait` before it touches memory that an
+// earlier kernel may write or read, and `griddepcontrol.launch_dependents`
+// at its start.  Every grid of this library is persistent and fully resident,
+// so the overlap cannot deadlock.
+bool pdl_enabled();
+
 // Encoded 2-D tensor maps cached by everything that defines them (base
 // address, sizes, strides, box, element type, swizzle, promotion); a launch on
 // the same buffers reuses the encoding instead of re-encoding.  `encode`

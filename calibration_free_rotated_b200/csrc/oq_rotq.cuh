@@ -44,6 +44,11 @@ struct Cfg {
   static constexpr int STAGES = CFG == 2 ? 1 : 2;  // ring slots (compile-time: slot and phase are shifts)
 };
 
+// Programmatic dependent launch: let the next kernel in the stream launch, and
+// wait until the previous one has completed (no-ops without the attribute).
+__device__ __forceinline__ void pdl_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
@@ -634,6 +639,7 @@ __device__ __forceinline__ void quantize(const Args& a, const Thread& t, int it,
 template <int BITS, int LOGHB, int CFG, bool PERM>
 __global__ void __launch_bounds__(CFG == 2 ? 512 : 384, 1) rotq_kernel(const __grid_constant__ Args a) {
   extern __shared__ __align__(1024) unsigned char smem[];
+  pdl_launch_dependents();
   const int d = a.d, P = a.P;
   Thread t;
   t.tid = threadIdx.x;
@@ -665,8 +671,12 @@ __global__ void __launch_bounds__(CFG == 2 ? 512 : 384, 1) rotq_kernel(const __g
   }
   // The first stages' copies start now, so their HBM latency overlaps the
   // table loads below (only warp 0, which made the barriers, touches them
-  // before the CTA barrier).
+  // before the CTA barrier).  X may be written by the previous kernel in the
+  // stream, and the codes and norms read by it: warp 0 waits for that kernel
+  // first (every other thread's global accesses before the CTA barrier are
+  // to the handles' tables; its writes come after data that warp 0 requested).
   if (warp == 0) {
+    pdl_wait();
     __syncwarp();
     for (int s = 0; s < Cfg<CFG>::STAGES; ++s) issue_stage_load<CFG>(a, t.s_ring, t.s_bars, s, t.lane);
   }
