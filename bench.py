@@ -5,6 +5,11 @@ norm-rescale + bias epilogue, on the FLUX-like attention projection
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
+The value is timed over K steps with events only at the ends of the region;
+the per-kernel split behind the roofline fields comes from a second region of K
+steps with events around each kernel (those events keep the two kernels from
+overlapping, so that region runs slower; its step time is reported too).
+
 Prints ONE JSON line (rank 0).  Multi-GPU (torchrun, one rank per GPU): every
 rank runs its own copy of the workload (the path is row-parallel with no
 exchange), timing is the max over ranks, value is the whole-job throughput.
@@ -315,8 +320,14 @@ def run_ours(args, world, rank, local):
     torch.cuda.synchronize()
     oq.device_status()
 
+    # Two timed regions of K steps each.  (1) The value: events only at its two
+    # ends, so consecutive kernels stay adjacent in the stream (a user's layer
+    # sequence; programmatic dependent launch overlaps them).  (2) The kernel
+    # split for the roofline: an event before, between and after the two
+    # kernels of every step (which serialises them).
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    start2, end2 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     if world > 1:
         import torch.distributed as dist
         dist.barrier()
@@ -324,16 +335,25 @@ def run_ours(args, world, rank, local):
     with ClockSampler(torch.cuda.current_device()) as clk:
         start.record(stream)
         for i in range(args.steps):
-            step(i, evs[i])
+            step(i)
         end.record(stream)
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+        start2.record(stream)
+        for i in range(args.steps):
+            step(i, evs[i])
+        end2.record(stream)
         torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
     oq.device_status()
     total_s = start.elapsed_time(end) / 1e3
+    split_s = start2.elapsed_time(end2) / 1e3
     k1 = [e[0].elapsed_time(e[1]) / 1e3 for e in evs]
     k2 = [e[1].elapsed_time(e[2]) / 1e3 for e in evs]
-    total_s, k1_avg, k2_avg = reduce_max([total_s, sum(k1) / len(k1), sum(k2) / len(k2)], world)
+    total_s, split_s, k1_avg, k2_avg = reduce_max([total_s, split_s, sum(k1) / len(k1), sum(k2) / len(k2)], world)
 
     aq_bytes, flops = algorithmic(M, K, N, 4, 4)
     value = whole_job_value(flops * args.steps, world, total_s) / 1e12
@@ -412,9 +432,14 @@ def run_ours(args, world, rank, local):
                                "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": aq_gbs / peaks["hbm_gbs"],
                                "traffic": aq_traffic, "peak_source": f"{peak_kind} copy bandwidth",
                                "algorithmic_per_launch": aq_bytes},
-        "kernel_ms": {"rotq_kernel": 1e3 * k1_avg, "cbgemm_kernel": 1e3 * k2_avg},
+        "kernel_ms": {"rotq_kernel": 1e3 * k1_avg, "cbgemm_kernel": 1e3 * k2_avg,
+                      "region": "a second timed region of K steps with an event before, between and after the two "
+                                "kernels of every step",
+                      "ms_per_step_with_kernel_events": 1e3 * split_s / args.steps},
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": M * K * 2, "d2h_bytes_per_step": M * N * 2},
         "gpu_launches": 2 * args.steps,
+        "timing": "value: K steps between two events (kernels adjacent in the stream); kernel_ms: a second region of "
+                  "K steps with per-kernel events",
         "clocks": clk.summary(),
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -453,6 +478,10 @@ def run_profile_case(args):
         X = torch.randn(M, d, device="cuda").to(torch.bfloat16)
         codes, norms = oq.quantize_act(r, cb, X)
         run = lambda: oq.quantize_act(r, cb, X, codes, norms)
+    elif args.profile == "flatness":
+        X = torch.randn(M, d, device="cuda").to(torch.bfloat16)
+        r3, ri, bm = oq.row_flatness(X)
+        run = lambda: oq.row_flatness(X, r3, ri, bm)
     else:
         cba, cbw = oq.Codebook(d, args.bits_a), oq.Codebook(d, args.bits_w)
         a = torch.randint(0, 256, (M, d * args.bits_a // 8), dtype=torch.uint8, device="cuda")
@@ -479,6 +508,8 @@ def run_profile_case(args):
            "median_ms": ms}
     if args.profile == "rotq":
         out["GB/s"] = algorithmic(M, d, N, args.bits_a, args.bits_w)[0] / ms / 1e6
+    elif args.profile == "flatness":
+        out["GB/s"] = (2.0 * M * d + 8.0 * M + 8) / ms / 1e6
     else:
         out["TFLOP/s"] = algorithmic(M, d, N, args.bits_a, args.bits_w)[1] / ms / 1e9
     print(json.dumps(out))
@@ -526,6 +557,52 @@ def run_ablation(args):
                               "d": d, "bits": 4,
                               "median_us": 1e3 * ms, "GB/s": gbs, "frac_hbm": gbs / peaks["hbm_gbs"],
                               "peak_source": src}), flush=True)
+    return 0
+
+
+def run_ablation_steps(args):
+    """Back-to-back steps of the bench workload (act-quant + GEMM, bf16 out) with
+    CUDA events only at the two ends of the timed region, so that consecutive
+    kernels stay adjacent in the stream and programmatic dependent launch can
+    overlap them (the contract line's per-kernel events serialise them).  Run it
+    once as is and once with OQ_NO_PDL=1 to compare.  One JSON line."""
+    import torch
+    from calibration_free_rotated_b200 import build
+    build.build()
+    from calibration_free_rotated_b200 import inputs
+    from calibration_free_rotated_b200 import orbitquant as oq
+    w = WORKLOAD
+    M, K, N, h = w["M"], w["K"], w["N"], w["block"]
+    dev = torch.device("cuda")
+    bf = lambda bits: torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).to(dev).view(torch.bfloat16)
+    r, cb = oq.Rpbh(w["seed"], K, h), oq.Codebook(K, 4)
+    X0 = bf(inputs.activations(2, M, K))
+    wc0, wn = oq.quantize_weight(r, cb, bf(inputs.weights(2, inputs.T_W, N, K)))
+    bias = bf(inputs.bias(2, N))
+    sets = [dict(X=X0.clone(), wc=wc0.clone(), codes=torch.empty((M, K // 2), dtype=torch.uint8, device=dev),
+                 norms=torch.empty((M,), device=dev), Y=torch.empty((M, N), dtype=torch.bfloat16, device=dev))
+            for _ in range(N_SETS)]
+    stream = torch.cuda.current_stream()
+
+    def step(i):
+        s = sets[i % N_SETS]
+        oq.quantize_act(r, cb, s["X"], s["codes"], s["norms"], stream=stream)
+        oq.linear_codes(K, cb, cb, s["codes"], s["norms"], s["wc"], wn, bias=bias, out_bf16=s["Y"], want_f32=False,
+                        want_bf16=True, stream=stream)
+
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for i in range(args.steps):
+        step(i)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    oq.device_status()
+    ms = e0.elapsed_time(e1) / args.steps
+    print(json.dumps({"ablation": "steps", "pdl": os.environ.get("OQ_NO_PDL", "0") != "1", "ms_per_step": ms,
+                      "TFLOP/s": 2.0 * M * N * K / ms / 1e9, "steps": args.steps}), flush=True)
     return 0
 
 
@@ -784,8 +861,10 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-parity", action="store_true", help="skip the sampled-row parity check of the bench line")
-    ap.add_argument("--profile", choices=["rotq", "gemm"], help="launch one kernel only (for ncu captures)")
-    ap.add_argument("--ablation", choices=["rotation"], help="time the rotation variants of the ablation table")
+    ap.add_argument("--profile", choices=["rotq", "gemm", "flatness"], help="launch one kernel only (for ncu captures)")
+    ap.add_argument("--ablation", choices=["rotation", "steps"],
+                    help="rotation: the rotation variants of the ablation table; steps: back-to-back steps without "
+                         "per-kernel events (programmatic dependent launch on, or off with OQ_NO_PDL=1)")
     ap.add_argument("--workload", choices=["flux_mlp", "wan_ffn", "flux_qkv_w3a3"],
                     help="per-kernel times of a layer workload")
     ap.add_argument("--sweep", action="store_true", help="the rotate+quantize sweep with empirical MSE")
@@ -802,6 +881,8 @@ def main():
     args = ap.parse_args()
     if args.profile:
         return run_profile_case(args)
+    if args.ablation == "steps":
+        return run_ablation_steps(args)
     if args.ablation:
         return run_ablation(args)
     if args.workload:
