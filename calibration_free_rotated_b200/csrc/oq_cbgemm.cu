@@ -514,11 +514,6 @@ __device__ __forceinline__ unsigned long long f2_fma(unsigned long long a, unsig
   return r;
 }
 
-__device__ __forceinline__ unsigned long long f2_add(unsigned long long a, unsigned long long b) {
-  unsigned long long r;
-  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
-  return r;
-}
 __device__ __forceinline__ float rcp_approx(float x) {
   float r;
   asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));
@@ -531,35 +526,36 @@ __device__ __forceinline__ float ex2_approx(float x) {
 }
 
 // GELU (exact erf form) of two values:  GELU(y) = y Phi(y),
-// Phi(y) = (1 + erf(y / sqrt 2)) / 2.  erf is the rational approximation of
-// Abramowitz & Stegun, Handbook of Mathematical Functions, 7.1.26 (Hastings):
-//   erf(x) = 1 - t (a1 + t (a2 + t (a3 + t (a4 + t a5)))) exp(-x^2),
+// Phi(y) = (1 + erf(y / sqrt 2)) / 2, computed as
+//   y Phi(y) = relu(y) - |y| (1 - erf(|y| / sqrt 2)) / 2
+// (no sign restore, no cancellation in either tail).  1 - erf is the rational
+// approximation of Abramowitz & Stegun, Handbook of Mathematical Functions,
+// 7.1.26 (Hastings):
+//   1 - erf(x) = t (a1 + t (a2 + t (a3 + t (a4 + t a5)))) exp(-x^2),
 //   t = 1 / (1 + p x),  x >= 0,  |error| <= 1.5e-7,
-// with x = |y| / sqrt 2 folded into p and the exponent, and the halving of
-// Phi folded into the a_i.  Branch-free, packed f32x2 except the two
-// reciprocals and exponentials; large |y| gives exp -> 0 and Phi -> 0 or 1.
+// with x = |y| / sqrt 2 folded into p and the exponent, and the factor -1/2
+// folded into the a_i.  Branch-free, packed f32x2 except the two reciprocals,
+// exponentials and maxima; large |y| gives exp -> 0.
 __device__ __forceinline__ unsigned long long gelu2(unsigned long long y) {
   constexpr float kP = 0.3275911f * 0.70710678118654752f;  // p / sqrt 2
-  constexpr float kA1 = 0.5f * 0.254829592f, kA2 = 0.5f * -0.284496736f, kA3 = 0.5f * 1.421413741f,
-                  kA4 = 0.5f * -1.453152027f, kA5 = 0.5f * 1.061405429f;
+  constexpr float kA1 = -0.5f * 0.254829592f, kA2 = -0.5f * -0.284496736f, kA3 = -0.5f * 1.421413741f,
+                  kA4 = -0.5f * -1.453152027f, kA5 = -0.5f * 1.061405429f;
   constexpr float kE = -0.72134752044448170f;  // -log2(e) / 2: exp(-y^2/2) = 2^(kE y^2)
   float y0, y1;
   f2_unpack(y, y0, y1);
+  const unsigned long long ay = f2_pack(fabsf(y0), fabsf(y1));
   float d0, d1;
-  f2_unpack(f2_fma(f2_pack(fabsf(y0), fabsf(y1)), f2_pack(kP, kP), f2_pack(1.0f, 1.0f)), d0, d1);
+  f2_unpack(f2_fma(ay, f2_pack(kP, kP), f2_pack(1.0f, 1.0f)), d0, d1);
   const unsigned long long t = f2_pack(rcp_approx(d0), rcp_approx(d1));
   unsigned long long q = f2_fma(t, f2_pack(kA5, kA5), f2_pack(kA4, kA4));
   q = f2_fma(q, t, f2_pack(kA3, kA3));
   q = f2_fma(q, t, f2_pack(kA2, kA2));
   q = f2_fma(q, t, f2_pack(kA1, kA1));
-  q = f2_mul(q, t);  // (1 - erf(|y| / sqrt 2)) / 2 before the Gaussian factor
+  q = f2_mul(q, t);  // -(1 - erf(|y| / sqrt 2)) / 2 before the Gaussian factor
   float w0, w1;
   f2_unpack(f2_mul(y, f2_mul(y, f2_pack(kE, kE))), w0, w1);
   q = f2_mul(q, f2_pack(ex2_approx(w0), ex2_approx(w1)));
-  float m0, m1;  // erf(|y| / sqrt 2) / 2, then given the sign of y
-  f2_unpack(f2_fma(q, f2_pack(-1.0f, -1.0f), f2_pack(0.5f, 0.5f)), m0, m1);
-  const unsigned long long phi = f2_add(f2_pack(copysignf(m0, y0), copysignf(m1, y1)), f2_pack(0.5f, 0.5f));
-  return f2_mul(y, phi);
+  return f2_fma(ay, q, f2_pack(fmaxf(y0, 0.0f), fmaxf(y1, 0.0f)));
 }
 
 __device__ __forceinline__ float bf16_to_f32(uint16_t v) { return __uint_as_float((uint32_t)v << 16); }
