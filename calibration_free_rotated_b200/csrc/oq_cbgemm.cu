@@ -26,6 +26,9 @@
 //                finished accumulator.
 //   warps 16..19 epilogue: tcgen05.ld of the accumulator (each warp its 32-lane
 //                quadrant), rescale, bias, GELU, fp32/bf16 stores.
+//   (GELU tiles of short K with bf16 output: three converter groups, warps
+//   0..11, and eight epilogue warps, 12..19, two per quadrant, that split the
+//   tile's columns between them.)
 // Keeping A in TMEM removes A's expanded stores and tensor-core reads from
 // shared memory, whose bandwidth otherwise caps the kernel near 2/3 of the
 // tensor rate.  TMEM: one 256-column fp32 accumulator plus 4 A stages of 32
@@ -47,18 +50,29 @@ namespace oq {
 namespace {
 
 constexpr int BM = 128, BN = 256, BK = 64;  // per-CTA A rows, tile N, K step
-constexpr int NUM_GROUPS = 4;                // converter groups; group g expands k-steps g, g+4, ...
 constexpr int GROUP_WARPS = 4;               // one warp per SM sub-partition and TMEM lane quarter
-constexpr int NUM_CONV_WARPS = NUM_GROUPS * GROUP_WARPS;  // warps 0..15
-constexpr int ESTAGES = NUM_GROUPS;          // expanded ring: stage g belongs to group g
-constexpr int EPI_WARP0 = 16;
 constexpr int TMA_WARP = 20;
 constexpr int MMA_WARP = 21;
 constexpr int NUM_THREADS = 22 * 32;
 constexpr int TMEM_COLS = 512;
 constexpr int A_COL0 = BN;                   // A stage s: TMEM columns A_COL0 + 32 s .. + 31
-constexpr int SPARE_COL = A_COL0 + 32 * ESTAGES;  // the last 128 columns: epilogue spill area
-static_assert(SPARE_COL + BN / 2 == TMEM_COLS, "TMEM plan");
+
+// Warp roles for NG converter groups (group g expands k-steps g, g + NG, ...):
+// warps 0 .. 4 NG - 1 convert, the next 20 - 4 NG run the epilogue (four, one
+// per TMEM lane quarter, for NG = 4; eight, two per quarter, for NG = 3), warp
+// 20 is the TMA producer and warp 21 issues the MMAs.  NG = 3 is for GELU
+// tiles with short K, where the epilogue's arithmetic, not the converters,
+// paces the tiles.
+template <int NG>
+struct Roles {
+  static_assert(NG == 3 || NG == 4, "converter groups");
+  static constexpr int CONV_WARPS = NG * GROUP_WARPS;
+  static constexpr int EPI_WARP0 = CONV_WARPS;
+  static constexpr int NEPI = TMA_WARP - EPI_WARP0;
+  static constexpr int ESTAGES = NG;                     // expanded ring: stage g belongs to group g
+  static constexpr int SPARE_COL = A_COL0 + 32 * ESTAGES;  // 128 columns: epilogue spill area
+  static_assert(SPARE_COL + BN / 2 <= TMEM_COLS, "TMEM plan");
+};
 constexpr unsigned long long kWaitLimitNs = 1000000000ull;
 
 struct GemmArgs {
@@ -97,8 +111,9 @@ struct PackedUnit {
 // ---- shared memory plan (offsets from a 1024-aligned base) -------------------
 // PAIR: two CTAs of a cluster share one 256 x 256 tile (cta_group::2); each holds
 // 128 rows of A and 128 of the 256 B rows.  Otherwise one CTA owns 128 x 256.
-template <int BA, int BW, bool PAIR>
+template <int BA, int BW, bool PAIR, int NG = 4>
 struct Smem {
+  static constexpr int ESTAGES = Roles<NG>::ESTAGES;
   static constexpr int kBnCta = PAIR ? BN / 2 : BN;
   static constexpr int kExpBBytes = kBnCta * BK * 2;
   static constexpr int kPkA = BM * PackedUnit<BA, BW>::kRowA;
@@ -108,14 +123,19 @@ struct Smem {
   // bytes that do not depend on the ring depth or the output staging
   static constexpr int kFixed = ESTAGES * kExpBBytes + 256 + 4 * 2 * BN * 4 + 512 + 16 + 1024;
   static constexpr int kBudget = 227 * 1024;
-  // Packed ring: 8 stages (two per group) where they fit, else 4. Output staging:
-  // 128 rows x 128-byte swizzled blocks of 16 KB (64 bf16 or 32 fp32 columns).
-  static constexpr int kPS = kFixed + 8 * (kPkAStride + kPkBStride) + (PAIR ? 4 : 2) * 16384 <= kBudget ? 8 : 4;
-  static constexpr int kRest = kBudget - kFixed - kPS * (kPkAStride + kPkBStride);
+  // Packed ring: 8 stages (two per group) where they fit, else 4 (always 4 for
+  // NG = 3, whose second epilogue half has two staging blocks of its own).
+  // Output staging: 128 rows x 128-byte swizzled blocks of 16 KB (64 bf16 or
+  // 32 fp32 columns).
+  static constexpr int kXtraBlocks = NG == 3 ? 2 : 0;
+  static constexpr int kPS =
+      NG == 4 && kFixed + 8 * (kPkAStride + kPkBStride) + (PAIR ? 4 : 2) * 16384 <= kBudget ? 8 : 4;
+  static constexpr int kRest = kBudget - kFixed - kPS * (kPkAStride + kPkBStride) - kXtraBlocks * 16384;
   static constexpr int kStageBlocks = (PAIR && kRest >= 4 * 16384) ? 4 : (kRest >= 2 * 16384 ? 2 : 1);
+  static_assert(NG == 4 || (PAIR && kStageBlocks == 4), "the split epilogue needs four staging blocks");
   static constexpr int kExpB = 0;
   static constexpr int kStage = kExpB + ESTAGES * kExpBBytes;
-  static constexpr int kPackA = kStage + kStageBlocks * 16384;
+  static constexpr int kPackA = kStage + (kStageBlocks + kXtraBlocks) * 16384;
   static constexpr int kPackB = kPackA + kPS * kPkAStride;
   static constexpr int kLut = kPackB + kPS * kPkBStride;
   static constexpr int kEpi = kLut + 256;                 // 4 warps x (r'[256], bias[256]) floats
@@ -590,19 +610,19 @@ __device__ __forceinline__ uint4 epi8_bf16(const uint32_t* v, const float* col_r
   return make_uint4(o[0], o[1], o[2], o[3]);
 }
 
-// Named barrier 1 over the four epilogue warps.
-__device__ __forceinline__ void epi_bar() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+// Named barrier `id` over four epilogue warps (one epilogue group: ids 1, 2).
+__device__ __forceinline__ void epi_bar(uint32_t id = 1) { asm volatile("bar.sync %0, 128;" ::"r"(id) : "memory"); }
 
-// True in every epilogue thread if `p` holds in any of them (named barrier 1).
-__device__ __forceinline__ bool epi_any(bool p) {
+// True in every thread of the epilogue group if `p` holds in any of them.
+__device__ __forceinline__ bool epi_any(bool p, uint32_t id = 1) {
   uint32_t r;
   asm volatile(
       "{\n\t.reg .pred a, b;\n\t"
       "setp.ne.u32 a, %1, 0;\n\t"
-      "bar.red.or.pred b, 1, 128, a;\n\t"
+      "bar.red.or.pred b, %2, 128, a;\n\t"
       "selp.u32 %0, 1, 0, b;\n\t}"
       : "=r"(r)
-      : "r"((uint32_t)p)
+      : "r"((uint32_t)p), "r"(id)
       : "memory");
   return r != 0;
 }
@@ -639,12 +659,14 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t* v) {
       : "r"(taddr));
 }
 
-template <int BA, int BW, bool PAIR>
+template <int BA, int BW, bool PAIR, int NG>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     cbgemm_kernel(const __grid_constant__ GemmArgs args, const __grid_constant__ CUtensorMap map_a,
                   const __grid_constant__ CUtensorMap map_b, const __grid_constant__ CUtensorMap map_y16,
                   const __grid_constant__ CUtensorMap map_y32) {
-  using S = Smem<BA, BW, PAIR>;
+  using S = Smem<BA, BW, PAIR, NG>;
+  using R = Roles<NG>;
+  constexpr int ESTAGES = R::ESTAGES;
   constexpr int BN_CTA = S::kBnCta;
   constexpr int TILE_M = PAIR ? 2 * BM : BM;
   constexpr uint32_t NCTA = PAIR ? 2 : 1;
@@ -677,7 +699,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       mbar_init(bar(EX_EMPTY + s), 1);
     }
     mbar_init(bar(ACC_FULL), 1);
-    mbar_init(bar(ACC_EMPTY), 4 * NCTA);                   // epilogue warps of both CTAs
+    mbar_init(bar(ACC_EMPTY), R::NEPI * NCTA);             // epilogue warps of both CTAs
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
@@ -737,7 +759,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         }
       }
     }
-  } else if (warp < NUM_CONV_WARPS) {
+  } else if (warp < R::CONV_WARPS) {
     // ---- converters: group g = warp / 4 expands k-steps g, g+4, g+8, ... ----
     // Thread (quad q = warp % 4, lane) owns row r = 32 q + lane of both operands:
     // the activation row goes to TMEM lane r (32 columns of fp16 pairs, lower K
@@ -757,7 +779,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     const uint32_t t_lane = tmem_base + ((uint32_t)(32 * q) << 16) + (uint32_t)(A_COL0 + 32 * g);
     constexpr int KP = PackedUnit<BA, BW>::KP;
     constexpr int ROW_A = PackedUnit<BA, BW>::kRowA, ROW_B = PackedUnit<BA, BW>::kRowB;
-    for (uint32_t pc = (uint32_t)g, j = 0; pc < total_steps; pc += NUM_GROUPS, ++j) {
+    for (uint32_t pc = (uint32_t)g, j = 0; pc < total_steps; pc += NG, ++j) {
       const uint32_t pu = pc / KP;  // packed stage that holds k-step pc
       const int ps = pu % PSTAGES;
       const uint32_t pph = (pu / PSTAGES) & 1u;
@@ -842,7 +864,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         __syncwarp();
       }
     }
-  } else if (warp >= EPI_WARP0 && warp < EPI_WARP0 + 4) {
+  } else if (warp >= R::EPI_WARP0 && warp < R::EPI_WARP0 + R::NEPI) {
     // ---- epilogue: this CTA's 128 accumulator rows ----
     // TMEM -> registers -> scale, bias, GELU -> swizzled staging -> bulk tensor
     // stores. The accumulator is released right after its last TMEM read, so the
@@ -857,13 +879,31 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     // from those copies while the next tile's MMAs proceed.  The first half is
     // converted in place (each thread rewrites only its own row, and a raw
     // chunk is always read before a bf16 chunk lands on it).
+    //
+    // With NG = 3 the eight epilogue warps form two groups of four (named
+    // barriers 1 and 2), one warp of each per TMEM lane quarter, and split
+    // every tile (bf16-only output, which the launcher guarantees): group 0
+    // evacuates columns 0..127 as raw fp32 into staging blocks 0..3 and
+    // converts them in place (blocks 0, 1); group 1 evacuates columns
+    // 128..255 into the spare TMEM columns and converts them into staging
+    // blocks 4, 5.  Each group's leader issues and waits for its own stores.
     const int quad = warp & 3;  // TMEM lanes 32*quad .. 32*quad+31
     const int rl = quad * 32 + lane;  // row within the CTA's 128
-    const bool leader = (warp == EPI_WARP0 && lane == 0);
+    const int sub = (warp - R::EPI_WARP0) >> 2;  // epilogue group (0 unless NG == 3)
+    const uint32_t bid = 1u + (uint32_t)sub;     // its named barrier
+    const bool leader = (warp == R::EPI_WARP0 + 4 * sub && lane == 0);
     const uint32_t stage = sbase + S::kStage;
     float* col_r = reinterpret_cast<float*>(smem + S::kEpi) + quad * 2 * BN;
     float* col_b = col_r + BN;
     const uint32_t taddr = tmem_base + ((uint32_t)(quad * 32) << 16);
+    constexpr int J0 = 0, JN = BN / 32;  // the 32-column chunks of the factors this warp loads
+    const int j0 = NG == 3 ? 4 * sub : J0, jn = NG == 3 ? 4 * sub + 4 : JN;
+    if constexpr (NG == 3) {
+      if ((args.y16 == nullptr || args.y32 != nullptr) && leader && sub == 0) {
+        atomicExch(args.status, OQ_ERR_UNSUPPORTED);  // never launched this way
+        *abort_flag = 1;
+      }
+    }
     uint32_t lt = 0;
     for (int t = unit; t < num_tiles; t += nunits, ++lt) {
       const int m0 = (t % args.tiles_m) * TILE_M + (int)rank * BM, n0 = (t / args.tiles_m) * BN;
@@ -871,7 +911,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       // this tile's factors, fetched while the MMAs run: a_row / d, r'_n and bias_n
       const float a_scale = row < args.M ? args.a_norm[row] * args.inv_d : 0.0f;
 #pragma unroll
-      for (int j = 0; j < BN / 32; ++j) {
+      for (int j = J0; j < JN; ++j) {
+        if (j < j0 || j >= jn) continue;
         const int n = n0 + lane + 32 * j;
         const bool in = n < args.N;
         col_r[lane + 32 * j] = in ? bf16_to_f32(args.w_norm[n]) : 0.0f;
@@ -879,11 +920,108 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       }
       __syncwarp();
       const bool got = wait_bounded(bar(ACC_FULL), lt & 1u, abort_flag, args.status);
-      if (epi_any(!got)) break;
+      if (epi_any(!got, bid)) break;
       tc_fence_after();
+      if constexpr (NG == 3) {
+        constexpr int H = BN / 2;
+        const uint32_t rsw = (uint32_t)(rl & 7);  // the row's 128-byte swizzle
+        const unsigned long long as2 = f2_pack(a_scale, a_scale);
+        const bool gelu = args.epilogue == OQ_EPI_GELU;
+        if (leader) bulk_wait_read();  // this group's previous stores have read its staging blocks
+        epi_bar(bid);
+        if (sub == 0) {
+#pragma unroll 1
+          for (int c = 0; c < H; c += 32) {  // columns 0.. -> staging block c / 32, raw fp32
+            uint32_t v[32];
+            __syncwarp();
+            tmem_ld16(taddr + (uint32_t)c, v);
+            tmem_ld16(taddr + (uint32_t)(c + 16), v + 16);
+            asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+            const uint32_t rowb = stage + (uint32_t)(c / 32) * 16384u + (uint32_t)rl * 128u;
+#pragma unroll
+            for (int j = 0; j < 8; ++j)
+              sts_v4(rowb + (((uint32_t)j ^ rsw) << 4), make_uint4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]));
+          }
+        } else {
+          const uint32_t spare = taddr + (uint32_t)R::SPARE_COL;
+#pragma unroll 1
+          for (int c = 0; c < H; c += 32) {  // columns H.. -> spare TMEM columns
+            uint32_t v[32];
+            __syncwarp();
+            tmem_ld16(taddr + (uint32_t)(H + c), v);
+            tmem_ld16(taddr + (uint32_t)(H + c + 16), v + 16);
+            asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+            tmem_st16(spare + (uint32_t)c, v);
+            tmem_st16(spare + (uint32_t)(c + 16), v + 16);
+          }
+          asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) {
+          if constexpr (PAIR) mbar_arrive_cluster(bar(ACC_EMPTY), 0);  // the leader's barrier
+          else mbar_arrive(bar(ACC_EMPTY));
+        }
+        if (sub == 0) {
+          // columns 0..127: raw fp32 (blocks 0..3) -> bf16 (blocks 0, 1), in place
+#pragma unroll 1
+          for (int c0 = 0; c0 < H; c0 += 16) {
+            const uint32_t src = stage + (uint32_t)(c0 / 32) * 16384u + (uint32_t)rl * 128u;
+            const uint32_t jr = (uint32_t)(c0 % 32) / 4;
+            uint32_t v[16];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              const uint4 w = lds_v4(src + (((jr + i) ^ rsw) << 4));
+              v[4 * i] = w.x; v[4 * i + 1] = w.y; v[4 * i + 2] = w.z; v[4 * i + 3] = w.w;
+            }
+            const uint32_t dst = stage + (uint32_t)(c0 / 64) * 16384u + (uint32_t)rl * 128u;
+            const uint32_t jb = (uint32_t)(c0 % 64) / 8;
+            sts_v4(dst + ((jb ^ rsw) << 4), epi8_bf16(v, col_r, col_b, c0, as2, gelu));
+            sts_v4(dst + (((jb + 1) ^ rsw) << 4), epi8_bf16(v + 8, col_r, col_b, c0 + 8, as2, gelu));
+          }
+        } else {
+          // columns 128..255: spare TMEM -> bf16 (blocks 4, 5); the next load is in flight during the arithmetic
+          const uint32_t spare = taddr + (uint32_t)R::SPARE_COL;
+          uint32_t va[16], vb[16];
+          __syncwarp();
+          tmem_ld16(spare, va);
+          asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll 1
+          for (int c0 = 0; c0 < H; c0 += 32) {
+            __syncwarp();
+            tmem_ld16(spare + (uint32_t)(c0 + 16), vb);
+            {
+              const uint32_t dst = stage + (uint32_t)(4 + c0 / 64) * 16384u + (uint32_t)rl * 128u;
+              const uint32_t jb = (uint32_t)(c0 % 64) / 8;
+              sts_v4(dst + ((jb ^ rsw) << 4), epi8_bf16(va, col_r, col_b, H + c0, as2, gelu));
+              sts_v4(dst + (((jb + 1) ^ rsw) << 4), epi8_bf16(va + 8, col_r, col_b, H + c0 + 8, as2, gelu));
+            }
+            asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+            __syncwarp();
+            if (c0 + 32 < H) tmem_ld16(spare + (uint32_t)(c0 + 32), va);
+            {
+              const uint32_t dst = stage + (uint32_t)(4 + (c0 + 16) / 64) * 16384u + (uint32_t)rl * 128u;
+              const uint32_t jb = (uint32_t)((c0 + 16) % 64) / 8;
+              sts_v4(dst + ((jb ^ rsw) << 4), epi8_bf16(vb, col_r, col_b, H + c0 + 16, as2, gelu));
+              sts_v4(dst + (((jb + 1) ^ rsw) << 4), epi8_bf16(vb + 8, col_r, col_b, H + c0 + 24, as2, gelu));
+            }
+            asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+          }
+        }
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        epi_bar(bid);
+        if (leader) {
+          const int b0 = sub == 0 ? 0 : 4, x0 = n0 + (sub == 0 ? 0 : H);
+          for (int b = 0; b < 2; ++b)
+            if (x0 + 64 * b < args.N && m0 < args.M)
+              tma_store_2d(&map_y16, stage + (uint32_t)(b0 + b) * 16384u, x0 + 64 * b, m0);
+          bulk_commit();
+        }
+        continue;
+      }
       if (S::kStageBlocks == 4 && args.y16 != nullptr && args.y32 == nullptr) {
         constexpr int H = BN / 2;
-        const uint32_t spare = taddr + (uint32_t)SPARE_COL;
+        const uint32_t spare = taddr + (uint32_t)R::SPARE_COL;
         const uint32_t rsw = (uint32_t)(rl & 7);  // the row's 128-byte swizzle
         if (leader) bulk_wait_read();  // the previous tile's stores have read the staging buffer
         epi_bar();
@@ -1122,9 +1260,9 @@ int make_out_map(CUtensorMap* map, void* base, int M, int N, CUtensorMapDataType
 
 using GemmKernel = void (*)(GemmArgs, CUtensorMap, CUtensorMap, CUtensorMap, CUtensorMap);
 
-template <int BA, int BW, bool PAIR>
+template <int BA, int BW, bool PAIR, int NG>
 int launch_t(GemmArgs& a, const uint8_t* a_codes, const uint8_t* w_codes, int nsm, cudaStream_t stream) {
-  using S = Smem<BA, BW, PAIR>;
+  using S = Smem<BA, BW, PAIR, NG>;
   CUtensorMap ma, mb;
   if (int rc = make_code_map(&ma, a_codes, a.M, a.K * BA / 8, PackedUnit<BA, BW>::kRowA, BM)) return rc;
   if (int rc = make_code_map(&mb, w_codes, a.N, a.K * BW / 8, PackedUnit<BA, BW>::kRowB, S::kBnCta)) return rc;
@@ -1137,7 +1275,7 @@ int launch_t(GemmArgs& a, const uint8_t* a_codes, const uint8_t* w_codes, int ns
     if (int rc = make_out_map(&my16, a.y16, a.M, a.N, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2)) return rc;
   if (a.y32)
     if (int rc = make_out_map(&my32, a.y32, a.M, a.N, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4)) return rc;
-  GemmKernel k = cbgemm_kernel<BA, BW, PAIR>;
+  GemmKernel k = cbgemm_kernel<BA, BW, PAIR, NG>;
   const int smem = S::kAlloc;
   const int tile_m = PAIR ? 2 * BM : BM;
   a.tiles_m = (a.M + tile_m - 1) / tile_m;
@@ -1178,9 +1316,16 @@ int launch_t(GemmArgs& a, const uint8_t* a_codes, const uint8_t* w_codes, int ns
 template <int BA, int BW>
 int launch_pick(GemmArgs& a, const uint8_t* a_codes, const uint8_t* w_codes, int nsm, cudaStream_t stream) {
   // CTA pairs halve the operand expansion per tensor-core flop; one CTA suffices
-  // when a single 128-row tile covers M.
-  if (a.M > BM) return launch_t<BA, BW, true>(a, a_codes, w_codes, nsm, stream);
-  return launch_t<BA, BW, false>(a, a_codes, w_codes, nsm, stream);
+  // when a single 128-row tile covers M.  GELU tiles of short K (at most 32
+  // k-steps) with bf16-only output take three converter groups and eight
+  // epilogue warps: there the epilogue's arithmetic, not the expansion, sets
+  // the pace.
+  if (a.M > BM) {
+    if (a.epilogue == OQ_EPI_GELU && a.y16 != nullptr && a.y32 == nullptr && a.K <= 32 * BK)
+      return launch_t<BA, BW, true, 3>(a, a_codes, w_codes, nsm, stream);
+    return launch_t<BA, BW, true, 4>(a, a_codes, w_codes, nsm, stream);
+  }
+  return launch_t<BA, BW, false, 4>(a, a_codes, w_codes, nsm, stream);
 }
 
 }  // namespace
