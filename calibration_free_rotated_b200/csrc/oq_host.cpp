@@ -482,36 +482,79 @@ static uint16_t composed_slot(uint32_t c, bool first_round) {
   return (uint16_t)((g << 5) | ((ch ^ (g & 15u)) << 1) | (c & 1u));
 }
 
-int rpbh_composed_tables(oq_rpbh_t r, const uint16_t** slots, const uint32_t** signs) {
+// Register order of the block-transposed FWHT for blocks of L = h / 32 lanes
+// (R = 32 / L): thread g (lane l = g mod L of its block) gathers into register
+// r coordinate 32 (g - l) + 32 ((r / R) ^ l) + R l + r mod R (layout A), and
+// holds output coordinate 32 g + R (u ^ l) + b in register R u + b (layout B).
+static uint32_t xch_gather_coord(uint32_t g, uint32_t r, uint32_t L) {
+  const uint32_t R = 32u / L, l = g & (L - 1u);
+  return 32u * (g - l) + 32u * ((r / R) ^ l) + R * l + r % R;
+}
+static uint32_t xch_output_reg(uint32_t c, uint32_t L) {  // the register that holds output coordinate c
+  const uint32_t R = 32u / L, l = (c >> 5) & (L - 1u), i = c & 31u;
+  return R * ((i / R) ^ l) + i % R;
+}
+
+int rpbh_composed_tables(oq_rpbh_t r, const uint16_t** slots, const uint32_t** signs, bool xch) {
   int dev;
   if (int rc = current_device(&dev)) return rc;
+  const uint32_t L = (uint32_t)r->h / 32u;
+  const bool xch_ok = L >= 2 && L <= 8 && r->d % 32 == 0;
+  if (xch && !xch_ok) return fail(OQ_ERR_UNSUPPORTED, "no block-transposed layout for block %d", r->h);
   std::lock_guard<std::mutex> lk(r->mu);
   if (!r->dev_slots[dev]) {
     const int d = r->d, words = (d + 31) / 32;
-    std::vector<uint16_t> sl((size_t)r->rounds * d);
-    std::vector<uint32_t> sg((size_t)r->rounds * words);
+    std::vector<uint16_t> sl((size_t)r->rounds * d), xsl(xch_ok ? (size_t)r->rounds * d : 0);
+    std::vector<uint32_t> sg((size_t)r->rounds * words), xsg(xch_ok ? (size_t)r->rounds * words : 0, 0u);
     for (int k = 0; k < r->rounds; ++k) {
       const int32_t* perm = k == 0 ? r->perm.data() : r->perm_more.data() + (size_t)(k - 1) * d;
       const uint32_t* bits = k == 0 ? r->sign_bits.data() : r->sign_bits_more.data() + (size_t)(k - 1) * words;
       for (int j = 0; j < d; ++j) sl[(size_t)k * d + j] = composed_slot((uint32_t)perm[j], k == 0);
       std::memcpy(sg.data() + (size_t)k * words, bits, sizeof(uint32_t) * words);
+      if (!xch_ok) continue;
+      for (uint32_t g = 0; g < (uint32_t)d / 32u; ++g) {
+        for (uint32_t reg = 0; reg < 32u; ++reg) {
+          const uint32_t j = xch_gather_coord(g, reg, L);
+          const uint32_t c = (uint32_t)perm[j];  // the input coordinate this register reads
+          uint16_t slot;
+          if (k == 0) {
+            slot = composed_slot(c, true);      // round 1: the pair words, in coordinate order
+          } else {                              // later rounds: where the previous round stored c
+            slot = composed_slot((c & ~31u) | xch_output_reg(c, L), false);
+          }
+          xsl[(size_t)k * d + 32u * g + reg] = slot;
+          if ((bits[j >> 5] >> (j & 31u)) & 1u) xsg[(size_t)k * words + g] |= 1u << reg;
+        }
+      }
     }
-    uint16_t* dsl = nullptr;
-    uint32_t* dsg = nullptr;
+    uint16_t *dsl = nullptr, *dxsl = nullptr;
+    uint32_t *dsg = nullptr, *dxsg = nullptr;
     cudaError_t e = dev_malloc(reinterpret_cast<void**>(&dsl), sizeof(uint16_t) * sl.size());
     if (e == cudaSuccess) e = dev_malloc(reinterpret_cast<void**>(&dsg), sizeof(uint32_t) * sg.size());
     if (e == cudaSuccess) e = cudaMemcpy(dsl, sl.data(), sizeof(uint16_t) * sl.size(), cudaMemcpyHostToDevice);
     if (e == cudaSuccess) e = cudaMemcpy(dsg, sg.data(), sizeof(uint32_t) * sg.size(), cudaMemcpyHostToDevice);
+    if (e == cudaSuccess && xch_ok) {
+      e = dev_malloc(reinterpret_cast<void**>(&dxsl), sizeof(uint16_t) * xsl.size());
+      if (e == cudaSuccess) e = dev_malloc(reinterpret_cast<void**>(&dxsg), sizeof(uint32_t) * xsg.size());
+      if (e == cudaSuccess)
+        e = cudaMemcpy(dxsl, xsl.data(), sizeof(uint16_t) * xsl.size(), cudaMemcpyHostToDevice);
+      if (e == cudaSuccess)
+        e = cudaMemcpy(dxsg, xsg.data(), sizeof(uint32_t) * xsg.size(), cudaMemcpyHostToDevice);
+    }
     if (e != cudaSuccess) {
       cudaFree(dsl);
       cudaFree(dsg);
+      cudaFree(dxsl);
+      cudaFree(dxsg);
       return fail(OQ_ERR_CUDA, "uploading composed rotation tables: %s", cudaGetErrorString(e));
     }
     r->dev_slots[dev] = dsl;
     r->dev_csigns[dev] = dsg;
+    r->dev_xslots[dev] = dxsl;
+    r->dev_xcsigns[dev] = dxsg;
   }
-  *slots = r->dev_slots[dev];
-  *signs = r->dev_csigns[dev];
+  *slots = xch ? r->dev_xslots[dev] : r->dev_slots[dev];
+  *signs = xch ? r->dev_xcsigns[dev] : r->dev_csigns[dev];
   return OQ_OK;
 }
 
@@ -765,6 +808,8 @@ void oq_free_rpbh(oq_rpbh_t r) {
       cudaFree(r->dev_signs[dev]);
       cudaFree(r->dev_slots[dev]);
       cudaFree(r->dev_csigns[dev]);
+      cudaFree(r->dev_xslots[dev]);
+      cudaFree(r->dev_xcsigns[dev]);
     }
   }
   if (have_prev) cudaSetDevice(prev);

@@ -26,6 +26,10 @@ struct oq_rpbh_s {
   uint32_t* dev_signs[OQ_MAX_DEVICES] = {};  // sign words [d/32]
   uint16_t* dev_slots[OQ_MAX_DEVICES] = {};  // composed kernel: [rounds][d] shared-memory slots
   uint32_t* dev_csigns[OQ_MAX_DEVICES] = {};  // composed kernel: [rounds][d/32] sign words
+  // The same for the block-transposed FWHT (blocks of 64..256): slots and sign
+  // bits in each thread's register order instead of coordinate order.
+  uint16_t* dev_xslots[OQ_MAX_DEVICES] = {};
+  uint32_t* dev_xcsigns[OQ_MAX_DEVICES] = {};
 };
 
 struct oq_codebook_s {
@@ -58,7 +62,9 @@ uint16_t double_to_fp16_rne(double v);
 // Device-side state (oq_host.cpp).
 int current_device(int* dev);
 int rpbh_device_tables(oq_rpbh_t r, const uint16_t** perm, const uint32_t** signs);
-int rpbh_composed_tables(oq_rpbh_t r, const uint16_t** slots, const uint32_t** signs);
+// Tables of the composed kernel: coordinate order, or (xch) the register order
+// of the block-transposed FWHT (OQ_ERR_UNSUPPORTED when the block has none).
+int rpbh_composed_tables(oq_rpbh_t r, const uint16_t** slots, const uint32_t** signs, bool xch = false);
 int codebook_device_qtable(oq_codebook_t cb, const uint32_t** qtable);
 void build_qtable(oq_codebook_t cb);
 int device_status_word(int** status);

@@ -29,7 +29,13 @@
 //     block transform in registers;
 //   * the sum of squares comes from round 1's gathered input (the rotation is
 //     orthogonal); the k factors sqrt(h) of the unnormalised transforms are
-//     folded into the search multiplier.
+//     folded into the search multiplier;
+//   * for blocks of 64..256 coordinates (where the packed codes allow it) each
+//     round runs the block-transposed transform of the one-round kernel: the
+//     slot and sign tables are then in each thread's register order (layout A
+//     of that transform), a later round's slots point at where the previous
+//     round stored each coordinate from layout B, and the codes of the last
+//     round are moved back to coordinate order before the store.
 #include <cuda_runtime.h>
 
 #include <algorithm>
@@ -140,6 +146,15 @@ __global__ void __launch_bounds__(512, 1) rotq_composed_kernel(const __grid_cons
   const int nwarps = blockDim.x >> 5;
   const uint32_t rowb = (uint32_t)a.d * 2u;  // bytes of a bf16 row
   const uint32_t ring = fbase + a.ring_off, bars = fbase + a.bar_off;
+  constexpr bool XCH = Xch<BITS, LOGHB>::ok();
+  const int bl = lane & ((1 << LOGHB) - 1);  // lane within the Hadamard block
+  unsigned long long sg[3], nsg[3];          // block-transposed stages: (s, s), (-s, -s)
+#pragma unroll
+  for (int k = 0; k < 3; ++k) {
+    const float s = ((bl >> k) & 1) ? -1.0f : 1.0f;
+    sg[k] = f2_pack(s, s);
+    nsg[k] = f2_pack(-s, -s);
+  }
 
   if (tid == 0) {
     for (int s = 0; s < a.stages; ++s)
@@ -199,7 +214,10 @@ __global__ void __launch_bounds__(512, 1) rotq_composed_kernel(const __grid_cons
 #pragma unroll
         for (int i = 0; i < 32; ++i) sq[i & 3] = f2_fma(v[i], v[i], sq[i & 3]);
       }
-      fwht_pairs<LOGHB>(v, lane);
+      if constexpr (XCH)
+        fwht_xch<LOGHB>(v, sg, nsg);
+      else
+        fwht_pairs<LOGHB>(v, lane);
       if (r + 1 < a.rounds) {
         __syncthreads();  // every thread has gathered this round's input
         if (active) store_run(run, rot, v);
@@ -232,6 +250,10 @@ __global__ void __launch_bounds__(512, 1) rotq_composed_kernel(const __grid_cons
       const float A_b = sum_b > 0.0f ? a.alpha * rsqrtf(sum_b) : 0.0f;
       uint32_t wa[BITS], wb[BITS];
       search_pack<BITS>(v, A_a, A_b, a.nb, qkey, wa, wb);
+      if constexpr (XCH) {  // register group u holds the codes of group u ^ bl
+        xor_groups<BITS, LOGHB>(wa, bl);
+        xor_groups<BITS, LOGHB>(wb, bl);
+      }
       const size_t cb = (size_t)(a.d / 8 * BITS);
       uint8_t* dst = a.codes + (size_t)row * cb + (size_t)tid * (4 * BITS);
       store_words<BITS>(dst, wa);
@@ -253,6 +275,30 @@ __global__ void __launch_bounds__(512, 1) rotq_composed_kernel(const __grid_cons
 }
 
 using ComposedFn = void (*)(ComposedArgs);
+
+// Whether rotq_composed_kernel<bits, loghb> runs the block-transposed transform
+// (and so reads the register-order tables).
+template <int BITS>
+bool composed_xch_bits(int loghb) {
+  switch (loghb) {
+    case 1: return Xch<BITS, 1>::ok();
+    case 2: return Xch<BITS, 2>::ok();
+    case 3: return Xch<BITS, 3>::ok();
+    default: return false;
+  }
+}
+
+bool composed_xch(int bits, int loghb) {
+  switch (bits) {
+    case 1: return composed_xch_bits<1>(loghb);
+    case 2: return composed_xch_bits<2>(loghb);
+    case 3: return composed_xch_bits<3>(loghb);
+    case 4: return composed_xch_bits<4>(loghb);
+    case 5: return composed_xch_bits<5>(loghb);
+    case 6: return composed_xch_bits<6>(loghb);
+    default: return false;
+  }
+}
 
 template <int BITS>
 ComposedFn pick_composed_bits(int loghb) {
@@ -294,7 +340,7 @@ int launch_rotq_composed(oq_rpbh_t r, oq_codebook_t cb, const void* X, int M, ui
   if (!kern) return fail(OQ_ERR_UNSUPPORTED, "no composed rotate+quantize kernel for bits=%d h=%d", bits, h);
   const uint16_t* slots;
   const uint32_t* signs;
-  if (int rc = rpbh_composed_tables(r, &slots, &signs)) return rc;
+  if (int rc = rpbh_composed_tables(r, &slots, &signs, rotq::composed_xch(bits, loghb))) return rc;
   const uint32_t* qtable;
   if (int rc = codebook_device_qtable(cb, &qtable)) return rc;
   int nsm;

@@ -255,7 +255,10 @@ def test_empirical_distortion_matches_lloyd_max(oq, codebooks, d, h, bits):
 
 @pytest.mark.parametrize("d,h,bits,rounds", [(256, 64, 4, 2), (3072, 128, 4, 2), (3072, 128, 2, 3), (1536, 256, 6, 2),
                                               (12288, 128, 4, 2), (16384, 1024, 4, 3), (512, 32, 3, 2),
-                                              (8960, 128, 5, 3), (1024, 1024, 1, 2)])
+                                              (8960, 128, 5, 3), (1024, 1024, 1, 2),
+                                              # block-transposed transform in every round (blocks of 64..256)
+                                              (3072, 64, 3, 2), (3072, 64, 6, 3), (1536, 128, 6, 2),
+                                              (2048, 256, 4, 2), (2048, 256, 1, 3), (8960, 256, 2, 2)])
 def test_composed_rounds(oq, codebooks, d, h, bits, rounds):
     # [RHT] Methodology: Pi_k ... Pi_1, k RPBH rounds from one SplitMix64
     # stream, against the oracle; ragged M, sparse rows and a zero row included
