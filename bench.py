@@ -521,15 +521,15 @@ def run_ablation(args):
     times oq_quantize_act (4-bit) under RPBH, Block-RHT (no permutation) and Full
     RHT (d's largest power-of-two block) on N(0,1) bf16 rows, and the composed
     RPBH of 2 and 3 rounds ([RHT] Methodology).  L2 is flushed
-    (a 256 MB write) before every timed launch; CUDA events bracket the launch
-    alone.  Prints one JSON line per (shape, rotation); not the contract line."""
+    (L2Flush: a 256 MB write, then a 256 MB read) before every timed launch;
+    CUDA events bracket the launch alone.  Prints one JSON line per (shape, rotation); not the contract line."""
     import torch
     from calibration_free_rotated_b200 import build
     build.build()
     from calibration_free_rotated_b200 import orbitquant as oq
     peaks, src = load_peaks()
     torch.manual_seed(0)
-    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+    flush = L2Flush()
     d = args.d
     for M in (args.rows, 32768):
         X = torch.randn(M, d, device="cuda").to(torch.bfloat16)
@@ -543,7 +543,7 @@ def run_ablation(args):
                 oq.quantize_act(r, cb, X, codes, norms)
             times = []
             for _ in range(args.steps):
-                flush.zero_()
+                flush()
                 e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
                 e0.record()
                 oq.quantize_act(r, cb, X, codes, norms)
@@ -606,14 +606,31 @@ def run_ablation_steps(args):
     return 0
 
 
+class L2Flush:
+    """Leaves L2 cold and clean before a timed launch: a 256 MB write (the
+    flush), then a 256 MB read of another buffer, which evicts the written
+    lines, so their write-back to HBM happens here and not inside the timed
+    window (a write alone leaves up to the whole L2 dirty, and an HBM-bound
+    kernel timed after it shares the bus with that write-back)."""
+
+    def __init__(self, device="cuda"):
+        import torch
+        self.buf = torch.empty(256 << 20, dtype=torch.uint8, device=device)
+        self.clean = torch.ones(64 << 20, dtype=torch.float32, device=device)
+
+    def __call__(self):
+        self.buf.zero_()
+        self.clean.sum()
+
+
 def _flush_and_time(fn, flush, steps, warmup):
-    """Median CUDA-event time (ms) of fn() with a 256 MB L2 flush before each call."""
+    """Median CUDA-event time (ms) of fn() with an L2 flush (L2Flush) before each call."""
     import torch
     for _ in range(warmup):
         fn()
     times = []
     for _ in range(steps):
-        flush.zero_()
+        flush()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record()
         fn()
@@ -623,6 +640,27 @@ def _flush_and_time(fn, flush, steps, warmup):
     return statistics.median(times)
 
 
+def _flush_and_time_many(fns, flush, steps, warmup):
+    """Median CUDA-event times (ms) of several launches, each timed alone after
+    an L2 flush, taken round-robin (one of each per repetition) so that a clock
+    change during the run affects them alike."""
+    import torch
+    for fn in fns:
+        for _ in range(warmup):
+            fn()
+    times = [[] for _ in fns]
+    for _ in range(steps):
+        for i, fn in enumerate(fns):
+            flush()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            fn()
+            e1.record()
+            e1.synchronize()
+            times[i].append(e0.elapsed_time(e1))
+    return [statistics.median(t) for t in times]
+
+
 def run_workload(args):
     """Per-kernel times of the two-layer workloads (one JSON line each; not the
     contract line).  flux_mlp: X[4608 x 3072] -> fc1 [12288 x 3072] + GELU ->
@@ -630,7 +668,8 @@ def run_workload(args):
     -> fc1 [8960 x 1536] + GELU -> fc2 [1536 x 8960], W4A6, block 128.
     flux_qkv_w3a3: the FLUX-like QKV projection (X[4608 x 3072] -> W[9216 x 3072]
     + bias) at W3A3 ([OQ] Experiments, Qualitative Results).  Every launch is
-    timed alone after a 256 MB L2 flush."""
+    timed alone after an L2 flush (L2Flush), the launches round-robin; the SM
+    clock is sampled meanwhile."""
     import torch
     from calibration_free_rotated_b200 import build
     build.build()
@@ -640,7 +679,7 @@ def run_workload(args):
     h = 128
     dev = torch.device("cuda")
     bf = lambda bits: torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).to(dev).view(torch.bfloat16)
-    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    flush = L2Flush(dev)
     if args.workload == "flux_qkv_w3a3":
         M, d, N, b = 4608, 3072, 9216, 3
         r, cb = oq.Rpbh(0, d, h), oq.Codebook(d, b)
@@ -649,16 +688,18 @@ def run_workload(args):
         bias = bf(inputs.bias(2, N))
         ac, an = oq.quantize_act(r, cb, X)
         Y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
-        ms_q = _flush_and_time(lambda: oq.quantize_act(r, cb, X, ac, an), flush, args.steps, args.warmup)
-        ms_g = _flush_and_time(lambda: oq.linear_codes(d, cb, cb, ac, an, wc, wn, bias=bias, out_bf16=Y,
-                                                       want_f32=False, want_bf16=True), flush, args.steps, args.warmup)
+        with ClockSampler(torch.cuda.current_device()) as clk:
+            ms_q, ms_g = _flush_and_time_many(
+                [lambda: oq.quantize_act(r, cb, X, ac, an),
+                 lambda: oq.linear_codes(d, cb, cb, ac, an, wc, wn, bias=bias, out_bf16=Y, want_f32=False,
+                                         want_bf16=True)], flush, args.steps, args.warmup)
         oq.device_status()
         gbs, tfs = algorithmic(M, d, N, b, b)[0] / ms_q / 1e6, 2.0 * M * N * d / ms_g / 1e9
         print(json.dumps({"workload": args.workload, "M": M, "d": d, "N": N, "bits_w": b, "bits_a": b, "block": h,
                           "kernels": {"act_quant": {"ms": ms_q, "GB/s": gbs, "frac": gbs / peaks["hbm_gbs"]},
                                       "qkv": {"ms": ms_g, "TFLOP/s": tfs, "frac": tfs / peaks["bf16_tflops"]}},
                           "peak_source": src, "step_ms": ms_q + ms_g,
-                          "TFLOP/s": 2.0 * M * N * d / (ms_q + ms_g) / 1e9}), flush=True)
+                          "TFLOP/s": 2.0 * M * N * d / (ms_q + ms_g) / 1e9, "clocks": clk.summary()}), flush=True)
         return 0
     wl, M, d1, d2, bw, ba = {"flux_mlp": (3, 4608, 3072, 12288, 2, 4),
                              "wan_ffn": (4, 32760, 1536, 8960, 4, 6)}[args.workload]
@@ -698,8 +739,9 @@ def run_workload(args):
            "kernels": {}, "peak_source": src}
     total = 0.0
     folded = 0.0
-    for name, fn, bound, work in steps:
-        ms = _flush_and_time(fn, flush, args.steps, args.warmup)
+    with ClockSampler(torch.cuda.current_device()) as clk:
+        all_ms = _flush_and_time_many([fn for _, fn, _, _ in steps], flush, args.steps, args.warmup)
+    for (name, fn, bound, work), ms in zip(steps, all_ms):
         if name in ("act_quant_1", "fc2") or name.endswith("_folded"):
             folded += ms
         if not name.endswith("_folded"):
@@ -715,13 +757,14 @@ def run_workload(args):
     out["TFLOP/s"] = 4.0 * M * d1 * d2 / total / 1e9
     out["step_ms_folded_permutation"] = folded
     out["TFLOP/s_folded_permutation"] = 4.0 * M * d1 * d2 / folded / 1e9
+    out["clocks"] = clk.summary()
     print(json.dumps(out), flush=True)
     return 0
 
 
 def run_flatness(args):
     """The flatness check ([RHT] Key contribution 4: rho3 and rhoinf of every
-    row, and the batch maxima) timed alone after a 256 MB L2 flush, with per-row
+    row, and the batch maxima) timed alone after an L2 flush (L2Flush), with per-row
     outputs and with the batch maxima only, on N(0,1) bf16 rows.  Algorithmic
     bytes: the rows once (2 M d) plus 8 bytes per row written (4 per measure)
     and the maxima.  One JSON line per shape; not the contract line."""
@@ -731,7 +774,7 @@ def run_flatness(args):
     from calibration_free_rotated_b200 import orbitquant as oq
     peaks, src = load_peaks()
     torch.manual_seed(0)
-    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+    flush = L2Flush()
     for M, d in ((4608, 3072), (32768, 3072), (32760, 8960), (16384, 12288)):
         X = torch.randn(M, d, device="cuda").to(torch.bfloat16)
         r3 = torch.empty(M, device="cuda")
@@ -789,7 +832,7 @@ def run_sweep(args):
     from calibration_free_rotated_b200 import orbitquant as oq
     peaks, src = load_peaks()
     dev = torch.device("cuda")
-    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    flush = L2Flush(dev)
     Ms = [int(x) for x in args.sweep_rows.split(",")]
     for d in (1536, 3072, 12288):
         for M in Ms:
