@@ -354,6 +354,8 @@ def run_ours(args, world, rank, local):
     k1 = [e[0].elapsed_time(e[1]) / 1e3 for e in evs]
     k2 = [e[1].elapsed_time(e[2]) / 1e3 for e in evs]
     total_s, split_s, k1_avg, k2_avg = reduce_max([total_s, split_s, sum(k1) / len(k1), sum(k2) / len(k2)], world)
+    pct = lambda v: {q: 1e3 * sorted(v)[round(f * (len(v) - 1))] for q, f in (("p10", 0.1), ("median", 0.5), ("p90", 0.9))}
+    k1_pct, k2_pct = pct(k1), pct(k2)  # this rank's spread
 
     aq_bytes, flops = algorithmic(M, K, N, 4, 4)
     value = whole_job_value(flops * args.steps, world, total_s) / 1e12
@@ -433,8 +435,9 @@ def run_ours(args, world, rank, local):
                                "traffic": aq_traffic, "peak_source": f"{peak_kind} copy bandwidth",
                                "algorithmic_per_launch": aq_bytes},
         "kernel_ms": {"rotq_kernel": 1e3 * k1_avg, "cbgemm_kernel": 1e3 * k2_avg,
+                      "rotq_kernel_spread": k1_pct, "cbgemm_kernel_spread": k2_pct,
                       "region": "a second timed region of K steps with an event before, between and after the two "
-                                "kernels of every step",
+                                "kernels of every step (means, max over ranks; spreads of rank 0's K steps)",
                       "ms_per_step_with_kernel_events": 1e3 * split_s / args.steps},
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": M * K * 2, "d2h_bytes_per_step": M * N * 2},
         "gpu_launches": 2 * args.steps,
