@@ -1349,7 +1349,9 @@ int launch_cbgemm(int d, oq_codebook_t cb_a, oq_codebook_t cb_w, const uint8_t* 
   a.N = N;
   a.K = d;
   a.epilogue = epilogue;
-  a.inv_d = (float)(1.0 / (double)d);
+  // the two tables are fp16(sqrt(d_cb) c): the product carries d_cb (= d unless
+  // the codebooks are for the block)
+  a.inv_d = (float)(1.0 / std::sqrt((double)cb_a->d * (double)cb_w->d));
   a.stall = take_test_stall(2);
   for (int i = 0; i < 32; ++i) {
     auto entry = [](oq_codebook_t cb, int k) -> uint32_t {

@@ -882,7 +882,11 @@ static int check_quant_args(oq_rpbh_t r, oq_codebook_t cb, const void* X, int M,
                             const void* norms) {
   if (!r || !cb) return fail(OQ_ERR_ARG, "NULL handle");
   if (M < 0) return fail(OQ_ERR_ARG, "M must be >= 0 (got %d)", M);
-  if (r->d != cb->d) return fail(OQ_ERR_ARG, "rpbh d=%d and codebook d=%d differ", r->d, cb->d);
+  // The codebook is C^(d,b) for the row width d; C^(h,b) for the rotation's
+  // block h is accepted too (the literal reading of a "codebook for d = h" on
+  // rows of width d: the rows are unit vectors either way).
+  if (cb->d != r->d && cb->d != r->h)
+    return fail(OQ_ERR_ARG, "codebook d=%d is neither the rows' d=%d nor the block %d", cb->d, r->d, r->h);
   if (r->d % 32 != 0 || r->d > 16384)
     return fail(OQ_ERR_UNSUPPORTED, "kernels need d %% 32 == 0 and d <= 16384 (d=%d)", r->d);
   if (r->h < 32 || r->h > 1024) return fail(OQ_ERR_UNSUPPORTED, "kernels need 32 <= block <= 1024 (h=%d)", r->h);
@@ -937,8 +941,8 @@ static int check_linear_args(int d, oq_codebook_t cb_a, oq_codebook_t cb_w, int 
                              const void* w_norm, int N, const void* bias, int epilogue, const void* Y_f32,
                              const void* Y_bf16) {
   if (!cb_a || !cb_w) return fail(OQ_ERR_ARG, "NULL codebook handle");
-  if (cb_a->d != d || cb_w->d != d)
-    return fail(OQ_ERR_ARG, "codebook dims (%d, %d) must equal d=%d", cb_a->d, cb_w->d, d);
+  if (cb_a->d != cb_w->d || cb_a->d <= 0 || d % cb_a->d != 0)
+    return fail(OQ_ERR_ARG, "codebook dims (%d, %d) must be equal and divide d=%d", cb_a->d, cb_w->d, d);
   if (M < 0 || N < 0) return fail(OQ_ERR_ARG, "M and N must be >= 0");
   if (epilogue != OQ_EPI_NONE && epilogue != OQ_EPI_GELU) return fail(OQ_ERR_ARG, "unknown epilogue %d", epilogue);
   if (d % 64 != 0) return fail(OQ_ERR_UNSUPPORTED, "the GEMM needs d %% 64 == 0 (d=%d)", d);

@@ -204,7 +204,10 @@ OQ_API void oq_free_codebook(oq_codebook_t cb);
  * X     : device bf16 [M][d] (row-major, rows contiguous).
  * codes : device uint8 [M][d*b/8], packed as described at the top.
  * norms : device float [M], s per row (the norm of x' equals that of x).
- * M >= 0 (M == 0 launches nothing).  d must match both handles.
+ * M >= 0 (M == 0 launches nothing).  d is the rotation's width; the codebook
+ * is C^(d,b), or C^(h,b) for the rotation's block h (a reading of a
+ * "codebook for d = h" on rows of width d; the rows are unit vectors either
+ * way, so the codes are well defined).  Any other codebook: OQ_ERR_ARG.
  * ------------------------------------------------------------------------- */
 OQ_API int oq_quantize_act(oq_rpbh_t r, oq_codebook_t cb, const void* X, int M, uint8_t* codes, float* norms,
                     void* stream);
@@ -250,9 +253,12 @@ OQ_API int oq_row_flatness(const void* X, int M, int d, float* rho3, float* rhoi
  * Codebook linear on codes  ([OQ] "Online Activation Quantization", last
  * paragraph: W^' x^' ~= W Pi^T Pi x = W x, no inverse rotation)
  *   y[m][n] = s_m r'_n sum_k v_a[ca[m][k]] v_w[cw[n][k]]  (+ bias_n) (-> GELU)
- * with v = lut_fp16 / sqrt(d) of each codebook.  Accumulation is fp32 on the
- * tensor cores (fp16 x fp16 products).
- * d           : common inner dimension; cb_a and cb_w must both have it.
+ * with v = lut_fp16 / sqrt(d_cb) of each codebook (d_cb its dimension).
+ * Accumulation is fp32 on the tensor cores (fp16 x fp16 products).
+ * d           : common inner dimension.  cb_a and cb_w must have the same
+ *               dimension d_cb, which divides d (d_cb = d, or the rotation's
+ *               block when the codes were made with C^(h,b)); OQ_ERR_ARG
+ *               otherwise.
  * a_codes     : device uint8 [M][d*ba/8];  a_norm : device float [M].
  * w_codes     : device uint8 [N][d*bw/8];  w_norm : device bf16 [N].
  * bias        : device bf16 [N] or NULL.

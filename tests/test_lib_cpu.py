@@ -84,6 +84,13 @@ def test_argument_errors_without_gpu(oq):
     assert lib.oq_quantize_act(r.handle, cb8.handle, None, 4, None, None, None) == oq.OQ_ERR_UNSUPPORTED
     assert lib.oq_quantize_act(r.handle, cb.handle, None, 4, None, None, None) == oq.OQ_ERR_ARG
     assert lib.oq_quantize_act(r.handle, cb.handle, None, 0, None, None, None) == oq.OQ_OK  # M == 0: nothing
+    # a codebook for the block (C^(64,4) on rows of width 256) passes the dimension check; others do not
+    cb_blk = oq.Codebook(64, 4)
+    cb128 = oq.Codebook(128, 4)
+    assert lib.oq_quantize_act(r.handle, cb_blk.handle, None, 0, None, None, None) == oq.OQ_OK
+    assert lib.oq_quantize_act(r.handle, cb128.handle, None, 0, None, None, None) == oq.OQ_ERR_ARG
+    assert b"neither" in lib.oq_last_error()
+    assert lib.oq_quantize_act(r.handle, cb_other.handle, None, 0, None, None, None) == oq.OQ_ERR_ARG
     assert lib.oq_quantize_act(r.handle, cb.handle, ctypes.c_void_p(8), 4, ctypes.c_void_p(16),
                                ctypes.c_void_p(16), None) == oq.OQ_ERR_ALIGN
     r_small = oq.Rpbh(0, 48, 16)
@@ -102,6 +109,14 @@ def test_argument_errors_without_gpu(oq):
                                None, None, None) == oq.OQ_ERR_ARG                          # no output
     assert lib.oq_linear_codes(256, cb.handle, cb2.handle, None, None, 0, None, None, 32, None, 0,
                                None, None, None) == oq.OQ_OK                               # M == 0
+    # codebook dimensions: equal, and dividing d
+    assert lib.oq_linear_codes(256, cb_blk.handle, cb_blk.handle, None, None, 0, None, None, 32, None, 0,
+                               None, None, None) == oq.OQ_OK
+    assert lib.oq_linear_codes(256, cb_blk.handle, cb.handle, None, None, 0, None, None, 32, None, 0,
+                               None, None, None) == oq.OQ_ERR_ARG
+    assert lib.oq_linear_codes(256, cb_other.handle, cb_other.handle, None, None, 0, None, None, 32, None, 0,
+                               None, None, None) == oq.OQ_ERR_ARG
+    assert b"divide" in lib.oq_last_error()
 
 
 def test_workspace_bytes(oq):

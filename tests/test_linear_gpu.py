@@ -86,6 +86,34 @@ def _run_codes(oq, codebooks, ca, s, cw, r16, d, ba, bw, bias_bits=None, epilogu
     return y32.cpu().double().numpy(), (None if y16 is None else y16.float().cpu().double().numpy()), ref
 
 
+def test_single_linear_workload_block_codebook(oq, codebooks):
+    # The literal reading of the single-linear workload's codebook: C^(64,4)
+    # (the block's dimension) for both operands on K = 256.  The dequant table
+    # is lut_fp16 / sqrt(64), so the epilogue divides by 64, not by K.
+    d, h, dc = 256, 64, 64
+    X = inputs.activations(1, 64, d)
+    W = inputs.weights(1, inputs.T_W, 256, d)
+    book = codebooks(dc, 4)
+    perm, signs = orpbh.draw_permutation_and_signs(0, d)
+    ca, s, _ = oqz.quantize_rows(inputs.bf16_bits_to_f64(X), perm, signs, h, book["centroids"])
+    cw, r16, _, _ = oqz.quantize_weight_rows(inputs.bf16_bits_to_f64(W), perm, signs, h, book["centroids"])
+    cb = oq.Codebook(dc, 4)
+    # the GEMM on the oracle's codes
+    y32, _ = oq.linear_codes(d, cb, cb, _dev_u8(oqz.pack_codes(ca, 4)), torch.from_numpy(s.astype(np.float32)).cuda(),
+                             _dev_u8(oqz.pack_codes(cw, 4)), _dev_bf16(oqz.bf16_bits(r16)))
+    torch.cuda.synchronize()
+    oq.device_status()
+    ref = olin.linear_from_codes(ca, s, cw, r16, book["centroids"], book["centroids"], dc)
+    assert _rel_fro(y32.cpu().double().numpy(), ref) <= TOL
+    # the whole layer: the GPU quantizes both operands with the same handles
+    r = oq.Rpbh(0, d, h)
+    wc, wn = oq.quantize_weight(r, cb, _dev_bf16(W))
+    y, _ = oq.linear(r, cb, cb, _dev_bf16(X), wc, wn)
+    torch.cuda.synchronize()
+    oq.device_status()
+    assert _rel_fro(y.cpu().double().numpy(), ref) <= TOL
+
+
 @pytest.mark.parametrize("ba,bw", [(4, 4), (4, 2), (6, 4), (2, 2), (6, 6), (2, 4), (3, 3)])
 def test_codes_gemm_small_ragged(oq, codebooks, ba, bw):
     # several tiles in both M and N, M and N tails (M=200, N=272), K = 256

@@ -37,10 +37,10 @@ def oq():
 _handles = {}
 
 
-def _lib_handles(oq, seed, d, h, bits, kind="rpbh", rounds=1):
-    key = (seed, d, h, bits, kind, rounds)
+def _lib_handles(oq, seed, d, h, bits, kind="rpbh", rounds=1, cb_d=None):
+    key = (seed, d, h, bits, kind, rounds, cb_d)
     if key not in _handles:
-        _handles[key] = (oq.Rpbh(seed, d, h, kind=kind, rounds=rounds), oq.Codebook(d, bits))
+        _handles[key] = (oq.Rpbh(seed, d, h, kind=kind, rounds=rounds), oq.Codebook(cb_d or d, bits))
     return _handles[key]
 
 
@@ -49,9 +49,10 @@ def _to_dev(bits_u16):
 
 
 def _check_rows(oq, codebooks, X_bits, d, h, bits, seed=0, weight=False, rows=None, report=None, kind="rpbh",
-                rounds=1):
-    """Runs the kernel on all of X_bits; checks rows `rows` (default all) against the oracle."""
-    r, cb = _lib_handles(oq, seed, d, h, bits, kind, rounds)
+                rounds=1, cb_d=None):
+    """Runs the kernel on all of X_bits; checks rows `rows` (default all) against the oracle.
+    cb_d: the codebook's dimension when it is not the row width d."""
+    r, cb = _lib_handles(oq, seed, d, h, bits, kind, rounds, cb_d)
     X = _to_dev(X_bits)
     if weight:
         codes, norms = oq.quantize_weight(r, cb, X)
@@ -68,7 +69,7 @@ def _check_rows(oq, codebooks, X_bits, d, h, bits, seed=0, weight=False, rows=No
     perm, signs = orpbh.draw_permutation_and_signs(seed, d)
     if kind != "rpbh":  # Block-RHT / Full RHT: the same signs, no permutation
         perm = np.arange(d)
-    ref = codebooks(d, bits)
+    ref = codebooks(cb_d or d, bits)
     xs = inputs.bf16_bits_to_f64(X_bits[rows])
     if rounds > 1:
         R = orpbh.draw_rounds(seed, d, rounds)
@@ -105,6 +106,19 @@ def test_single_linear_workload_act_and_weight(oq, codebooks, bits):
     W = inputs.weights(1, inputs.T_W, 256, 256)
     _check_rows(oq, codebooks, X, 256, 64, bits)
     _check_rows(oq, codebooks, W, 256, 64, bits, weight=True)
+
+
+@pytest.mark.parametrize("bits", [4, 2])
+def test_single_linear_workload_block_codebook(oq, codebooks, bits):
+    # The single-linear workload's "4-bit codebook for d=64" read literally:
+    # C^(64,b), the block's dimension, on the same rows of width 256.  The rows
+    # are unit vectors either way, so the codes are well defined; they crowd
+    # into the middle cells (the codebook is built for wider coordinates).
+    X = inputs.activations(1, 64, 256)
+    W = inputs.weights(1, inputs.T_W, 256, 256)
+    got, _ = _check_rows(oq, codebooks, X, 256, 64, bits, cb_d=64)
+    _check_rows(oq, codebooks, W, 256, 64, bits, weight=True, cb_d=64)
+    assert len(np.unique(got)) >= 2
 
 
 @pytest.mark.parametrize("d,h", [(256, 64), (8960, 128), (1024, 1024), (512, 32), (1536, 512)])
