@@ -307,8 +307,7 @@ OQ_API int oq_linear(oq_rpbh_t r, oq_codebook_t cb_a, oq_codebook_t cb_w, const 
  *     already has the library's status word (any earlier launching call on
  *     the device, or oq_get_device_status(), creates it).
  *   - The first call on a device looks up the array's device address with
- *     cudaGetSymbolAddress (with that device current) and caches it; make
- *     that first call before any stream capture.
+ *     cudaGetSymbolAddress (with that device current) and caches it.
  *   - All calls share the one array, which keeps the last call's contents;
  *     nothing in it has to start at zero (the quantize kernel rewrites the
  *     codes and norms of all M rows before the GEMM reads them).  Calls that
