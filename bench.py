@@ -664,6 +664,60 @@ def _flush_and_time_many(fns, flush, steps, warmup):
     return [statistics.median(t) for t in times]
 
 
+def oracle_workload_sample(workload, rows):
+    """The oracle on `rows` tokens of a two-layer workload or the W3A3
+    projection, timed on the host cores (the cpu_baseline of the workload
+    lines).  Weights are quantized beforehand, untimed; the timed part is what
+    the GPU times: act-quant, linear (+ GELU, bf16 rounding of the hidden
+    layer, act-quant, linear).  Returns (seconds, flops of the sample)."""
+    from calibration_free_rotated_b200 import inputs
+    from oracle import codebook as ocb
+    from oracle import linear as olin
+    from oracle import quantize as oqz
+    from oracle import rpbh as orpbh
+    h = 128
+    f64 = inputs.bf16_bits_to_f64
+    if workload == "flux_qkv_w3a3":
+        d, N, b = 3072, 9216, 3
+        perm, signs = orpbh.draw_permutation_and_signs(0, d)
+        cb = ocb.lloyd_max(d, b)
+        cw, r16, _, _ = oqz.quantize_weight_rows(f64(inputs.weights(2, inputs.T_W, N, d)), perm, signs, h,
+                                                 cb["centroids"])
+        bias = f64(inputs.bias(2, N))
+        X = f64(inputs.activations(2, 4608, d, rows=(0, rows)))
+        t0 = time.perf_counter()
+        ca, s, _ = oqz.quantize_rows(X, perm, signs, h, cb["centroids"])
+        y = olin.linear_from_codes(ca, s, cw, r16, cb["centroids"], cb["centroids"], d, bias=bias)
+        dt = time.perf_counter() - t0
+        assert np.isfinite(y).all()
+        return dt, 2.0 * rows * N * d
+    wl, M, d1, d2, bw, ba = {"flux_mlp": (3, 4608, 3072, 12288, 2, 4),
+                             "wan_ffn": (4, 32760, 1536, 8960, 4, 6)}[workload]
+    p1, s1 = orpbh.draw_permutation_and_signs(0, d1)
+    p2, s2 = orpbh.draw_permutation_and_signs(0, d2)
+    ca1, cw1, ca2, cw2 = (ocb.lloyd_max(d1, ba)["centroids"], ocb.lloyd_max(d1, bw)["centroids"],
+                          ocb.lloyd_max(d2, ba)["centroids"], ocb.lloyd_max(d2, bw)["centroids"])
+    w1c, w1r, _, _ = oqz.quantize_weight_rows(f64(inputs.weights(wl, inputs.T_W, d2, d1)), p1, s1, h, cw1)
+    w2c, w2r, _, _ = oqz.quantize_weight_rows(f64(inputs.weights(wl, inputs.T_W2, d1, d2)), p2, s2, h, cw2)
+    X = f64(inputs.activations(wl, M, d1, rows=(0, rows)))
+    t0 = time.perf_counter()
+    a1, n1, _ = oqz.quantize_rows(X, p1, s1, h, ca1)
+    y1 = oqz.bf16_round(olin.linear_from_codes(a1, n1, w1c, w1r, ca1, cw1, d1, gelu=True))
+    a2, n2, _ = oqz.quantize_rows(y1, p2, s2, h, ca2)
+    y2 = olin.linear_from_codes(a2, n2, w2c, w2r, ca2, cw2, d2)
+    dt = time.perf_counter() - t0
+    assert np.isfinite(y2).all()
+    return dt, 4.0 * rows * d1 * d2
+
+
+def _workload_cpu_baseline(args, rows):
+    if getattr(args, "no_cpu_baseline", False):
+        return None
+    dt, flops = oracle_workload_sample(args.workload, rows)
+    return {"value": flops / dt / 1e12, "unit": "TFLOP/s", "cores": cpu_threads(), "kind": "oracle",
+            "sample": f"{rows} tokens through the timed launches; weights quantized beforehand, untimed"}
+
+
 def run_workload(args):
     """Per-kernel times of the two-layer workloads (one JSON line each; not the
     contract line).  flux_mlp: X[4608 x 3072] -> fc1 [12288 x 3072] + GELU ->
@@ -702,7 +756,8 @@ def run_workload(args):
                           "kernels": {"act_quant": {"ms": ms_q, "GB/s": gbs, "frac": gbs / peaks["hbm_gbs"]},
                                       "qkv": {"ms": ms_g, "TFLOP/s": tfs, "frac": tfs / peaks["bf16_tflops"]}},
                           "peak_source": src, "step_ms": ms_q + ms_g,
-                          "TFLOP/s": 2.0 * M * N * d / (ms_q + ms_g) / 1e9, "clocks": clk.summary()}), flush=True)
+                          "TFLOP/s": 2.0 * M * N * d / (ms_q + ms_g) / 1e9, "clocks": clk.summary(),
+                          "cpu_baseline": _workload_cpu_baseline(args, 2048)}), flush=True)
         return 0
     wl, M, d1, d2, bw, ba = {"flux_mlp": (3, 4608, 3072, 12288, 2, 4),
                              "wan_ffn": (4, 32760, 1536, 8960, 4, 6)}[args.workload]
@@ -761,6 +816,7 @@ def run_workload(args):
     out["step_ms_folded_permutation"] = folded
     out["TFLOP/s_folded_permutation"] = 4.0 * M * d1 * d2 / folded / 1e9
     out["clocks"] = clk.summary()
+    out["cpu_baseline"] = _workload_cpu_baseline(args, 1024)
     print(json.dumps(out), flush=True)
     return 0
 

@@ -71,3 +71,11 @@ def test_sweep_rotation_equals_the_oracle(d, h, rounds):
     got = bench.rotate_rows_f64(torch.from_numpy(X), tables, h).numpy()
     ref = rpbh.rotate_composed(X, R, h)
     assert np.allclose(got, ref, rtol=0, atol=1e-12)
+
+
+def test_workload_cpu_baseline_runs_the_oracle_chain():
+    # the oracle leg of `bench.py --workload`: a bounded sample through the same
+    # launches the GPU times, with the weights quantized beforehand
+    import bench
+    dt, flops = bench.oracle_workload_sample("flux_qkv_w3a3", 4)
+    assert dt > 0 and flops == 2.0 * 4 * 9216 * 3072
