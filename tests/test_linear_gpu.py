@@ -127,6 +127,23 @@ def test_codes_gemm_small_ragged(oq, codebooks, ba, bw):
     assert _rel_fro(y, ref) <= TOL
 
 
+@pytest.mark.parametrize("M,N,d,ba,bw", [(1, 16, 64, 4, 4), (1, 16, 64, 6, 2), (128, 256, 64, 4, 4),
+                                          (129, 16, 128, 4, 4), (257, 272, 192, 2, 4), (3, 48, 256, 3, 3)])
+def test_codes_gemm_degenerate_shapes(oq, codebooks, M, N, d, ba, bw):
+    # the smallest shapes the GEMM accepts (one row, N = 16, K = 64), the
+    # largest single-CTA M (128) and the first CTA-pair M (129, one pair with
+    # 127 empty rows), and tails in every dimension
+    h = 64
+    rng = np.random.default_rng(M * 7 + N)
+    X = inputs.to_bf16_bits(rng.standard_normal((M, d)))
+    W = inputs.to_bf16_bits(rng.standard_normal((N, d)) * 0.02)
+    ca, s = _oracle_act(codebooks, X, d, h, ba)
+    cw, r16 = _oracle_weight(codebooks, W, d, h, bw)
+    y, _, ref = _run_codes(oq, codebooks, ca, s, cw, r16, d, ba, bw)
+    assert y.shape == (M, N)
+    assert _rel_fro(y, ref) <= TOL
+
+
 def test_codes_gemm_single_linear_workload(oq, codebooks):
     # X[64 x 256] (3 outlier channels x20), W[256 x 256]; block 64; W4A4
     d, h = 256, 64

@@ -175,6 +175,14 @@ def test_edge_rows(oq, codebooks):
     _check_rows(oq, codebooks, X, d, h, 4, weight=True)
 
 
+@pytest.mark.parametrize("d,h,bits", [(64, 64, 4), (3072, 128, 4), (8960, 128, 6), (16384, 256, 2)])
+def test_single_row(oq, codebooks, d, h, bits):
+    # M = 1 in each row-width configuration of the kernel (one CTA, half a pair)
+    X = inputs.to_bf16_bits(np.random.default_rng(d).standard_normal((1, d)))
+    _check_rows(oq, codebooks, X, d, h, bits)
+    _check_rows(oq, codebooks, X, d, h, bits, weight=True)
+
+
 def test_empty_batch(oq):
     r, cb = _lib_handles(oq, 0, 256, 64, 4)
     X = torch.empty((0, 256), dtype=torch.bfloat16, device="cuda")
