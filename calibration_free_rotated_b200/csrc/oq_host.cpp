@@ -495,72 +495,187 @@ static uint32_t xch_output_reg(uint32_t c, uint32_t L) {  // the register that h
   return R * ((i / R) ^ l) + i % R;
 }
 
-int rpbh_composed_tables(oq_rpbh_t r, const uint16_t** slots, const uint32_t** signs, bool xch) {
+// Splits the edges `ids` of a bipartite multigraph in which every vertex has
+// an even number of them into two halves that give every vertex half of its
+// edges each (bit[e] = 0 or 1): closed walks over unused edges, labelled
+// alternately.  A closed walk in a bipartite graph has even length, so every
+// pass through a vertex, the start included, uses one edge of each label.
+static void euler_split(int nv, const std::vector<std::pair<int, int>>& E, const std::vector<int>& ids,
+                        std::vector<uint8_t>& bit) {
+  std::vector<std::vector<int>> adj((size_t)nv);
+  for (int e : ids) {
+    adj[(size_t)E[e].first].push_back(e);
+    adj[(size_t)E[e].second].push_back(e);
+  }
+  std::vector<uint8_t> used(E.size(), 0);
+  std::vector<size_t> next((size_t)nv, 0);
+  auto take = [&](int x) -> int {  // an unused edge at x, or -1
+    auto& a = adj[(size_t)x];
+    size_t& i = next[(size_t)x];
+    while (i < a.size() && used[(size_t)a[i]]) ++i;
+    return i < a.size() ? a[i] : -1;
+  };
+  for (int s = 0; s < nv; ++s) {
+    while (take(s) >= 0) {
+      int cur = s;
+      uint8_t label = 0;
+      for (int e = take(cur); e >= 0; e = take(cur)) {
+        used[(size_t)e] = 1;
+        bit[(size_t)e] = label;
+        label ^= 1u;
+        cur = E[e].first == cur ? E[e].second : E[e].first;
+      }
+    }
+  }
+}
+
+// Shared-memory layout of one round's output for the composed kernel, free of
+// bank conflicts on both sides.  Coordinate c is stored by one register of
+// one thread (the store group: half-warp and register) and gathered by one
+// register of one thread of the next round (the load group); each group is
+// at most 16 lanes.  An 8-byte slot s sits on bank pair s mod 16, so a group
+// whose 16 slots fall on 16 different bank pairs moves in the minimum two
+// wavefronts.  Colouring the bipartite (store group, load group) multigraph
+// with 16 colours, one per bank pair, such that no group repeats a colour is
+// an edge colouring of a graph of degree 16, which always exists (Konig);
+// padded with dummy edges to exactly degree 16, four levels of Euler splits
+// find one.  Returns sigma[c], the slot of coordinate c, all below 32 * TP.
+static std::vector<uint16_t> conflict_free_layout(int d, const std::vector<uint32_t>& store_group,
+                                                  const std::vector<uint32_t>& load_group, int ngroups) {
+  std::vector<std::pair<int, int>> E;  // vertices: store groups 0.., load groups ngroups..
+  E.reserve((size_t)ngroups * 16);
+  std::vector<int> ds((size_t)ngroups, 0), dl((size_t)ngroups, 0);
+  for (int c = 0; c < d; ++c) {
+    E.emplace_back((int)store_group[(size_t)c], ngroups + (int)load_group[(size_t)c]);
+    ++ds[store_group[(size_t)c]];
+    ++dl[load_group[(size_t)c]];
+  }
+  // pad to degree 16 (both sides miss the same number of edges)
+  for (int u = 0, v = 0; u < ngroups; ++u) {
+    while (ds[(size_t)u] < 16) {
+      while (dl[(size_t)v] >= 16) ++v;
+      E.emplace_back(u, ngroups + v);
+      ++ds[(size_t)u];
+      ++dl[(size_t)v];
+    }
+  }
+  std::vector<uint8_t> colour(E.size(), 0), bit(E.size(), 0);
+  std::vector<std::vector<int>> classes(1);
+  for (size_t e = 0; e < E.size(); ++e) classes[0].push_back((int)e);
+  for (int level = 0; level < 4; ++level) {
+    std::vector<std::vector<int>> split;
+    for (const auto& ids : classes) {
+      euler_split(2 * ngroups, E, ids, bit);
+      std::vector<int> a, b;
+      for (int e : ids) {
+        (bit[(size_t)e] ? b : a).push_back(e);
+        colour[(size_t)e] = (uint8_t)(colour[(size_t)e] | (bit[(size_t)e] << level));
+      }
+      split.push_back(std::move(a));
+      split.push_back(std::move(b));
+    }
+    classes.swap(split);
+  }
+  std::vector<uint16_t> sigma((size_t)d);
+  int fill[16] = {};
+  for (int c = 0; c < d; ++c) {
+    const int k = colour[(size_t)c];
+    sigma[(size_t)c] = (uint16_t)(16 * fill[k]++ + k);
+  }
+  return sigma;
+}
+
+// The composed kernel's tables for one register order (coordinate order, or
+// the block-transposed layout's):
+//   gather[k][32 g + r]: the slot register r of thread g reads in round k
+//                        (round 1: the interleaved bf16 pair words; later
+//                        rounds: where the previous round stored it);
+//   store[k][32 g + r]:  the slot it stores its output to (rounds before the last);
+//   signs[k][g]:         bit r = the sign of the coordinate register r gathers.
+static void build_composed_tables(const oq_rpbh_s* r, bool xch, std::vector<uint16_t>& gather,
+                                  std::vector<uint16_t>& store, std::vector<uint32_t>& signs) {
+  const int d = r->d, T = d / 32, words = (d + 31) / 32, rounds = r->rounds;
+  const uint32_t L = (uint32_t)r->h / 32u, R = xch ? 32u / L : 32u;
+  gather.assign((size_t)rounds * d, 0);
+  store.assign((size_t)rounds * d, 0);
+  signs.assign((size_t)rounds * words, 0u);
+  auto in_j = [&](uint32_t g, uint32_t reg) { return xch ? xch_gather_coord(g, reg, L) : 32u * g + reg; };
+  auto out_c = [&](uint32_t g, uint32_t reg) {
+    return xch ? 32u * g + R * ((reg / R) ^ (g & (L - 1u))) + reg % R : 32u * g + reg;
+  };
+  const int ngroups = ((T + 15) / 16) * 32;  // (half-warp, register)
+  std::vector<uint16_t> sigma;  // slots of the previous round's output
+  for (int k = 0; k < rounds; ++k) {
+    const int32_t* perm = k == 0 ? r->perm.data() : r->perm_more.data() + (size_t)(k - 1) * d;
+    const uint32_t* bits = k == 0 ? r->sign_bits.data() : r->sign_bits_more.data() + (size_t)(k - 1) * words;
+    for (uint32_t g = 0; g < (uint32_t)T; ++g) {
+      for (uint32_t reg = 0; reg < 32u; ++reg) {
+        const uint32_t j = in_j(g, reg), c = (uint32_t)perm[j];
+        gather[(size_t)k * d + 32u * g + reg] = k == 0 ? composed_slot(c, true) : sigma[c];
+        if ((bits[j >> 5] >> (j & 31u)) & 1u) signs[(size_t)k * words + g] |= 1u << reg;
+      }
+    }
+    if (k + 1 == rounds) break;
+    // this round's output layout, chosen against the next round's gathers
+    const int32_t* pnext = r->perm_more.data() + (size_t)k * d;
+    std::vector<uint32_t> sgrp((size_t)d), lgrp((size_t)d);
+    for (uint32_t g = 0; g < (uint32_t)T; ++g)
+      for (uint32_t reg = 0; reg < 32u; ++reg) {
+        sgrp[out_c(g, reg)] = (g >> 4) * 32u + reg;
+        lgrp[(uint32_t)pnext[in_j(g, reg)]] = (g >> 4) * 32u + reg;
+      }
+    sigma = conflict_free_layout(d, sgrp, lgrp, ngroups);
+    for (uint32_t g = 0; g < (uint32_t)T; ++g)
+      for (uint32_t reg = 0; reg < 32u; ++reg) store[(size_t)k * d + 32u * g + reg] = sigma[out_c(g, reg)];
+  }
+}
+
+int rpbh_composed_tables(oq_rpbh_t r, const uint16_t** slots, const uint16_t** store, const uint32_t** signs,
+                         bool xch) {
   int dev;
   if (int rc = current_device(&dev)) return rc;
   const uint32_t L = (uint32_t)r->h / 32u;
   const bool xch_ok = L >= 2 && L <= 8 && r->d % 32 == 0;
   if (xch && !xch_ok) return fail(OQ_ERR_UNSUPPORTED, "no block-transposed layout for block %d", r->h);
   std::lock_guard<std::mutex> lk(r->mu);
-  if (!r->dev_slots[dev]) {
-    const int d = r->d, words = (d + 31) / 32;
-    std::vector<uint16_t> sl((size_t)r->rounds * d), xsl(xch_ok ? (size_t)r->rounds * d : 0);
-    std::vector<uint32_t> sg((size_t)r->rounds * words), xsg(xch_ok ? (size_t)r->rounds * words : 0, 0u);
-    for (int k = 0; k < r->rounds; ++k) {
-      const int32_t* perm = k == 0 ? r->perm.data() : r->perm_more.data() + (size_t)(k - 1) * d;
-      const uint32_t* bits = k == 0 ? r->sign_bits.data() : r->sign_bits_more.data() + (size_t)(k - 1) * words;
-      for (int j = 0; j < d; ++j) sl[(size_t)k * d + j] = composed_slot((uint32_t)perm[j], k == 0);
-      std::memcpy(sg.data() + (size_t)k * words, bits, sizeof(uint32_t) * words);
-      if (!xch_ok) continue;
-      for (uint32_t g = 0; g < (uint32_t)d / 32u; ++g) {
-        for (uint32_t reg = 0; reg < 32u; ++reg) {
-          const uint32_t j = xch_gather_coord(g, reg, L);
-          const uint32_t c = (uint32_t)perm[j];  // the input coordinate this register reads
-          uint16_t slot;
-          if (k == 0) {
-            slot = composed_slot(c, true);      // round 1: the pair words, in coordinate order
-          } else {                              // later rounds: where the previous round stored c
-            slot = composed_slot((c & ~31u) | xch_output_reg(c, L), false);
-          }
-          xsl[(size_t)k * d + 32u * g + reg] = slot;
-          if ((bits[j >> 5] >> (j & 31u)) & 1u) xsg[(size_t)k * words + g] |= 1u << reg;
+  if (!r->dev_ctab[0][dev]) {  // both register orders at once, so no later launch allocates
+    for (int v = 0; v < (xch_ok ? 2 : 1); ++v) {
+      std::vector<uint16_t> gather, st;
+      std::vector<uint32_t> sg;
+      build_composed_tables(r, v == 1, gather, st, sg);
+      // one allocation: gather slots, store slots, sign words
+      const size_t nslot = gather.size(), bytes = sizeof(uint16_t) * 2 * nslot + sizeof(uint32_t) * sg.size();
+      unsigned char* dbuf = nullptr;
+      cudaError_t e = dev_malloc(reinterpret_cast<void**>(&dbuf), bytes);
+      if (e == cudaSuccess) e = cudaMemcpy(dbuf, gather.data(), sizeof(uint16_t) * nslot, cudaMemcpyHostToDevice);
+      if (e == cudaSuccess)
+        e = cudaMemcpy(dbuf + sizeof(uint16_t) * nslot, st.data(), sizeof(uint16_t) * nslot, cudaMemcpyHostToDevice);
+      if (e == cudaSuccess)
+        e = cudaMemcpy(dbuf + sizeof(uint16_t) * 2 * nslot, sg.data(), sizeof(uint32_t) * sg.size(),
+                       cudaMemcpyHostToDevice);
+      if (e != cudaSuccess) {
+        cudaFree(dbuf);
+        if (v == 1) {  // keep the pair all-or-nothing
+          cudaFree(r->dev_ctab[0][dev]);
+          r->dev_ctab[0][dev] = nullptr;
         }
+        return fail(OQ_ERR_CUDA, "uploading composed rotation tables: %s", cudaGetErrorString(e));
       }
+      r->dev_ctab[v][dev] = dbuf;
     }
-    uint16_t *dsl = nullptr, *dxsl = nullptr;
-    uint32_t *dsg = nullptr, *dxsg = nullptr;
-    cudaError_t e = dev_malloc(reinterpret_cast<void**>(&dsl), sizeof(uint16_t) * sl.size());
-    if (e == cudaSuccess) e = dev_malloc(reinterpret_cast<void**>(&dsg), sizeof(uint32_t) * sg.size());
-    if (e == cudaSuccess) e = cudaMemcpy(dsl, sl.data(), sizeof(uint16_t) * sl.size(), cudaMemcpyHostToDevice);
-    if (e == cudaSuccess) e = cudaMemcpy(dsg, sg.data(), sizeof(uint32_t) * sg.size(), cudaMemcpyHostToDevice);
-    if (e == cudaSuccess && xch_ok) {
-      e = dev_malloc(reinterpret_cast<void**>(&dxsl), sizeof(uint16_t) * xsl.size());
-      if (e == cudaSuccess) e = dev_malloc(reinterpret_cast<void**>(&dxsg), sizeof(uint32_t) * xsg.size());
-      if (e == cudaSuccess)
-        e = cudaMemcpy(dxsl, xsl.data(), sizeof(uint16_t) * xsl.size(), cudaMemcpyHostToDevice);
-      if (e == cudaSuccess)
-        e = cudaMemcpy(dxsg, xsg.data(), sizeof(uint32_t) * xsg.size(), cudaMemcpyHostToDevice);
-    }
-    if (e != cudaSuccess) {
-      cudaFree(dsl);
-      cudaFree(dsg);
-      cudaFree(dxsl);
-      cudaFree(dxsg);
-      return fail(OQ_ERR_CUDA, "uploading composed rotation tables: %s", cudaGetErrorString(e));
-    }
-    r->dev_slots[dev] = dsl;
-    r->dev_csigns[dev] = dsg;
-    r->dev_xslots[dev] = dxsl;
-    r->dev_xcsigns[dev] = dxsg;
   }
-  *slots = xch ? r->dev_xslots[dev] : r->dev_slots[dev];
-  *signs = xch ? r->dev_xcsigns[dev] : r->dev_csigns[dev];
+  const int v = xch ? 1 : 0;
+  const size_t nslot = (size_t)r->rounds * r->d;
+  unsigned char* base = r->dev_ctab[v][dev];
+  *slots = reinterpret_cast<const uint16_t*>(base);
+  *store = reinterpret_cast<const uint16_t*>(base + sizeof(uint16_t) * nslot);
+  *signs = reinterpret_cast<const uint32_t*>(base + sizeof(uint16_t) * 2 * nslot);
   return OQ_OK;
 }
 
 int rpbh_tables_if_present(oq_rpbh_t r, int dev) {
   std::lock_guard<std::mutex> lk(r->mu);
-  return r->dev_perm[dev] && (r->rounds == 1 || r->dev_slots[dev]) ? OQ_OK : OQ_ERR_ARG;
+  return r->dev_perm[dev] && (r->rounds == 1 || r->dev_ctab[0][dev]) ? OQ_OK : OQ_ERR_ARG;
 }
 
 int codebook_qtable_if_present(oq_codebook_t cb, int dev) {
@@ -657,9 +772,9 @@ static int make_rotation(uint64_t seed, int d, int block, int kind, int rounds, 
         return rc;
       }
       if (rounds > 1) {
-        const uint16_t* sl;
+        const uint16_t *sl, *st;
         const uint32_t* sg;
-        if (int rc = rpbh_composed_tables(r, &sl, &sg)) {
+        if (int rc = rpbh_composed_tables(r, &sl, &st, &sg)) {
           oq_free_rpbh(r);
           return rc;
         }
@@ -711,6 +826,24 @@ static int finish(int rc, void* stream) {
 int oq_set_debug(int on) {
   clear_error();
   g_debug.store(on ? 1 : 0);
+  return OQ_OK;
+}
+
+int oq_test_composed_tables(oq_rpbh_t r, int xch, uint16_t* gather, uint16_t* store, uint32_t* signs) {
+  clear_error();
+  if (!r || !gather || !store || !signs) return fail(OQ_ERR_ARG, "NULL argument");
+  if (r->rounds < 2) return fail(OQ_ERR_ARG, "not a composed rotation");
+  const uint32_t L = (uint32_t)r->h / 32u;
+  if (xch && !(L >= 2 && L <= 8)) return fail(OQ_ERR_UNSUPPORTED, "no block-transposed layout for block %d", r->h);
+  std::vector<uint16_t> g, st;
+  std::vector<uint32_t> sg;
+  {
+    std::lock_guard<std::mutex> lk(r->mu);
+    build_composed_tables(r, xch != 0, g, st, sg);
+  }
+  std::memcpy(gather, g.data(), sizeof(uint16_t) * g.size());
+  std::memcpy(store, st.data(), sizeof(uint16_t) * st.size());
+  std::memcpy(signs, sg.data(), sizeof(uint32_t) * sg.size());
   return OQ_OK;
 }
 
@@ -802,14 +935,12 @@ void oq_free_rpbh(oq_rpbh_t r) {
   int prev = -1;
   bool have_prev = cudaGetDevice(&prev) == cudaSuccess;
   for (int dev = 0; dev < OQ_MAX_DEVICES; ++dev) {
-    if (!r->dev_perm[dev] && !r->dev_signs[dev] && !r->dev_slots[dev] && !r->dev_csigns[dev]) continue;
+    if (!r->dev_perm[dev] && !r->dev_signs[dev] && !r->dev_ctab[0][dev] && !r->dev_ctab[1][dev]) continue;
     if (cudaSetDevice(dev) == cudaSuccess) {
       cudaFree(r->dev_perm[dev]);
       cudaFree(r->dev_signs[dev]);
-      cudaFree(r->dev_slots[dev]);
-      cudaFree(r->dev_csigns[dev]);
-      cudaFree(r->dev_xslots[dev]);
-      cudaFree(r->dev_xcsigns[dev]);
+      cudaFree(r->dev_ctab[0][dev]);
+      cudaFree(r->dev_ctab[1][dev]);
     }
   }
   if (have_prev) cudaSetDevice(prev);

@@ -24,12 +24,10 @@ struct oq_rpbh_s {
   std::mutex mu;
   uint16_t* dev_perm[OQ_MAX_DEVICES] = {};   // pi as uint16 [d]
   uint32_t* dev_signs[OQ_MAX_DEVICES] = {};  // sign words [d/32]
-  uint16_t* dev_slots[OQ_MAX_DEVICES] = {};  // composed kernel: [rounds][d] shared-memory slots
-  uint32_t* dev_csigns[OQ_MAX_DEVICES] = {};  // composed kernel: [rounds][d/32] sign words
-  // The same for the block-transposed FWHT (blocks of 64..256): slots and sign
-  // bits in each thread's register order instead of coordinate order.
-  uint16_t* dev_xslots[OQ_MAX_DEVICES] = {};
-  uint32_t* dev_xcsigns[OQ_MAX_DEVICES] = {};
+  // composed kernel, per register order (0: coordinate order, 1: the
+  // block-transposed layout's): gather slots uint16[rounds][d], store slots
+  // uint16[rounds][d], sign words uint32[rounds][d/32], in one allocation
+  unsigned char* dev_ctab[2][OQ_MAX_DEVICES] = {};
 };
 
 struct oq_codebook_s {
@@ -63,8 +61,10 @@ uint16_t double_to_fp16_rne(double v);
 int current_device(int* dev);
 int rpbh_device_tables(oq_rpbh_t r, const uint16_t** perm, const uint32_t** signs);
 // Tables of the composed kernel: coordinate order, or (xch) the register order
-// of the block-transposed FWHT (OQ_ERR_UNSUPPORTED when the block has none).
-int rpbh_composed_tables(oq_rpbh_t r, const uint16_t** slots, const uint32_t** signs, bool xch = false);
+// of the block-transposed FWHT (OQ_ERR_UNSUPPORTED when the block has none):
+// gather slots, store slots (rounds before the last) and sign words.
+int rpbh_composed_tables(oq_rpbh_t r, const uint16_t** slots, const uint16_t** store, const uint32_t** signs,
+                         bool xch = false);
 int codebook_device_qtable(oq_codebook_t cb, const uint32_t** qtable);
 void build_qtable(oq_codebook_t cb);
 int device_status_word(int** status);

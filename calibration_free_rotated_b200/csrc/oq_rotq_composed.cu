@@ -22,11 +22,14 @@
 //     thread index, so the 128-bit writes are free of bank conflicts;
 //   * round 1 gathers those words (one 32-bit load feeds both rows) and widens
 //     them to f32 while flipping its signs; later rounds gather f32 pairs from
-//     a shared array F of d 8-byte slots (256-byte runs, rotated the same
-//     way), which the previous round wrote between two CTA barriers; each
-//     round reads through a table of precomputed slot indices (the
-//     permutation composed with the chunk rotation) and runs the unnormalised
-//     block transform in registers;
+//     a shared array F of 8-byte slots, which the previous round wrote between
+//     two CTA barriers; each round reads through a table of precomputed slot
+//     indices and runs the unnormalised block transform in registers;
+//   * where a round stores each coordinate is chosen on the host (a table of
+//     store slots): every half-warp's store of one register, and the next
+//     round's gather of it, fall on 16 different bank pairs (an edge colouring
+//     of the store-group / gather-group graph), so both move in the minimum
+//     two wavefronts instead of conflicting at random;
 //   * the sum of squares comes from round 1's gathered input (the rotation is
 //     orthogonal); the k factors sqrt(h) of the unnormalised transforms are
 //     folded into the search multiplier;
@@ -52,7 +55,8 @@ struct ComposedArgs {
   uint8_t* codes;
   float* norm_f32;
   uint16_t* norm_bf16;
-  const uint16_t* slots;  // [rounds][d]: slot that round r's coordinate j reads (round 1: 4-byte words)
+  const uint16_t* slots;  // [rounds][d]: slot that round r's register reads (round 1: 4-byte words)
+  const uint16_t* store;  // [rounds][d]: slot that round r's register is stored to (rounds before the last)
   const uint32_t* signs;  // [rounds][d / 32]: sign words
   const uint32_t* qtable;
   int* status;
@@ -68,15 +72,21 @@ __device__ __forceinline__ unsigned long long lds_u64(uint32_t addr) {
   return v;
 }
 
-// Writes the 32 f32 pairs of this thread to its 256-byte run of F (chunk c of
-// the run at position c ^ (g & 15)).
-__device__ __forceinline__ void store_run(uint32_t run, uint32_t rot, const unsigned long long (&v)[32]) {
+// Writes the 32 f32 pairs of this thread to their 8-byte slots of F, from its
+// 32 store-slot indices (16-bit each, four 128-bit words).
+__device__ __forceinline__ void store_round(uint32_t fbase, const uint4* st, const unsigned long long (&v)[32]) {
 #pragma unroll
-  for (int c = 0; c < 16; ++c) {
-    uint32_t a0, b0, a1, b1;
-    u2_unpack(v[2 * c], a0, b0);
-    u2_unpack(v[2 * c + 1], a1, b1);
-    sts_u128(run + ((((uint32_t)c) ^ rot) << 4), a0, b0, a1, b1);
+  for (int q = 0; q < 4; ++q) {
+    const uint4 S = st[q];
+    const uint32_t s4[4] = {S.x, S.y, S.z, S.w};
+#pragma unroll
+    for (int m = 0; m < 8; ++m) {
+      const int i = 8 * q + m;
+      const uint32_t slot = (s4[m >> 1] >> (16 * (m & 1))) & 0xFFFFu;
+      uint32_t lo, hi;
+      u2_unpack(v[i], lo, hi);
+      asm volatile("st.shared.v2.b32 [%0], {%1, %2};" ::"r"(fbase + 8u * slot), "r"(lo), "r"(hi) : "memory");
+    }
   }
 }
 
@@ -142,7 +152,6 @@ __global__ void __launch_bounds__(512, 1) rotq_composed_kernel(const __grid_cons
   float2* part = reinterpret_cast<float2*>(smem + a.part_off);
   for (int i = tid; i < a.qtable_len; i += blockDim.x) qtab[i] = a.qtable[i];
   const uint32_t qkey = smem_u32(qtab) - 0x2D000000u;  // = qtab - 4 * bits(1.5 * 2^23)
-  const uint32_t run = fbase + 256u * (uint32_t)tid, rot = (uint32_t)tid & 15u;
   const int nwarps = blockDim.x >> 5;
   const uint32_t rowb = (uint32_t)a.d * 2u;  // bytes of a bf16 row
   const uint32_t ring = fbase + a.ring_off, bars = fbase + a.bar_off;
@@ -220,7 +229,7 @@ __global__ void __launch_bounds__(512, 1) rotq_composed_kernel(const __grid_cons
         fwht_pairs<LOGHB>(v, lane);
       if (r + 1 < a.rounds) {
         __syncthreads();  // every thread has gathered this round's input
-        if (active) store_run(run, rot, v);
+        if (active) store_round(fbase, reinterpret_cast<const uint4*>(a.store + (size_t)r * a.d) + 4 * tid, v);
         __syncthreads();
       }
     }
@@ -338,9 +347,9 @@ int launch_rotq_composed(oq_rpbh_t r, oq_codebook_t cb, const void* X, int M, ui
   if (qlen > 4097) return fail(OQ_ERR_UNSUPPORTED, "codebook d=%d bits=%d needs a %d-entry search table", cb->d, bits, qlen);
   rotq::ComposedFn kern = rotq::pick_composed(bits, loghb);
   if (!kern) return fail(OQ_ERR_UNSUPPORTED, "no composed rotate+quantize kernel for bits=%d h=%d", bits, h);
-  const uint16_t* slots;
+  const uint16_t *slots, *store;
   const uint32_t* signs;
-  if (int rc = rpbh_composed_tables(r, &slots, &signs, rotq::composed_xch(bits, loghb))) return rc;
+  if (int rc = rpbh_composed_tables(r, &slots, &store, &signs, rotq::composed_xch(bits, loghb))) return rc;
   const uint32_t* qtable;
   if (int rc = codebook_device_qtable(cb, &qtable)) return rc;
   int nsm;
@@ -354,6 +363,7 @@ int launch_rotq_composed(oq_rpbh_t r, oq_codebook_t cb, const void* X, int M, ui
   a.norm_f32 = norm_f32;
   a.norm_bf16 = norm_bf16;
   a.slots = slots;
+  a.store = store;
   a.signs = signs;
   a.qtable = qtable;
   a.M = M;
@@ -364,7 +374,7 @@ int launch_rotq_composed(oq_rpbh_t r, oq_codebook_t cb, const void* X, int M, ui
   int* status;
   if (int rc = device_status_word(&status)) return rc;
   a.status = status;
-  a.qt_off = (uint32_t)threads * 256u;  // F: one 256-byte run per thread (round 1 uses the first half)
+  a.qt_off = (uint32_t)threads * 256u;  // F: 32 8-byte slots per thread (round 1 uses the first half as words)
   a.part_off = (a.qt_off + 4u * (uint32_t)qlen + 15u) & ~15u;
   a.bar_off = (a.part_off + (uint32_t)(threads / 32) * 8u + 15u) & ~15u;
   a.ring_off = (a.bar_off + 16u + 127u) & ~127u;

@@ -55,6 +55,7 @@ _SIGS = {
                            _c_void_p, _c_int, _c_void_p, _c_void_p, _c_void_p, _c_size_t, _c_void_p]),
     "oq_linear_noalloc": (_c_int, [_c_void_p, _c_void_p, _c_void_p, _c_void_p, _c_int, _c_void_p, _c_void_p,
                                    _c_int, _c_void_p, _c_int, _c_void_p, _c_void_p, _c_void_p]),
+    "oq_test_composed_tables": (_c_int, [_c_void_p, _c_int, _c_void_p, _c_void_p, _c_void_p]),
 }
 NOALLOC_SCRATCH_BYTES = 32 << 20
 for _name, (_res, _args) in _SIGS.items():

@@ -98,6 +98,21 @@ OQ_API int oq_set_debug(int on);
  * Errors: OQ_ERR_ARG for a kernel outside 0..2. */
 OQ_API int oq_test_stall_next(int kernel);
 
+/* Test hook (host only, no device needed): the composed-rotation kernel's
+ * tables for handle r (rounds >= 2), as the library builds them, for the
+ * coordinate register order (xch = 0) or the block-transposed one (xch = 1,
+ * blocks of 64..256):
+ *   gather : uint16 [rounds][d]   slot that register r of thread g reads in
+ *                                 round k, at [k][32 g + r] (round 1: 4-byte
+ *                                 bf16 pair words; later rounds: 8-byte slots);
+ *   store  : uint16 [rounds][d]   slot it stores its output to in round k
+ *                                 (rounds before the last; the last is 0);
+ *   signs  : uint32 [rounds][d/32] bit r of word [k][g]: the sign of the
+ *                                 coordinate register r of thread g gathers.
+ * Buffers are caller-owned host arrays of those sizes.  Errors: OQ_ERR_ARG
+ * (NULL, one-round handle), OQ_ERR_UNSUPPORTED (xch for another block). */
+OQ_API int oq_test_composed_tables(oq_rpbh_t r, int xch, uint16_t* gather, uint16_t* store, uint32_t* signs);
+
 /* ---------------------------------------------------------------------------
  * RPBH rotation  Pi_d = blkdiag(H_h D_1, ..., H_h D_{d/h}) P_pi
  * [OQ] Methodology, "Randomized Permuted Block-Hadamard (RPBH) Rotation".
